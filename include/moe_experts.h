@@ -1,0 +1,80 @@
+/*
+ * moe_experts.h -- the routed experts and the shared expert.
+ *
+ * Every expert is a bias-free SwiGLU MLP, w2(silu(w1 x) * w3 x) with
+ * silu(a) = a * sigmoid(a): the pages print only the constructor
+ * Expert(dim, moe_inter_dim) (moe-init excerpt of "DeepSeek-V3.2-Exp ·
+ * Mixture of experts"), and three bias-free [inter, dim] / [dim, inter]
+ * matrices match the per-expert count 3 * 7168 * 2048 = 44,040,192 of that
+ * page's "Exact per-instance accounting" table.  The shared expert (MLP of
+ * n_shared * moe_inter_dim features) is applied to every token.
+ *
+ * Computes, for the rows that moe_dispatch_build grouped by expert:
+ *   h[p,:]   = round_act(silu(x[t] w1_e^T) * (x[t] w3_e^T))  t = sorted_token[p]
+ *   out_perm[p,:]   = h[p,:] w2_e^T           p in [offsets[e], offsets[e+1])
+ *   out_shared[t,:] = same expert on x[t] with the shared weights, every t
+ * Accumulation is fp32; h is rounded once to the activation dtype (it is the
+ * second matmul's operand); outputs are fp32 and not yet multiplied by the
+ * gates (moe_combine applies them, as the excerpt multiplies the expert's
+ * output by the weight before adding it into y).  Experts with no rows
+ * launch no work (the excerpt skips them).
+ */
+#ifndef MOE_EXPERTS_H
+#define MOE_EXPERTS_H
+#include "moe_common.h"
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/*
+ * Weights of all n_routed + n_shared experts, stacked: routed experts
+ * 0 .. n_routed-1, then the shared expert(s).
+ *   w1, w3  [n_routed + n_shared, inter, dim]
+ *   w2      [n_routed + n_shared, dim, inter]
+ *   w_dt    MOE_BF16, MOE_F32 or MOE_E4M3
+ *   s1, s3  [n_routed + n_shared, inter/128, dim/128] fp32 (MOE_E4M3 only)
+ *   s2      [n_routed + n_shared, dim/128, inter/128] fp32 (MOE_E4M3 only)
+ * For MOE_E4M3 the weight is value(q) * scale of its 128 x 128 block.
+ */
+typedef struct {
+  const void *w1, *w3, *w2;
+  moe_dtype w_dt;
+  const float *s1, *s3, *s2;
+} moe_expert_weights;
+
+/* Bytes of device workspace moe_experts_forward needs. */
+size_t moe_experts_workspace_size(const moe_cfg *cfg, int64_t T, moe_dtype x_dt,
+                                  moe_dtype w_dt);
+
+/*
+ * x            [T, dim], x_dt = MOE_BF16 or MOE_F32
+ * offsets      [n_routed + 1] int32 from moe_dispatch_build
+ * sorted_token [T * topk] int32 from moe_dispatch_build
+ * out_perm     [T * topk, dim] fp32 out, row p = expert output of row p
+ * out_shared   [T, dim] fp32 out (may be NULL when n_shared == 0)
+ * Paths: bf16 activations with bf16 or e4m3 weights run on the tcgen05
+ * tensor cores (dim % 128 == 0, inter % 128 == 0); any other combination
+ * (fp32 activations or weights) runs on the CUDA cores in fp32.
+ * Limits: n_shared <= 1, T * topk < 2^31.
+ * Device errors: MOE_ERR_TIMEOUT if a pipeline wait expired (the kernel then
+ * stops early; outputs are unspecified).
+ */
+moe_status moe_experts_forward(const moe_cfg *cfg, int64_t T, const void *x, moe_dtype x_dt,
+                               const moe_expert_weights *w, const int32_t *offsets,
+                               const int32_t *sorted_token, float *out_perm, float *out_shared,
+                               void *ws, size_t ws_bytes, int32_t *dev_status,
+                               moe_stream_t stream);
+
+/*
+ * Self-test of the bounded pipeline wait used by the tensor-core kernels:
+ * one CTA waits on a barrier that nothing signals, with a limit of
+ * `limit_ns` nanoseconds, then writes MOE_ERR_TIMEOUT to dev_status and
+ * returns.  The context stays usable.  limit_ns must be in (0, 2e9].
+ */
+moe_status moe_experts_selftest_wait(int64_t limit_ns, int32_t *dev_status,
+                                     moe_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif

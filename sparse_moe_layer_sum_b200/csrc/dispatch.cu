@@ -1,0 +1,167 @@
+// moe_dispatch: per-expert histogram, exclusive scan and stable scatter.
+//
+// Restates, for all experts at once and without a host round trip, what the
+// moe-forward code excerpt of "DeepSeek-V3.2-Exp · Mixture of experts" does
+// with torch.bincount(indices) and, per expert, torch.where(indices == i):
+// every expert's (token, slot) pairs, tokens ascending.
+//
+// The pairs are cut into chunks of CHUNK_TOKENS tokens:
+//  1. dispatch_hist:    per-chunk expert histograms (shared-memory atomics).
+//  2. dispatch_scan:    per expert, an exclusive scan over chunks; then an
+//                       exclusive scan over experts gives offsets; each
+//                       chunk's base row for each expert is their sum.
+//  3. dispatch_scatter: one warp per chunk walks its pairs in order, 32 at a
+//                       time; lanes holding the same expert rank themselves
+//                       with __match_any_sync, so the order inside an expert
+//                       is the pair order (token ascending) -- deterministic.
+#include "common.cuh"
+#include "moe_dispatch.h"
+
+namespace moe {
+namespace {
+
+constexpr int CHUNK_TOKENS = 64;
+
+__global__ void __launch_bounds__(256) dispatch_hist(const int32_t *__restrict__ idx, int T, int k,
+                                                     int E, int32_t *__restrict__ chunk_hist,
+                                                     int32_t *status) {
+  extern __shared__ int32_t h[];
+  for (int e = threadIdx.x; e < E; e += blockDim.x) h[e] = 0;
+  __syncthreads();
+  const int t0 = blockIdx.x * CHUNK_TOKENS;
+  const int n = min(CHUNK_TOKENS, T - t0) * k;
+  const int32_t *src = idx + (size_t)t0 * k;
+  for (int i = threadIdx.x; i < n; i += blockDim.x) {
+    const int e = src[i];
+    if (e < 0 || e >= E)
+      set_status(status, MOE_ERR_RANGE);
+    else
+      atomicAdd(&h[e], 1);
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x) chunk_hist[(size_t)blockIdx.x * E + e] = h[e];
+}
+
+// One block of >= E threads (E <= 1024).
+__global__ void __launch_bounds__(1024) dispatch_scan(int32_t *__restrict__ chunk_hist,
+                                                      int nchunks, int E,
+                                                      int32_t *__restrict__ counts,
+                                                      int32_t *__restrict__ offsets) {
+  __shared__ int32_t warp_tot[32];
+  const int e = threadIdx.x;
+  int run = 0;
+  if (e < E) {
+    for (int c = 0; c < nchunks; ++c) {
+      const int v = chunk_hist[(size_t)c * E + e];
+      chunk_hist[(size_t)c * E + e] = run;
+      run += v;
+    }
+    counts[e] = run;
+  }
+  // exclusive scan of run over e: warp inclusive scans, then warp totals
+  const int lane = threadIdx.x % 32, w = threadIdx.x / 32;
+  int v = (e < E) ? run : 0;
+  int inc = v;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int o = __shfl_up_sync(0xffffffffu, inc, off);
+    if (lane >= off) inc += o;
+  }
+  if (lane == 31) warp_tot[w] = inc;
+  __syncthreads();
+  if (w == 0) {
+    const int nw = (blockDim.x + 31) / 32;
+    int t = lane < nw ? warp_tot[lane] : 0;
+    int tinc = t;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int o = __shfl_up_sync(0xffffffffu, tinc, off);
+      if (lane >= off) tinc += o;
+    }
+    warp_tot[lane] = tinc - t;  // exclusive prefix of the warp totals
+  }
+  __syncthreads();
+  const int excl = inc - v + warp_tot[w];
+  if (e < E) {
+    offsets[e] = excl;
+    if (e == E - 1) offsets[E] = excl + v;
+    for (int c = 0; c < nchunks; ++c) chunk_hist[(size_t)c * E + e] += excl;
+  }
+}
+
+// One warp per chunk.
+__global__ void __launch_bounds__(32) dispatch_scatter(const int32_t *__restrict__ idx, int T,
+                                                       int k, int E,
+                                                       const int32_t *__restrict__ chunk_base,
+                                                       int32_t *__restrict__ sorted_token,
+                                                       int32_t *__restrict__ slot_of) {
+  extern __shared__ int32_t base[];
+  const int lane = threadIdx.x;
+  for (int e = lane; e < E; e += 32) base[e] = chunk_base[(size_t)blockIdx.x * E + e];
+  __syncwarp();
+  const int t0 = blockIdx.x * CHUNK_TOKENS;
+  const int n = min(CHUNK_TOKENS, T - t0) * k;
+  const size_t flat0 = (size_t)t0 * k;
+  const unsigned lt = (1u << lane) - 1u;
+  for (int i0 = 0; i0 < n; i0 += 32) {
+    const int i = i0 + lane;
+    int e = -1;
+    if (i < n) e = idx[flat0 + i];
+    const bool ok = i < n && e >= 0 && e < E;
+    const int key = ok ? e : -1 - lane;  // invalid lanes get a key of their own
+    const unsigned same = __match_any_sync(0xffffffffu, key);
+    if (ok) {
+      const int rank = __popc(same & lt);
+      const int pos = base[e] + rank;
+      sorted_token[pos] = t0 + i / k;
+      slot_of[flat0 + i] = pos;
+    }
+    __syncwarp();
+    // the highest lane of each group advances that expert's next free row
+    if (ok && (same >> lane) == 1u) base[e] += __popc(same);
+    __syncwarp();
+  }
+}
+
+}  // namespace
+}  // namespace moe
+
+using namespace moe;
+
+MOE_EXPORT size_t moe_dispatch_workspace_size(const moe_cfg *cfg, int64_t T) {
+  if (check_cfg(cfg) != MOE_OK || T < 0) return 0;
+  const int64_t nchunks = (T + CHUNK_TOKENS - 1) / CHUNK_TOKENS;
+  return align_up((size_t)(nchunks > 0 ? nchunks : 1) * cfg->n_routed * sizeof(int32_t), 256);
+}
+
+MOE_EXPORT moe_status moe_dispatch_build(const moe_cfg *cfg, int64_t T, const int32_t *indices,
+                                         int32_t *counts, int32_t *offsets,
+                                         int32_t *sorted_token, int32_t *slot_of, void *ws,
+                                         size_t ws_bytes, int32_t *dev_status,
+                                         moe_stream_t stream) {
+  moe_status st = check_cfg(cfg);
+  if (st != MOE_OK) return st;
+  if (T < 0 || T * (int64_t)cfg->topk >= ((int64_t)1 << 31)) return MOE_ERR_INVALID;
+  if (!counts || !offsets || !ws) return MOE_ERR_INVALID;
+  if (T > 0 && (!indices || !sorted_token || !slot_of)) return MOE_ERR_INVALID;
+  if (cfg->n_routed > 1024) return MOE_ERR_UNSUPPORTED;
+  if (ws_bytes < moe_dispatch_workspace_size(cfg, T)) return MOE_ERR_WORKSPACE;
+  cudaStream_t s = as_stream(stream);
+  const int E = cfg->n_routed, k = cfg->topk;
+  const int nchunks = (int)((T + CHUNK_TOKENS - 1) / CHUNK_TOKENS);
+  int32_t *chunk_hist = static_cast<int32_t *>(ws);
+  const size_t hsmem = (size_t)E * sizeof(int32_t);
+  if (nchunks > 0) {
+    dispatch_hist<<<nchunks, 256, hsmem, s>>>(indices, (int)T, k, E, chunk_hist, dev_status);
+    if ((st = launch_status()) != MOE_OK) return st;
+  }
+  const int scan_threads = (E + 31) / 32 * 32;
+  dispatch_scan<<<1, scan_threads, 0, s>>>(chunk_hist, nchunks, E, counts, offsets);
+  if ((st = launch_status()) != MOE_OK) return st;
+  if (nchunks > 0) {
+    dispatch_scatter<<<nchunks, 32, hsmem, s>>>(indices, (int)T, k, E, chunk_hist, sorted_token,
+                                                slot_of);
+    if ((st = launch_status()) != MOE_OK) return st;
+  }
+  return MOE_OK;
+}

@@ -1,0 +1,820 @@
+// moe_experts: routed experts and the shared expert as grouped SwiGLU GEMMs.
+//
+// Expert body: w2(silu(w1 x) * w3 x), three bias-free matrices -- the reading
+// of Expert(dim, moe_inter_dim) in the moe-init excerpt of "DeepSeek-V3.2-Exp
+// · Mixture of experts" that matches that page's per-expert count of
+// 3 * 7168 * 2048 parameters.  The shared expert runs on every token.
+//
+// Tensor-core path (bf16 activations; bf16 or e4m3 weights), sm_100a:
+//   gather_rows   X_perm[p] = x[sorted_token[p]] (expert-contiguous rows),
+//                 followed by the T rows of x for the shared expert.
+//   GEMM1         h = silu(X W1^T) * (X W3^T), bf16 out
+//   GEMM2         o = h W2^T, fp32 out
+// Both GEMMs are one persistent, warp-specialised kernel template
+// (tc_expert_gemm): warp 0 issues TMA loads into a shared-memory ring, one
+// thread of warp 1 issues tcgen05.mma into a double-buffered TMEM
+// accumulator, warps 2-5 drain the accumulator with tcgen05.ld and run the
+// epilogue while the next tile's MMAs proceed.
+//
+// The operands are swapped relative to the usual token-major GEMM: the 128
+// rows of an MMA (M) are weight rows and the MMA's N is the expert's tokens.
+// N is a run-time field of the instruction descriptor, so a tile spends MMA
+// work only on the tokens its expert really has (rounded up to 16) -- from 1
+// token per expert at decode to 256 at prefill -- and each weight byte is
+// streamed from HBM once per token tile.  For GEMM1 a 128-row A tile holds 64
+// rows of W1 and the same 64 rows of W3, so one accumulator carries both
+// halves of the SwiGLU; the epilogue pairs the warps that hold them.
+//
+// CUDA-core path: any other dtype combination (the fp32 configuration) runs
+// on simt_gemm1 / simt_gemm2 in fp32.
+#include <cuda_bf16.h>
+#include <cuda_fp8.h>
+#include <cudaTypedefs.h>
+#include <math.h>
+
+#include "common.cuh"
+#include "moe_experts.h"
+#include "sm100.cuh"
+
+namespace moe {
+namespace {
+
+using bf16 = __nv_bfloat16;
+
+// ------------------------------------------------------------------ tiling
+
+// Per group g (routed experts 0..E-1, then the shared expert): its row count
+// n_g, split into ntt_g token tiles of tile_base[g] rows (a multiple of 16,
+// at most rows_max) and ft feature tiles; tile_start[g] is the exclusive
+// prefix of ntt_g * ft over the groups and tile_start[G] the total.
+struct Tiling {
+  int rows_max;
+  int ft;
+  int32_t *tile_start;  // [G + 1]
+  int32_t *tile_base;   // [G]
+};
+
+__device__ __forceinline__ void group_tiles(int n, int rows_max, int &base, int &ntt) {
+  if (n <= 0) {
+    base = 16;
+    ntt = 0;
+    return;
+  }
+  const int ntt0 = (n + rows_max - 1) / rows_max;
+  base = ((n + ntt0 - 1) / ntt0 + 15) / 16 * 16;
+  ntt = (n + base - 1) / base;
+}
+
+// One warp: lane l owns a contiguous run of groups.
+__global__ void __launch_bounds__(32) prep_tiles(const int32_t *__restrict__ offsets, int E,
+                                                 int G, int T, Tiling t0, Tiling t1) {
+  const int lane = threadIdx.x;
+  const int per = (G + 31) / 32;
+  const int g0 = min(G, lane * per), g1 = min(G, g0 + per);
+  for (int which = 0; which < 2; ++which) {
+    const Tiling tl = which == 0 ? t0 : t1;
+    if (!tl.tile_start) continue;
+    int local = 0;
+    for (int g = g0; g < g1; ++g) {
+      const int n = g < E ? offsets[g + 1] - offsets[g] : T;
+      int base, ntt;
+      group_tiles(n, tl.rows_max, base, ntt);
+      tl.tile_base[g] = base;
+      local += ntt * tl.ft;
+    }
+    int inc = local;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int o = __shfl_up_sync(0xffffffffu, inc, off);
+      if (lane >= off) inc += o;
+    }
+    int run = inc - local;
+    for (int g = g0; g < g1; ++g) {
+      const int n = g < E ? offsets[g + 1] - offsets[g] : T;
+      int base, ntt;
+      group_tiles(n, tl.rows_max, base, ntt);
+      tl.tile_start[g] = run;
+      run += ntt * tl.ft;
+    }
+    if (lane == 31) tl.tile_start[G] = inc;
+  }
+}
+
+struct Tile {
+  int g, ft, n0, nvalid, rowbase;
+};
+
+// rowbase: first row of the group in the expert-contiguous activation
+// buffers (routed: offsets[g]; shared: after the T*k routed rows).
+__device__ __forceinline__ Tile decode_tile(int tile, const int32_t *tstart, const int32_t *tbase,
+                                            const int32_t *off, int G, int E, int T,
+                                            int rows_routed) {
+  int lo = 0, hi = G;
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (tstart[mid] <= tile)
+      lo = mid;
+    else
+      hi = mid;
+  }
+  Tile t;
+  t.g = lo;
+  const int n = lo < E ? off[lo + 1] - off[lo] : T;
+  const int base = tbase[lo];
+  const int ntt = (n + base - 1) / base;
+  const int local = tile - tstart[lo];
+  t.ft = local / ntt;
+  const int tt = local - t.ft * ntt;
+  t.n0 = tt * base;
+  t.nvalid = min(base, n - t.n0);
+  t.rowbase = lo < E ? off[lo] : rows_routed + (lo - E) * T;
+  return t;
+}
+
+// ------------------------------------------------------------------ gather
+
+// X_perm[p] = x[sorted_token[p]] for p < rows_routed, then x itself for the
+// shared expert's rows.  One warp per row, 16-byte vectors.
+__global__ void __launch_bounds__(256) gather_rows(const uint4 *__restrict__ x,
+                                                   const int32_t *__restrict__ sorted_token,
+                                                   uint4 *__restrict__ xp, int rows_routed,
+                                                   int rows_total, int T, int vec_per_row) {
+  const int row = (int)((blockIdx.x * (size_t)blockDim.x + threadIdx.x) / 32);
+  const int lane = threadIdx.x % 32;
+  if (row >= rows_total) return;
+  const int src = row < rows_routed ? sorted_token[row] : (row - rows_routed) % T;
+  const uint4 *s = x + (size_t)src * vec_per_row;
+  uint4 *d = xp + (size_t)row * vec_per_row;
+  for (int v = lane; v < vec_per_row; v += 32) d[v] = __ldg(s + v);
+}
+
+// ------------------------------------------------------- tensor-core GEMMs
+
+namespace tc {
+
+constexpr int BK = 64;                 // K elements per ring stage (128 bytes bf16)
+constexpr int BM = 128;                // MMA M: weight rows per tile
+constexpr int A_BYTES = BM * BK * 2;   // 16 KB
+constexpr int THREADS = 192;           // warp 0 TMA, warp 1 MMA, warps 2-5 epilogue
+constexpr int EPI_WARPS = 4;
+constexpr int XB_STRIDE = 17;          // exchange buffer row stride (floats)
+
+struct Params {
+  const int32_t *tile_start;
+  const int32_t *tile_base;
+  const int32_t *offsets;
+  int E, G, T;
+  int KB;           // K blocks of 64
+  int I, D;
+  int rows_routed;  // T * k
+  void *out;        // GEMM1: h [rows, I] bf16; GEMM2: out_perm [T*k, D] fp32
+  float *out_shared;
+  int32_t *status;
+  int64_t timeout_ns;
+};
+
+template <int MODE, int BN_MAX, int BOXN, int STAGES>
+struct Layout {
+  static constexpr int B_BYTES = BN_MAX * BK * 2;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int BAR_OFF = STAGES * STAGE_BYTES;
+  static constexpr int NBARS = 2 * STAGES + 5;  // full, empty, acc_full x2, acc_empty x2, drain
+  static constexpr int MISC_OFF = BAR_OFF + NBARS * 8;
+  static constexpr int MISC_BYTES = 16 + 4 * STAGES;
+  static constexpr int XBUF_OFF = (MISC_OFF + MISC_BYTES + 127) / 128 * 128;
+  static constexpr int XBUF_BYTES = MODE == 1 ? 2 * 2 * 32 * XB_STRIDE * 4 : 0;
+  static constexpr int TAB_OFF = XBUF_OFF + XBUF_BYTES;
+  static constexpr uint32_t TMEM_COLS = 2 * BN_MAX < 32 ? 32 : 2 * BN_MAX;
+  static size_t smem_bytes(int G, int E) {
+    return 1024 + TAB_OFF + sizeof(int32_t) * (size_t)((G + 1) + G + (E + 1));
+  }
+  static_assert(BN_MAX % 16 == 0 && BN_MAX >= 16 && BN_MAX <= 256, "MMA N range");
+  static_assert(BOXN % 16 == 0 && BN_MAX % BOXN == 0, "B box rows");
+  static_assert((2 * BN_MAX & (2 * BN_MAX - 1)) == 0, "TMEM columns must be a power of two");
+};
+
+// Waits for a barrier phase with a time limit but ignores the abort flag;
+// used only to drain copies already in flight before the CTA exits.
+__device__ __forceinline__ void drain_wait(uint64_t *bar, uint32_t parity, int64_t limit_ns) {
+  const uint64_t t0 = sm100::globaltimer_ns();
+  while (!sm100::mbar_try_wait(bar, parity)) {
+    if ((int64_t)(sm100::globaltimer_ns() - t0) > limit_ns) break;
+  }
+}
+
+template <int MODE, int BN_MAX, int BOXN, int STAGES>
+__global__ void __launch_bounds__(THREADS, 1)
+    tc_expert_gemm(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA1,
+                   const __grid_constant__ CUtensorMap tmB, const Params p) {
+  using L = Layout<MODE, BN_MAX, BOXN, STAGES>;
+  using namespace sm100;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                            ~static_cast<uintptr_t>(1023));
+  uint64_t *full = reinterpret_cast<uint64_t *>(sm + L::BAR_OFF);
+  uint64_t *empty = full + STAGES;
+  uint64_t *accf = empty + STAGES;
+  uint64_t *acce = accf + 2;
+  uint64_t *drain = acce + 2;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + L::MISC_OFF);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + L::MISC_OFF + 4);
+  volatile int *pending = reinterpret_cast<volatile int *>(sm + L::MISC_OFF + 16);
+  float *xbuf = reinterpret_cast<float *>(sm + L::XBUF_OFF);
+  int32_t *s_tstart = reinterpret_cast<int32_t *>(sm + L::TAB_OFF);
+  int32_t *s_tbase = s_tstart + p.G + 1;
+  int32_t *s_off = s_tbase + p.G;
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(full + s, 1);
+      mbar_init(empty + s, 1);
+      pending[s] = -1;
+    }
+    mbar_init(accf + 0, 1);
+    mbar_init(accf + 1, 1);
+    mbar_init(acce + 0, EPI_WARPS);
+    mbar_init(acce + 1, EPI_WARPS);
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&tmA0);
+    if (MODE == 1) tma_prefetch_desc(&tmA1);
+    tma_prefetch_desc(&tmB);
+  }
+  for (int i = threadIdx.x; i <= p.G; i += THREADS) s_tstart[i] = p.tile_start[i];
+  for (int i = threadIdx.x; i < p.G; i += THREADS) s_tbase[i] = p.tile_base[i];
+  for (int i = threadIdx.x; i <= p.E; i += THREADS) s_off[i] = p.offsets[i];
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, L::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int total = s_tstart[p.G];
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---------------------------------------------------- TMA producer
+      const uint64_t pol_w = policy_evict_first();  // weights: streamed once
+      const uint64_t pol_x = policy_evict_last();   // activations: re-read per feature tile
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
+        const Tile t = decode_tile(tile, s_tstart, s_tbase, s_off, p.G, p.E, p.T, p.rows_routed);
+        const int arow = MODE == 1 ? t.g * p.I + t.ft * 64 : t.g * p.D + t.ft * BM;
+        const int nbox = (t.nvalid + BOXN - 1) / BOXN;
+        const uint32_t bytes = (uint32_t)(A_BYTES + nbox * BOXN * BK * 2);
+        for (int kb = 0; kb < p.KB; ++kb) {
+          if (!wait_bounded(empty + stage, phase ^ 1u, abort_flag, p.timeout_ns, p.status)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(full + stage, bytes);
+          pending[stage] = (int)phase;
+          uint8_t *a_dst = sm + stage * L::STAGE_BYTES;
+          uint8_t *b_dst = a_dst + A_BYTES;
+          if (MODE == 1) {
+            tma_load_2d_hint(&tmA0, a_dst, full + stage, kb * BK, arow, pol_w);
+            tma_load_2d_hint(&tmA1, a_dst + A_BYTES / 2, full + stage, kb * BK, arow, pol_w);
+          } else {
+            tma_load_2d_hint(&tmA0, a_dst, full + stage, kb * BK, arow, pol_w);
+          }
+          for (int i = 0; i < nbox; ++i)
+            tma_load_2d_hint(&tmB, b_dst + i * BOXN * BK * 2, full + stage, kb * BK,
+                             t.rowbase + t.n0 + i * BOXN, pol_x);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ------------------------------------------------------ MMA issuer
+      int stage = 0, acc = 0;
+      uint32_t phase = 0, acc_phase = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
+        const Tile t = decode_tile(tile, s_tstart, s_tbase, s_off, p.G, p.E, p.T, p.rows_routed);
+        if (!wait_bounded(acce + acc, acc_phase ^ 1u, abort_flag, p.timeout_ns, p.status)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN_MAX);
+        const int nmma = (t.nvalid + 15) & ~15;
+        const uint32_t idesc = idesc_bf16_f32(BM, nmma);
+        for (int kb = 0; kb < p.KB; ++kb) {
+          if (!wait_bounded(full + stage, phase, abort_flag, p.timeout_ns, p.status)) {
+            ok = false;
+            break;
+          }
+          pending[stage] = -1;
+          tc_fence_after();
+          const uint32_t a_addr = smem_u32(sm + stage * L::STAGE_BYTES);
+          const uint32_t b_addr = a_addr + A_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk)
+            mma_bf16(d_tmem, sdesc_sw128(a_addr + kk * 32), sdesc_sw128(b_addr + kk * 32), idesc,
+                     (kb | kk) != 0 ? 1u : 0u);
+          mma_commit(empty + stage);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        mma_commit(accf + acc);
+        acc ^= 1;
+        if (acc == 0) acc_phase ^= 1u;
+      }
+      if (!ok) {
+        // make sure no MMA is still writing TMEM before it is freed
+        mma_commit(drain);
+        drain_wait(drain, 0, p.timeout_ns);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp & 3;  // TMEM lane quarter this warp may access
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
+      const Tile t = decode_tile(tile, s_tstart, s_tbase, s_off, p.G, p.E, p.T, p.rows_routed);
+      if (!wait_bounded(accf + acc, acc_phase, abort_flag, p.timeout_ns, p.status)) break;
+      tc_fence_after();
+      const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN_MAX);
+      if (MODE == 2) {
+        // lanes are output features d, columns are tokens
+        float *out;
+        size_t row0;
+        if (t.g < p.E) {
+          out = static_cast<float *>(p.out);
+          row0 = (size_t)t.rowbase + t.n0;
+        } else {
+          out = p.out_shared;
+          row0 = (size_t)(t.g - p.E) * p.T + t.n0;
+        }
+        const int d = t.ft * BM + q * 32 + lane;
+        for (int c0 = 0; c0 < t.nvalid; c0 += 32) {
+          uint32_t v[32];
+          tmem_ld_32x32b_x32(tb + (uint32_t)c0, v);
+          tmem_wait_ld();
+#pragma unroll
+          for (int j = 0; j < 32; ++j)
+            if (c0 + j < t.nvalid) out[(row0 + c0 + j) * p.D + d] = __uint_as_float(v[j]);
+        }
+      } else {
+        // lanes 0-63 hold w1.x (a), lanes 64-127 hold w3.x (u) for the same
+        // 64 features; warps q and q+2 pair up through shared memory, each
+        // finishing half of the 32 columns of a chunk
+        const int pr = q & 1;
+        const bool is_a = q < 2;
+        float *buf_a = xbuf + pr * 2 * 32 * XB_STRIDE;  // a, columns 16-31 of the chunk
+        float *buf_u = buf_a + 32 * XB_STRIDE;          // u, columns 0-15 of the chunk
+        bf16 *out = static_cast<bf16 *>(p.out);
+        const int f = t.ft * 64 + pr * 32 + lane;
+        const size_t row0 = (size_t)t.rowbase + t.n0;
+        for (int c0 = 0; c0 < t.nvalid; c0 += 32) {
+          uint32_t v[32];
+          tmem_ld_32x32b_x32(tb + (uint32_t)c0, v);
+          tmem_wait_ld();
+          float *mine = is_a ? buf_a : buf_u;
+#pragma unroll
+          for (int j = 0; j < 16; ++j)
+            mine[lane * XB_STRIDE + j] = __uint_as_float(is_a ? v[16 + j] : v[j]);
+          named_bar_sync(1 + pr, 64);
+          const float *other = is_a ? buf_u : buf_a;
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const int col = is_a ? j : 16 + j;
+            const float a = is_a ? __uint_as_float(v[j]) : other[lane * XB_STRIDE + j];
+            const float u = is_a ? other[lane * XB_STRIDE + j] : __uint_as_float(v[16 + j]);
+            const float h = a / (1.0f + expf(-a)) * u;
+            if (c0 + col < t.nvalid) out[(row0 + c0 + col) * p.I + f] = __float2bfloat16_rn(h);
+          }
+          named_bar_sync(1 + pr, 64);
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(acce + acc);
+      acc ^= 1;
+      if (acc == 0) acc_phase ^= 1u;
+    }
+  }
+
+  __syncthreads();
+  if (threadIdx.x == 0 && *abort_flag) {
+    // a stalled pipeline stopped early: let copies already issued land
+    for (int s = 0; s < STAGES; ++s)
+      if (pending[s] >= 0) drain_wait(full + s, (uint32_t)pending[s], p.timeout_ns);
+  }
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, L::TMEM_COLS);
+  }
+}
+
+// single-CTA self-test of the bounded wait: nothing ever arrives
+__global__ void selftest_wait_kernel(int64_t limit_ns, int32_t *status) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    sm100::mbar_init(&bar, 1);
+    abort_flag = 0;
+    sm100::fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const bool ok = sm100::wait_bounded(&bar, 0, &abort_flag, limit_ns, status);
+    (void)ok;
+  }
+}
+
+}  // namespace tc
+
+// ----------------------------------------------------------- CUDA-core path
+
+__device__ __forceinline__ float ld_f(const float *p, size_t i) { return p[i]; }
+__device__ __forceinline__ float ld_f(const bf16 *p, size_t i) { return __bfloat162float(p[i]); }
+__device__ __forceinline__ float ld_f(const __nv_fp8_e4m3 *p, size_t i) { return float(p[i]); }
+
+// element (r, c) of group g's [rows, cols] matrix, with the 128 x 128 block
+// scale for e4m3 weights
+template <typename WT>
+__device__ __forceinline__ float w_at(const WT *w, const float *scale, int g, int r, int c,
+                                      int rows, int cols) {
+  const float v = ld_f(w, ((size_t)g * rows + r) * cols + c);
+  if (scale) {
+    const int sr = rows / 128, sc = cols / 128;
+    return v * scale[((size_t)g * sr + r / 128) * sc + c / 128];
+  }
+  return v;
+}
+
+constexpr int ST = 32;  // CUDA-core tile: 32 rows x 32 features
+
+struct SimtArgs {
+  const int32_t *tile_start, *tile_base, *offsets, *sorted_token;
+  int E, G, T, D, I, rows_routed, act_bf16;
+  float *h;  // [rows, I] fp32 (values rounded to bf16 when act_bf16)
+  float *out_perm, *out_shared;
+};
+
+template <typename XT, typename WT>
+__global__ void __launch_bounds__(256) simt_gemm1(const XT *__restrict__ x, const WT *w1,
+                                                  const WT *w3, const float *s1, const float *s3,
+                                                  SimtArgs a) {
+  __shared__ float xs[ST][ST + 1], as_[ST][ST + 1], us[ST][ST + 1];
+  __shared__ int tok[ST];
+  const int tile = blockIdx.x;
+  if (tile >= a.tile_start[a.G]) return;
+  const Tile t = decode_tile(tile, a.tile_start, a.tile_base, a.offsets, a.G, a.E, a.T,
+                             a.rows_routed);
+  if (threadIdx.x < ST) {
+    const int r = threadIdx.x;
+    tok[r] = r < t.nvalid ? (t.g < a.E ? a.sorted_token[t.rowbase + t.n0 + r] : t.n0 + r) : -1;
+  }
+  const int r = threadIdx.x / 8, fq = (threadIdx.x % 8) * 4;
+  float acc_a[4] = {0.f, 0.f, 0.f, 0.f}, acc_u[4] = {0.f, 0.f, 0.f, 0.f};
+  for (int k0 = 0; k0 < a.D; k0 += ST) {
+    __syncthreads();
+    for (int i = threadIdx.x; i < ST * ST; i += 256) {
+      const int rr = i / ST, kk = i % ST, kd = k0 + kk;
+      xs[rr][kk] = (tok[rr] >= 0 && kd < a.D) ? ld_f(x, (size_t)tok[rr] * a.D + kd) : 0.f;
+      const int f = t.ft * ST + rr;
+      const bool in = f < a.I && kd < a.D;
+      as_[rr][kk] = in ? w_at(w1, s1, t.g, f, kd, a.I, a.D) : 0.f;
+      us[rr][kk] = in ? w_at(w3, s3, t.g, f, kd, a.I, a.D) : 0.f;
+    }
+    __syncthreads();
+#pragma unroll 8
+    for (int kk = 0; kk < ST; ++kk) {
+      const float xv = xs[r][kk];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        acc_a[j] = fmaf(xv, as_[fq + j][kk], acc_a[j]);
+        acc_u[j] = fmaf(xv, us[fq + j][kk], acc_u[j]);
+      }
+    }
+  }
+  if (r < t.nvalid) {
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int f = t.ft * ST + fq + j;
+      if (f >= a.I) continue;
+      float h = acc_a[j] / (1.0f + expf(-acc_a[j])) * acc_u[j];
+      if (a.act_bf16) h = __bfloat162float(__float2bfloat16_rn(h));
+      a.h[((size_t)t.rowbase + t.n0 + r) * a.I + f] = h;
+    }
+  }
+}
+
+template <typename WT>
+__global__ void __launch_bounds__(256) simt_gemm2(const WT *w2, const float *s2, SimtArgs a) {
+  __shared__ float hs[ST][ST + 1], ws[ST][ST + 1];
+  const int tile = blockIdx.x;
+  if (tile >= a.tile_start[a.G]) return;
+  const Tile t = decode_tile(tile, a.tile_start, a.tile_base, a.offsets, a.G, a.E, a.T,
+                             a.rows_routed);
+  const int r = threadIdx.x / 8, dq = (threadIdx.x % 8) * 4;
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  for (int k0 = 0; k0 < a.I; k0 += ST) {
+    __syncthreads();
+    for (int i = threadIdx.x; i < ST * ST; i += 256) {
+      const int rr = i / ST, kk = i % ST, ki = k0 + kk;
+      hs[rr][kk] = (rr < t.nvalid && ki < a.I)
+                       ? a.h[((size_t)t.rowbase + t.n0 + rr) * a.I + ki]
+                       : 0.f;
+      const int d = t.ft * ST + rr;
+      ws[rr][kk] = (d < a.D && ki < a.I) ? w_at(w2, s2, t.g, d, ki, a.D, a.I) : 0.f;
+    }
+    __syncthreads();
+#pragma unroll 8
+    for (int kk = 0; kk < ST; ++kk) {
+      const float hv = hs[r][kk];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) acc[j] = fmaf(hv, ws[dq + j][kk], acc[j]);
+    }
+  }
+  if (r < t.nvalid) {
+    float *out;
+    size_t row;
+    if (t.g < a.E) {
+      out = a.out_perm;
+      row = (size_t)t.rowbase + t.n0 + r;
+    } else {
+      out = a.out_shared;
+      row = (size_t)(t.g - a.E) * a.T + t.n0 + r;
+    }
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int d = t.ft * ST + dq + j;
+      if (d < a.D) out[row * a.D + d] = acc[j];
+    }
+  }
+}
+
+// -------------------------------------------------------------- host side
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void *ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  }
+  return fn;
+}
+
+// 2-D row-major [rows, cols] matrix of `elem` bytes, box of box_rows rows x
+// box_cols columns, 128-byte swizzle (box_cols * elem must be 128).
+bool make_tmap(CUtensorMap *m, const void *base, CUtensorMapDataType dt, size_t elem,
+               uint64_t rows, uint64_t cols, uint32_t box_rows, uint32_t box_cols) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t gdim[2] = {cols, rows};
+  cuuint64_t gstride[1] = {cols * elem};
+  cuuint32_t box[2] = {box_cols, box_rows};
+  cuuint32_t estride[2] = {1, 1};
+  return fn(m, dt, 2, const_cast<void *>(base), gdim, gstride, box, estride,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+  return n;
+}
+
+struct WsLayout {
+  size_t tab, xperm, h, total;
+  int64_t rows_pad;
+};
+
+constexpr int ROW_PAD = 256;  // spare rows so a TMA box never starts past a buffer
+
+bool tc_path(const moe_cfg *c, moe_dtype x_dt, moe_dtype w_dt) {
+  return x_dt == MOE_BF16 && (w_dt == MOE_BF16) && c->dim % 128 == 0 && c->inter % 128 == 0;
+}
+
+WsLayout ws_layout(const moe_cfg *c, int64_t T, moe_dtype x_dt, moe_dtype w_dt) {
+  WsLayout l;
+  const int64_t G = c->n_routed + c->n_shared;
+  l.rows_pad = T * c->topk + T * c->n_shared + ROW_PAD;
+  l.tab = 0;
+  size_t off = align_up(sizeof(int32_t) * (size_t)(4 * G + 4), 1024);
+  const bool tc = tc_path(c, x_dt, w_dt);
+  l.xperm = off;
+  if (tc) off = align_up(off + (size_t)l.rows_pad * c->dim * 2, 1024);
+  l.h = off;
+  off = align_up(off + (size_t)l.rows_pad * c->inter * (tc ? 2 : 4), 1024);
+  l.total = off;
+  return l;
+}
+
+template <int MODE, int BN_MAX, int BOXN, int STAGES>
+moe_status launch_tc(const CUtensorMap &a0, const CUtensorMap &a1, const CUtensorMap &b,
+                     const tc::Params &p, cudaStream_t s) {
+  using L = tc::Layout<MODE, BN_MAX, BOXN, STAGES>;
+  auto kern = tc::tc_expert_gemm<MODE, BN_MAX, BOXN, STAGES>;
+  const size_t smem = L::smem_bytes(p.G, p.E);
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+      cudaSuccess)
+    return MOE_ERR_CUDA;
+  const int nsm = sm_count();
+  if (nsm <= 0) return MOE_ERR_CUDA;
+  kern<<<nsm, tc::THREADS, smem, s>>>(a0, a1, b, p);
+  return launch_status();
+}
+
+template <int BN_MAX, int BOXN, int STAGES>
+moe_status run_tc(const moe_cfg *c, int64_t T, const void *x, const moe_expert_weights *w,
+                  const int32_t *offsets, const int32_t *sorted_token, float *out_perm,
+                  float *out_shared, uint8_t *ws, const WsLayout &l, int32_t *dev_status,
+                  cudaStream_t s) {
+  const int E = c->n_routed, G = c->n_routed + c->n_shared, D = c->dim, I = c->inter;
+  const int rows_routed = (int)(T * c->topk);
+  const int rows_total = rows_routed + (int)(T * c->n_shared);
+  int32_t *tab = reinterpret_cast<int32_t *>(ws + l.tab);
+  Tiling t1{BN_MAX, I / 64, tab, tab + (G + 1)};
+  Tiling t2{BN_MAX, D / tc::BM, tab + (2 * G + 1), tab + (3 * G + 2)};
+  prep_tiles<<<1, 32, 0, s>>>(offsets, E, G, (int)T, t1, t2);
+  moe_status st = launch_status();
+  if (st != MOE_OK) return st;
+
+  bf16 *xperm = reinterpret_cast<bf16 *>(ws + l.xperm);
+  bf16 *h = reinterpret_cast<bf16 *>(ws + l.h);
+  {
+    const int vec = D * 2 / 16;
+    const int64_t threads = (int64_t)rows_total * 32;
+    gather_rows<<<(unsigned)((threads + 255) / 256), 256, 0, s>>>(
+        static_cast<const uint4 *>(x), sorted_token, reinterpret_cast<uint4 *>(xperm),
+        rows_routed, rows_total, (int)T, vec);
+    if ((st = launch_status()) != MOE_OK) return st;
+  }
+  CUtensorMap mw1, mw3, mw2, mx, mh;
+  const CUtensorMapDataType BF = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  if (!make_tmap(&mw1, w->w1, BF, 2, (uint64_t)G * I, D, 64, 64) ||
+      !make_tmap(&mw3, w->w3, BF, 2, (uint64_t)G * I, D, 64, 64) ||
+      !make_tmap(&mw2, w->w2, BF, 2, (uint64_t)G * D, I, tc::BM, 64) ||
+      !make_tmap(&mx, xperm, BF, 2, (uint64_t)l.rows_pad, D, BOXN, 64) ||
+      !make_tmap(&mh, h, BF, 2, (uint64_t)l.rows_pad, I, BOXN, 64))
+    return MOE_ERR_CUDA;
+
+  tc::Params p;
+  p.offsets = offsets;
+  p.E = E;
+  p.G = G;
+  p.T = (int)T;
+  p.I = I;
+  p.D = D;
+  p.rows_routed = rows_routed;
+  p.out_shared = out_shared;
+  p.status = dev_status;
+  p.timeout_ns = 1000000000LL;
+
+  p.tile_start = t1.tile_start;
+  p.tile_base = t1.tile_base;
+  p.KB = D / tc::BK;
+  p.out = h;
+  if ((st = launch_tc<1, BN_MAX, BOXN, STAGES>(mw1, mw3, mx, p, s)) != MOE_OK) return st;
+
+  p.tile_start = t2.tile_start;
+  p.tile_base = t2.tile_base;
+  p.KB = I / tc::BK;
+  p.out = out_perm;
+  return launch_tc<2, BN_MAX, BOXN, STAGES>(mw2, mw2, mh, p, s);
+}
+
+template <typename XT, typename WT>
+moe_status run_simt_t(const moe_cfg *c, int64_t T, const void *x, const moe_expert_weights *w,
+                      const int32_t *offsets, const int32_t *sorted_token, float *out_perm,
+                      float *out_shared, uint8_t *ws, const WsLayout &l, int act_bf16,
+                      cudaStream_t s) {
+  const int E = c->n_routed, G = c->n_routed + c->n_shared, D = c->dim, I = c->inter;
+  int32_t *tab = reinterpret_cast<int32_t *>(ws + l.tab);
+  Tiling t1{ST, (I + ST - 1) / ST, tab, tab + (G + 1)};
+  Tiling t2{ST, (D + ST - 1) / ST, tab + (2 * G + 1), tab + (3 * G + 2)};
+  prep_tiles<<<1, 32, 0, s>>>(offsets, E, G, (int)T, t1, t2);
+  moe_status st = launch_status();
+  if (st != MOE_OK) return st;
+  SimtArgs a;
+  a.offsets = offsets;
+  a.sorted_token = sorted_token;
+  a.E = E;
+  a.G = G;
+  a.T = (int)T;
+  a.D = D;
+  a.I = I;
+  a.rows_routed = (int)(T * c->topk);
+  a.act_bf16 = act_bf16;
+  a.h = reinterpret_cast<float *>(ws + l.h);
+  a.out_perm = out_perm;
+  a.out_shared = out_shared;
+  // upper bound on tiles: sum over groups of ceil(n_g / 16) times feature tiles
+  const int64_t rows = T * c->topk + T * c->n_shared;
+  const int64_t ub1 = (rows / 16 + G) * t1.ft, ub2 = (rows / 16 + G) * t2.ft;
+  a.tile_start = t1.tile_start;
+  a.tile_base = t1.tile_base;
+  simt_gemm1<XT, WT><<<(unsigned)ub1, 256, 0, s>>>(
+      static_cast<const XT *>(x), static_cast<const WT *>(w->w1), static_cast<const WT *>(w->w3),
+      w->w_dt == MOE_E4M3 ? w->s1 : nullptr, w->w_dt == MOE_E4M3 ? w->s3 : nullptr, a);
+  if ((st = launch_status()) != MOE_OK) return st;
+  a.tile_start = t2.tile_start;
+  a.tile_base = t2.tile_base;
+  simt_gemm2<WT><<<(unsigned)ub2, 256, 0, s>>>(static_cast<const WT *>(w->w2),
+                                               w->w_dt == MOE_E4M3 ? w->s2 : nullptr, a);
+  return launch_status();
+}
+
+template <typename XT>
+moe_status run_simt_x(const moe_cfg *c, int64_t T, const void *x, const moe_expert_weights *w,
+                      const int32_t *offsets, const int32_t *sorted_token, float *out_perm,
+                      float *out_shared, uint8_t *ws, const WsLayout &l, int act_bf16,
+                      cudaStream_t s) {
+  switch (w->w_dt) {
+    case MOE_F32:
+      return run_simt_t<XT, float>(c, T, x, w, offsets, sorted_token, out_perm, out_shared, ws, l,
+                                   act_bf16, s);
+    case MOE_BF16:
+      return run_simt_t<XT, bf16>(c, T, x, w, offsets, sorted_token, out_perm, out_shared, ws, l,
+                                  act_bf16, s);
+    case MOE_E4M3:
+      return run_simt_t<XT, __nv_fp8_e4m3>(c, T, x, w, offsets, sorted_token, out_perm,
+                                           out_shared, ws, l, act_bf16, s);
+  }
+  return MOE_ERR_UNSUPPORTED;
+}
+
+}  // namespace
+}  // namespace moe
+
+using namespace moe;
+
+MOE_EXPORT size_t moe_experts_workspace_size(const moe_cfg *cfg, int64_t T, moe_dtype x_dt,
+                                             moe_dtype w_dt) {
+  if (check_cfg(cfg) != MOE_OK || T < 0) return 0;
+  return ws_layout(cfg, T, x_dt, w_dt).total;
+}
+
+MOE_EXPORT moe_status moe_experts_forward(const moe_cfg *cfg, int64_t T, const void *x,
+                                          moe_dtype x_dt, const moe_expert_weights *w,
+                                          const int32_t *offsets, const int32_t *sorted_token,
+                                          float *out_perm, float *out_shared, void *ws,
+                                          size_t ws_bytes, int32_t *dev_status,
+                                          moe_stream_t stream) {
+  moe_status st = check_cfg(cfg);
+  if (st != MOE_OK) return st;
+  if (T < 0 || (T * (int64_t)cfg->topk + T) >= ((int64_t)1 << 31)) return MOE_ERR_INVALID;
+  if (T == 0) return MOE_OK;
+  if (!x || !w || !w->w1 || !w->w3 || !w->w2 || !offsets || !sorted_token || !out_perm || !ws)
+    return MOE_ERR_INVALID;
+  if (cfg->n_shared > 1) return MOE_ERR_UNSUPPORTED;
+  if (cfg->n_shared == 1 && !out_shared) return MOE_ERR_INVALID;
+  if (x_dt != MOE_F32 && x_dt != MOE_BF16) return MOE_ERR_UNSUPPORTED;
+  if (w->w_dt != MOE_F32 && w->w_dt != MOE_BF16 && w->w_dt != MOE_E4M3) return MOE_ERR_UNSUPPORTED;
+  if (w->w_dt == MOE_E4M3) {
+    if (!w->s1 || !w->s3 || !w->s2) return MOE_ERR_INVALID;
+    if (cfg->dim % 128 != 0 || cfg->inter % 128 != 0) return MOE_ERR_UNSUPPORTED;
+  }
+  const WsLayout l = ws_layout(cfg, T, x_dt, w->w_dt);
+  if (ws_bytes < l.total) return MOE_ERR_WORKSPACE;
+  cudaStream_t s = as_stream(stream);
+  uint8_t *wsb = static_cast<uint8_t *>(ws);
+  if (tc_path(cfg, x_dt, w->w_dt)) {
+    // few rows per expert (decode): narrow token tiles and a deep ring so
+    // that enough weight bytes are in flight; otherwise up to 256 tokens
+    if (T * cfg->topk <= (int64_t)16 * cfg->n_routed)
+      return run_tc<32, 32, 10>(cfg, T, x, w, offsets, sorted_token, out_perm, out_shared, wsb,
+                                l, dev_status, s);
+    return run_tc<256, 32, 4>(cfg, T, x, w, offsets, sorted_token, out_perm, out_shared, wsb, l,
+                              dev_status, s);
+  }
+  const int act_bf16 = x_dt == MOE_BF16;
+  if (x_dt == MOE_BF16)
+    return run_simt_x<bf16>(cfg, T, x, w, offsets, sorted_token, out_perm, out_shared, wsb, l,
+                            act_bf16, s);
+  return run_simt_x<float>(cfg, T, x, w, offsets, sorted_token, out_perm, out_shared, wsb, l,
+                           act_bf16, s);
+}
+
+MOE_EXPORT moe_status moe_experts_selftest_wait(int64_t limit_ns, int32_t *dev_status,
+                                                moe_stream_t stream) {
+  if (limit_ns <= 0 || limit_ns > 2000000000LL || !dev_status) return MOE_ERR_INVALID;
+  tc::selftest_wait_kernel<<<1, 32, 0, as_stream(stream)>>>(limit_ns, dev_status);
+  return launch_status();
+}

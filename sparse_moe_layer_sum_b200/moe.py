@@ -1,0 +1,241 @@
+"""Python binding for the MoE block libraries.
+
+Argument marshalling only: every step of the block runs in the CUDA kernels
+of the four C-ABI libraries; PyTorch provides device memory and the stream.
+
+    block = MoEBlock(shape, params)        # weights already on the GPU
+    y = block.forward(x)                   # x [T, dim] on the GPU -> y fp32
+"""
+from __future__ import annotations
+
+import ctypes
+from dataclasses import dataclass
+from typing import Optional
+
+import torch
+
+from . import _lib
+from ._lib import MoECfg, MoEExpertWeights, check, fn
+
+
+@dataclass(frozen=True)
+class BlockShape:
+    """Block hyper-parameters (names of the gate-init / moe-init excerpts)."""
+
+    dim: int
+    n_routed: int
+    n_groups: int
+    topk_groups: int
+    topk: int
+    inter: int
+    n_shared: int = 1
+    route_scale: float = 2.5
+    score_func: str = "sigmoid"
+    has_bias: bool = True
+
+    def cfg(self) -> MoECfg:
+        return MoECfg(self.dim, self.n_routed, self.n_groups, self.topk_groups, self.topk,
+                      self.inter, self.n_shared, self.route_scale,
+                      _lib.SCORE_FUNCS[self.score_func], int(self.has_bias))
+
+
+_TORCH_DT = {torch.float32: "f32", torch.bfloat16: "bf16", torch.uint8: "e4m3",
+             torch.float8_e4m3fn: "e4m3"}
+
+
+def _dt(t: torch.Tensor) -> int:
+    return _lib.DTYPES[_TORCH_DT[t.dtype]]
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def _stream() -> int:
+    return torch.cuda.current_stream().cuda_stream
+
+
+def _check_cuda(*ts: Optional[torch.Tensor]) -> None:
+    for t in ts:
+        if t is not None and (not t.is_cuda or not t.is_contiguous()):
+            raise ValueError("tensors must be contiguous CUDA tensors")
+
+
+def _ws(nbytes: int, device) -> torch.Tensor:
+    return torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device)
+
+
+# ---------------------------------------------------------------- the four
+
+
+def router_forward(shape: BlockShape, x: torch.Tensor, w_r: torch.Tensor,
+                   bias: Optional[torch.Tensor], *, gap: bool = False, ws=None, status=None):
+    """moe_router_forward: (weights [T,k] fp32, indices [T,k] int32, gap [T] or None)."""
+    _check_cuda(x, w_r, bias)
+    cfg = shape.cfg()
+    T = x.shape[0]
+    weights = torch.empty(T, shape.topk, dtype=torch.float32, device=x.device)
+    indices = torch.empty(T, shape.topk, dtype=torch.int32, device=x.device)
+    sel_gap = torch.empty(T, dtype=torch.float32, device=x.device) if gap else None
+    need = fn("moe_router", "moe_router_workspace_size")(ctypes.byref(cfg), T)
+    if ws is None or ws.numel() < need:
+        ws = _ws(need, x.device)
+    st = fn("moe_router", "moe_router_forward")(
+        ctypes.byref(cfg), T, x.data_ptr(), _dt(x), w_r.data_ptr(), _ptr(bias),
+        weights.data_ptr(), indices.data_ptr(), _ptr(sel_gap), ws.data_ptr(), ws.numel(),
+        _ptr(status), _stream())
+    check(st, "moe_router_forward")
+    return weights, indices, sel_gap
+
+
+def dispatch_build(shape: BlockShape, indices: torch.Tensor, *, ws=None, status=None):
+    """moe_dispatch_build: (counts [E], offsets [E+1], sorted_token [T*k], slot_of [T*k])."""
+    _check_cuda(indices)
+    cfg = shape.cfg()
+    T = indices.shape[0]
+    dev = indices.device
+    counts = torch.empty(shape.n_routed, dtype=torch.int32, device=dev)
+    offsets = torch.empty(shape.n_routed + 1, dtype=torch.int32, device=dev)
+    sorted_token = torch.empty(T * shape.topk, dtype=torch.int32, device=dev)
+    slot_of = torch.empty(T * shape.topk, dtype=torch.int32, device=dev)
+    need = fn("moe_dispatch", "moe_dispatch_workspace_size")(ctypes.byref(cfg), T)
+    if ws is None or ws.numel() < need:
+        ws = _ws(need, dev)
+    st = fn("moe_dispatch", "moe_dispatch_build")(
+        ctypes.byref(cfg), T, indices.data_ptr(), counts.data_ptr(), offsets.data_ptr(),
+        sorted_token.data_ptr(), slot_of.data_ptr(), ws.data_ptr(), ws.numel(), _ptr(status),
+        _stream())
+    check(st, "moe_dispatch_build")
+    return counts, offsets, sorted_token, slot_of
+
+
+def expert_weights_struct(w1, w3, w2, s1=None, s3=None, s2=None) -> MoEExpertWeights:
+    _check_cuda(w1, w3, w2, s1, s3, s2)
+    return MoEExpertWeights(w1.data_ptr(), w3.data_ptr(), w2.data_ptr(), _dt(w1), _ptr(s1),
+                            _ptr(s3), _ptr(s2))
+
+
+def experts_forward(shape: BlockShape, x: torch.Tensor, wstruct: MoEExpertWeights,
+                    offsets: torch.Tensor, sorted_token: torch.Tensor, *, out_perm=None,
+                    out_shared=None, ws=None, status=None):
+    """moe_experts_forward: (out_perm [T*k, dim] fp32, out_shared [T, dim] fp32 or None)."""
+    _check_cuda(x, offsets, sorted_token)
+    cfg = shape.cfg()
+    T = x.shape[0]
+    dev = x.device
+    if out_perm is None:
+        out_perm = torch.empty(T * shape.topk, shape.dim, dtype=torch.float32, device=dev)
+    if out_shared is None and shape.n_shared:
+        out_shared = torch.empty(T, shape.dim, dtype=torch.float32, device=dev)
+    need = fn("moe_experts", "moe_experts_workspace_size")(ctypes.byref(cfg), T, _dt(x),
+                                                            wstruct.w_dt)
+    if ws is None or ws.numel() < need:
+        ws = _ws(need, dev)
+    st = fn("moe_experts", "moe_experts_forward")(
+        ctypes.byref(cfg), T, x.data_ptr(), _dt(x), ctypes.byref(wstruct), offsets.data_ptr(),
+        sorted_token.data_ptr(), out_perm.data_ptr(), _ptr(out_shared), ws.data_ptr(),
+        ws.numel(), _ptr(status), _stream())
+    check(st, "moe_experts_forward")
+    return out_perm, out_shared
+
+
+def combine(shape: BlockShape, weights: torch.Tensor, slot_of: torch.Tensor,
+            out_perm: torch.Tensor, out_shared: Optional[torch.Tensor], *, y=None, status=None):
+    """moe_combine: y [T, dim] fp32."""
+    _check_cuda(weights, slot_of, out_perm, out_shared)
+    cfg = shape.cfg()
+    T = weights.shape[0]
+    if y is None:
+        y = torch.empty(T, shape.dim, dtype=torch.float32, device=weights.device)
+    st = fn("moe_combine", "moe_combine")(
+        ctypes.byref(cfg), T, weights.data_ptr(), slot_of.data_ptr(), out_perm.data_ptr(),
+        _ptr(out_shared), y.data_ptr(), _ptr(status), _stream())
+    check(st, "moe_combine")
+    return y
+
+
+def selftest_wait(limit_ns: int, status: torch.Tensor) -> None:
+    check(fn("moe_experts", "moe_experts_selftest_wait")(limit_ns, status.data_ptr(), _stream()),
+          "moe_experts_selftest_wait")
+
+
+# ------------------------------------------------------------- the block
+
+
+@dataclass
+class BlockParams:
+    """Device tensors of one block.  w1/w3 [E+S, I, D], w2 [E+S, D, I]
+    (bf16, fp32, or e4m3 codes as uint8 with s1/s3/s2 block scales)."""
+
+    w_r: torch.Tensor
+    bias: Optional[torch.Tensor]
+    w1: torch.Tensor
+    w3: torch.Tensor
+    w2: torch.Tensor
+    s1: Optional[torch.Tensor] = None
+    s3: Optional[torch.Tensor] = None
+    s2: Optional[torch.Tensor] = None
+
+
+class MoEBlock:
+    """One MoE block with its workspaces, for repeated forwards on a fixed T.
+
+    forward() enqueues router -> dispatch -> experts -> combine on the current
+    stream with no host synchronisation; all buffers are preallocated, so the
+    call can be captured in a CUDA graph.
+    """
+
+    def __init__(self, shape: BlockShape, params: BlockParams, T: int, x_dtype: torch.dtype,
+                 device=None):
+        self.shape, self.p, self.T = shape, params, T
+        dev = torch.device(device or params.w1.device)
+        self.cfg = shape.cfg()
+        k, D = shape.topk, shape.dim
+        self.wstruct = expert_weights_struct(params.w1, params.w3, params.w2, params.s1,
+                                             params.s3, params.s2)
+        cfgp = ctypes.byref(self.cfg)
+        x_dt = _lib.DTYPES[_TORCH_DT[x_dtype]]
+        self.ws_router = _ws(fn("moe_router", "moe_router_workspace_size")(cfgp, T), dev)
+        self.ws_dispatch = _ws(fn("moe_dispatch", "moe_dispatch_workspace_size")(cfgp, T), dev)
+        self.ws_experts = _ws(fn("moe_experts", "moe_experts_workspace_size")(
+            cfgp, T, x_dt, self.wstruct.w_dt), dev)
+        f32, i32 = torch.float32, torch.int32
+        self.weights = torch.empty(T, k, dtype=f32, device=dev)
+        self.indices = torch.empty(T, k, dtype=i32, device=dev)
+        self.sel_gap = torch.empty(T, dtype=f32, device=dev)
+        self.counts = torch.empty(shape.n_routed, dtype=i32, device=dev)
+        self.offsets = torch.empty(shape.n_routed + 1, dtype=i32, device=dev)
+        self.sorted_token = torch.empty(T * k, dtype=i32, device=dev)
+        self.slot_of = torch.empty(T * k, dtype=i32, device=dev)
+        self.out_perm = torch.empty(T * k, D, dtype=f32, device=dev)
+        self.out_shared = torch.empty(T, D, dtype=f32, device=dev) if shape.n_shared else None
+        self.y = torch.empty(T, D, dtype=f32, device=dev)
+        self.status = torch.zeros(1, dtype=i32, device=dev)
+
+    def forward(self, x: torch.Tensor) -> torch.Tensor:
+        """Enqueue the four libraries for x [T, dim]; returns self.y (fp32)."""
+        assert x.shape == (self.T, self.shape.dim) and x.is_cuda and x.is_contiguous()
+        cfgp = ctypes.byref(self.cfg)
+        s = _stream()
+        T, st = self.T, self.status.data_ptr()
+        p = self.p
+        check(fn("moe_router", "moe_router_forward")(
+            cfgp, T, x.data_ptr(), _dt(x), p.w_r.data_ptr(), _ptr(p.bias),
+            self.weights.data_ptr(), self.indices.data_ptr(), self.sel_gap.data_ptr(),
+            self.ws_router.data_ptr(), self.ws_router.numel(), st, s), "moe_router_forward")
+        check(fn("moe_dispatch", "moe_dispatch_build")(
+            cfgp, T, self.indices.data_ptr(), self.counts.data_ptr(), self.offsets.data_ptr(),
+            self.sorted_token.data_ptr(), self.slot_of.data_ptr(), self.ws_dispatch.data_ptr(),
+            self.ws_dispatch.numel(), st, s), "moe_dispatch_build")
+        check(fn("moe_experts", "moe_experts_forward")(
+            cfgp, T, x.data_ptr(), _dt(x), ctypes.byref(self.wstruct), self.offsets.data_ptr(),
+            self.sorted_token.data_ptr(), self.out_perm.data_ptr(), _ptr(self.out_shared),
+            self.ws_experts.data_ptr(), self.ws_experts.numel(), st, s), "moe_experts_forward")
+        check(fn("moe_combine", "moe_combine")(
+            cfgp, T, self.weights.data_ptr(), self.slot_of.data_ptr(), self.out_perm.data_ptr(),
+            _ptr(self.out_shared), self.y.data_ptr(), st, s), "moe_combine")
+        return self.y
+
+    def device_status(self) -> int:
+        """The first device-side error of the forwards so far (0 = none); syncs."""
+        return int(self.status.item())
