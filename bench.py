@@ -1,0 +1,391 @@
+#!/usr/bin/env python
+"""Throughput of the DeepSeek-V3 MoE block forward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+    python bench.py --impl reference ...      # the CPU oracle on the host cores
+
+One step = one forward of the whole block (router -> dispatch -> experts ->
+combine) over one batch of T tokens with inputs already resident in HBM.
+Prints one JSON line on rank 0.  Multi-GPU runs (torchrun) are independent
+replicas: every rank runs its own batch through its own copy of the weights
+(weak scaling); the time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+from datetime import timedelta
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from sparse_moe_layer_sum_b200 import moe  # noqa: E402
+from sparse_moe_layer_sum_b200.inputs import WORKLOADS, make_block, sample_tokens  # noqa: E402
+from sparse_moe_layer_sum_b200.roofline import block_work, kernel_work, load_peaks  # noqa: E402
+
+METRIC = "MoE block tokens/s (V3 shape, bf16, T=4096) and % of roofline on 1 B200"
+N_X_BATCHES = 4  # rotating input batches: with the 22.6 GB of weights, > L2 per step
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="v3_prefill_t4096", choices=sorted(WORKLOADS))
+    ap.add_argument("--cpu-sample", type=int, default=8,
+                    help="tokens the oracle pushes through the block for cpu_baseline")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def dist_env():
+    return (int(os.environ.get("RANK", 0)), int(os.environ.get("LOCAL_RANK", 0)),
+            int(os.environ.get("WORLD_SIZE", 1)))
+
+
+# ---------------------------------------------------------------- clocks
+
+
+class ClockSampler:
+    """nvidia-smi samples every 200 ms of this process's GPU while running."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device: int):
+        self.proc = None
+        self.path = None
+        try:
+            try:
+                props = torch.cuda.get_device_properties(device)
+                sel = (f"--id={props.pci_domain_id:08X}:{props.pci_bus_id:02X}:"
+                       f"{props.pci_device_id:02X}.0")
+            except AttributeError:
+                vis = os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",")
+                sel = f"--id={vis[device] if device < len(vis) and vis[device] else device}"
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", sel, f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:  # no nvidia-smi: clocks reported as unavailable
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) == 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(rows)}
+
+
+# ---------------------------------------------------------------- oracle leg
+
+
+def cpu_oracle_tokens_per_s(w, x, params, n_tokens: int, seed: int = 7):
+    """Time the oracle (as it stands) on a seeded sample of the workload's
+    tokens: routing and the block output of each sampled token.  Host copies
+    of the expert weights are fetched outside the timed part."""
+    from oracle import moe_oracle as O
+    from threadpoolctl import threadpool_info
+
+    toks = sample_tokens(w.T, n_tokens, seed).numpy()
+    xs = x[torch.from_numpy(toks).to(x.device)].float().cpu().numpy()
+    w_r = params.w_r.cpu().numpy()
+    bias = None if params.bias is None else params.bias.cpu().numpy()
+    b = w.shape
+    shape = O.MoEShape(dim=b.dim, n_routed_experts=b.n_routed, n_expert_groups=b.n_groups,
+                       n_limited_groups=b.topk_groups, n_activated_experts=b.topk,
+                       moe_inter_dim=b.inter, n_shared_experts=b.n_shared,
+                       route_scale=b.route_scale, score_func=b.score_func, has_bias=b.has_bias)
+    fetch_s = 0.0
+
+    def fetch(e):
+        nonlocal fetch_s
+        t0 = time.perf_counter()
+        mats = []
+        for wt, sc in ((params.w1, params.s1), (params.w3, params.s3), (params.w2, params.s2)):
+            if w.w_format == "e4m3":
+                mats.append(O.dequant_e4m3_block(wt[e].cpu().numpy(), sc[e].cpu().numpy()))
+            else:
+                mats.append(wt[e].float().cpu().numpy())
+        fetch_s += time.perf_counter() - t0
+        return mats
+
+    act = "bf16" if w.x_dtype == torch.bfloat16 else "f32"
+    t0 = time.perf_counter()
+    route = O.router(xs, w_r, bias, shape)
+    O.moe_forward(xs, route, fetch, lambda: fetch(shape.n_routed_experts),
+                  shape.n_routed_experts, act)
+    wall = time.perf_counter() - t0 - fetch_s
+    cores = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    return len(toks) / wall, cores, wall
+
+
+# ---------------------------------------------------------------- ours
+
+
+def traffic_for(kernel_name: str):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken
+    on the current kernel source (else None)."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            t = json.load(f)
+    except (OSError, ValueError):
+        return None
+    h = hashlib.sha256()
+    for rel in t.get("sources", []):
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    if h.hexdigest() != t.get("sha256"):
+        return None
+    entry = t.get("kernels", {}).get(kernel_name)
+    if not entry or entry.get("workload") != t.get("bench_workload"):
+        return None
+    return entry.get("dram_bytes_per_launch")
+
+
+def run_ours(args, rank, local_rank, world):
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    from sparse_moe_layer_sum_b200 import build
+    build.build_all()
+    w = WORKLOADS[args.workload]
+    sh = w.shape
+    x0, params = make_block(w, dev, x_seed_offset=1 + rank * N_X_BATCHES)
+    xs = [x0]
+    gx = torch.Generator(device=dev)
+    for i in range(1, N_X_BATCHES):
+        gx.manual_seed(w.seed + 104729 * (1 + rank * N_X_BATCHES + i))
+        xs.append(torch.randn(w.T, sh.dim, generator=gx, device=dev).to(w.x_dtype))
+    blk = moe.MoEBlock(sh, params, w.T, w.x_dtype, device=dev)
+
+    for i in range(max(args.warmup, 1)):
+        blk.forward(xs[i % N_X_BATCHES])
+    torch.cuda.synchronize()
+    st = blk.device_status()
+    if st != 0:
+        raise RuntimeError(f"device status {st} after warm-up")
+
+    K = args.steps
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(10)] for _ in range(K)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    counts = []
+    for i in range(N_X_BATCHES):   # routing of each input batch, for the byte counts
+        blk.forward(xs[i])
+        counts.append(blk.counts.cpu())
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local_rank)
+    time.sleep(0.25)
+    start.record()
+    for i in range(K):
+        blk.forward_profiled(xs[i % N_X_BATCHES], evs[i])
+    end.record()
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    if world > 1:
+        torch.distributed.barrier()
+    ms_total = start.elapsed_time(end)
+    if world > 1:
+        t = torch.tensor([ms_total], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms_total = float(t.item())
+    if blk.device_status() != 0:
+        raise RuntimeError(f"device status {blk.device_status()} in the timed region")
+    ms_step = ms_total / K
+    value = world * w.T * K / (ms_total / 1e3)
+
+    # per-kernel durations inside the timed region
+    spans = {"router": (0, 1), "dispatch": (1, 2), "gather": (3, 4), "gemm1": (4, 5),
+             "gemm2": (6, 7), "combine": (8, 9)}
+    dur = {k: statistics.mean(evs[i][a].elapsed_time(evs[i][b]) for i in range(K))
+           for k, (a, b) in spans.items()}
+    peaks, peak_src = load_peaks(ROOT)
+    w_bytes = {"bf16": 2, "f32": 4, "e4m3": 1}[w.w_format]
+    x_bytes = 2 if w.x_dtype == torch.bfloat16 else 4
+    scale_b = (3 * (sh.dim // 128) * (sh.inter // 128) * 4) if w.w_format == "e4m3" else 0
+    touched = [int((c > 0).sum()) for c in counts]
+    kw = [kernel_work(sh.dim, sh.n_routed, sh.inter, sh.topk, sh.n_shared, w.T, n, w_bytes,
+                      x_bytes, scale_b) for n in touched]
+    bw = [block_work(sh.dim, sh.n_routed, sh.inter, sh.topk, sh.n_shared, w.T, n, w_bytes,
+                     x_bytes, scale_b, sh.has_bias) for n in touched]
+    steps_per_batch = [sum(1 for i in range(K) if i % N_X_BATCHES == b) for b in range(N_X_BATCHES)]
+
+    def avg(f):
+        return sum(f(b) * steps_per_batch[b] for b in range(N_X_BATCHES)) / K
+
+    dominant = max(("gemm1", "gemm2", "router", "combine", "gather", "dispatch"), key=dur.get)
+    bytes_dom = avg(lambda b: kw[b][dominant].bytes)
+    flops_dom = avg(lambda b: kw[b][dominant].flops)
+    hbm, tflops = peaks["hbm_gbs"], peaks["bf16_tflops"]
+    t_hbm = bytes_dom / (hbm * 1e9)
+    t_tc = flops_dom / (tflops * 1e12)
+    dsec = dur[dominant] / 1e3
+    kname = {"gemm1": "tc_expert_gemm<1>", "gemm2": "tc_expert_gemm<2>"}.get(dominant, dominant)
+    if t_hbm >= t_tc:
+        roof = {"bound": "hbm", "achieved": bytes_dom / dsec / 1e9, "peak": hbm, "unit": "GB/s"}
+    else:
+        roof = {"bound": "tensor", "achieved": flops_dom / dsec / 1e12, "peak": tflops,
+                "unit": "TFLOP/s"}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    roof["traffic"] = traffic_for(kname)
+    roof["kernel"] = kname
+    roof["peak_source"] = f"{peak_src} ({'MEASURED_PEAKS.json' if peak_src == 'measured' else 'recipe fallback'})"
+    roof["algorithmic_bytes_per_launch"] = bytes_dom
+    roof["algorithmic_flops_per_launch"] = flops_dom
+    b_alg = avg(lambda b: bw[b].bytes)
+    f_alg = avg(lambda b: bw[b].flops)
+    t_roof = max(b_alg / (hbm * 1e9), f_alg / (tflops * 1e12))
+    step_roof = {"bytes": b_alg, "flops": f_alg, "t_roof_ms": t_roof * 1e3,
+                 "frac": t_roof * 1e3 / ms_step,
+                 "bound": "hbm" if b_alg / (hbm * 1e9) >= f_alg / (tflops * 1e12) else "tensor",
+                 "hbm_frac_vs_nominal_8TBs": b_alg / (ms_step / 1e3) / 8e12}
+
+    # end to end through the public API from pinned host memory
+    x_host = [xx.cpu().pin_memory() for xx in xs]
+    y_host = torch.empty(w.T, sh.dim, dtype=torch.float32).pin_memory()
+    x_dev = torch.empty_like(xs[0])
+    Ke = max(1, min(K, 50))
+    for i in range(2):
+        blk.forward_host(x_host[i % N_X_BATCHES], y_host, x_dev)
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for i in range(Ke):
+        blk.forward_host(x_host[i % N_X_BATCHES], y_host, x_dev)
+    e1.record()
+    torch.cuda.synchronize()
+    ms_e2e = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([ms_e2e], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms_e2e = float(t.item())
+    e2e = {"value": world * w.T * Ke / (ms_e2e / 1e3), "unit": "tokens/s",
+           "h2d_bytes_per_step": w.T * sh.dim * x_bytes, "d2h_bytes_per_step": w.T * sh.dim * 4,
+           "steps": Ke}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        try:
+            tps, cores, wall = cpu_oracle_tokens_per_s(w, x0, params, args.cpu_sample)
+            cpu = {"value": tps, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                   "sample": f"{args.cpu_sample} seeded tokens of the {w.name} batch: fp64 "
+                             f"routing and block output ({wall:.1f} s of oracle time; weight "
+                             "copies to the host excluded)"}
+        except Exception as exc:  # reported, never fatal
+            cpu = {"value": None, "error": repr(exc)[:200]}
+
+    hot = None
+    if w.hot_experts:
+        hot_ids = torch.randperm(sh.n_routed, generator=torch.Generator().manual_seed(2024))[:16]
+        hot = float(counts[0][hot_ids].sum() / counts[0].sum())
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16" if w.w_format != "f32" else "f32",
+        "data": "synthetic (seeded N(0,1) activations, N(0,1/fan_in) weights, U(-0.1,0.1) bias)",
+        "config": {"workload": w.name, "T": w.T, "dim": sh.dim, "n_routed": sh.n_routed,
+                   "topk": sh.topk, "inter": sh.inter, "weights": w.w_format,
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                   "l2": f"inputs larger than L2: {N_X_BATCHES} rotating x batches and "
+                         f"{(sh.n_routed + 1) * 3 * sh.dim * sh.inter * w_bytes / 1e9:.1f} GB "
+                         "of expert weights per step"},
+        "roofline": roof, "step_roofline": step_roof,
+        "kernels_ms": dur, "cpu_baseline": cpu, "e2e": e2e,
+        "gpu_launches": K * moe.MoEBlock.LAUNCHES_PER_FORWARD,
+        "clocks": clk, "touched_experts": touched, "hot_share": hot,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------- reference
+
+
+def run_reference(args, rank, world):
+    """The oracle, timed on the host cores on the same workload (one seeded
+    token per step, routed and pushed through its experts in fp64)."""
+    if rank != 0:
+        return
+    w = WORKLOADS[args.workload]
+    dev = torch.device("cuda", 0) if torch.cuda.is_available() else torch.device("cpu")
+    x, params = make_block(w, dev, x_seed_offset=1)
+    K, W = args.steps, args.warmup
+    per_step = 1
+    times = []
+    cores = 1
+    for i in range(W + K):
+        _, cores, wall = cpu_oracle_tokens_per_s(w, x, params, per_step, seed=1000 + i)
+        if i >= W:
+            times.append(wall)
+    ms = 1e3 * sum(times) / len(times)
+    value = per_step / (ms / 1e3)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": K, "warmup": W, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "T": w.T, "weights": w.w_format},
+        "cpu_baseline": {"kind": "oracle", "cores": cores, "value": value, "unit": "tokens/s",
+                         "sample": f"{per_step} seeded token per step of the {w.name} batch"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    rank, local_rank, world = dist_env()
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+    if world > 1:
+        torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group("nccl", timeout=timedelta(seconds=300),
+                                             device_id=torch.device("cuda", local_rank))
+    try:
+        run_ours(args, rank, local_rank, world)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

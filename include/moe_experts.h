@@ -66,6 +66,35 @@ moe_status moe_experts_forward(const moe_cfg *cfg, int64_t T, const void *x, moe
                                moe_stream_t stream);
 
 /*
+ * The two halves of moe_experts_forward, for callers that schedule them
+ * separately (moe_experts_forward(...) == moe_experts_up(...) followed by
+ * moe_experts_down(...) on the same stream and workspace).
+ *   moe_experts_up    gathers the expert-contiguous rows and computes
+ *                     h = round_act(silu(x w1^T) * (x w3^T)) for every row
+ *                     into the workspace
+ *   moe_experts_down  reads h from the workspace that moe_experts_up filled
+ *                     (same cfg, T, dtypes and offsets) and writes out_perm and
+ *                     out_shared
+ */
+moe_status moe_experts_up(const moe_cfg *cfg, int64_t T, const void *x, moe_dtype x_dt,
+                          const moe_expert_weights *w, const int32_t *offsets,
+                          const int32_t *sorted_token, void *ws, size_t ws_bytes,
+                          int32_t *dev_status, moe_stream_t stream);
+moe_status moe_experts_down(const moe_cfg *cfg, int64_t T, moe_dtype x_dt,
+                            const moe_expert_weights *w, const int32_t *offsets,
+                            float *out_perm, float *out_shared, void *ws, size_t ws_bytes,
+                            int32_t *dev_status, moe_stream_t stream);
+
+/*
+ * Profiling: register up to five caller-owned cudaEvent_t handles that later
+ * calls record on their stream: [0] before the row gather, [1] before the
+ * first GEMM, [2] after it, [3] before the second GEMM, [4] after it.  n = 0
+ * stops the recording.  Process-wide and not thread-safe; meant for
+ * benchmarks.  Returns MOE_ERR_INVALID for n outside [0, 5].
+ */
+moe_status moe_experts_set_profile_events(void *const *events, int32_t n);
+
+/*
  * Self-test of the bounded pipeline wait used by the tensor-core kernels:
  * one CTA waits on a barrier that nothing signals, with a limit of
  * `limit_ns` nanoseconds, then writes MOE_ERR_TIMEOUT to dev_status and

@@ -641,123 +641,244 @@ moe_status launch_tc(const CUtensorMap &a0, const CUtensorMap &a1, const CUtenso
   return launch_status();
 }
 
+// Optional profiling events (caller-owned cudaEvent_t), recorded on the call's
+// stream around the kernels of the experts: [0] before the gather, [1] before
+// GEMM1, [2] after GEMM1, [3] before GEMM2, [4] after GEMM2.
+cudaEvent_t g_prof[5] = {nullptr, nullptr, nullptr, nullptr, nullptr};
+int g_nprof = 0;
+
+void prof(int i, cudaStream_t s) {
+  if (i < g_nprof && g_prof[i]) cudaEventRecord(g_prof[i], s);
+}
+
+struct Job {
+  const moe_cfg *c;
+  int64_t T;
+  const void *x;
+  moe_dtype x_dt;
+  const moe_expert_weights *w;
+  const int32_t *offsets;
+  const int32_t *sorted_token;
+  float *out_perm;
+  float *out_shared;
+  uint8_t *ws;
+  WsLayout l;
+  int32_t *status;
+  cudaStream_t s;
+
+  int E() const { return c->n_routed; }
+  int G() const { return c->n_routed + c->n_shared; }
+  int rows_routed() const { return (int)(T * c->topk); }
+  int rows_total() const { return (int)(T * c->topk + T * c->n_shared); }
+  int32_t *tab() const { return reinterpret_cast<int32_t *>(ws + l.tab); }
+};
+
+tc::Params tc_params(const Job &j) {
+  tc::Params p;
+  p.offsets = j.offsets;
+  p.E = j.E();
+  p.G = j.G();
+  p.T = (int)j.T;
+  p.I = j.c->inter;
+  p.D = j.c->dim;
+  p.rows_routed = j.rows_routed();
+  p.out_shared = j.out_shared;
+  p.status = j.status;
+  p.timeout_ns = 1000000000LL;
+  return p;
+}
+
 template <int BN_MAX, int BOXN, int STAGES>
-moe_status run_tc(const moe_cfg *c, int64_t T, const void *x, const moe_expert_weights *w,
-                  const int32_t *offsets, const int32_t *sorted_token, float *out_perm,
-                  float *out_shared, uint8_t *ws, const WsLayout &l, int32_t *dev_status,
-                  cudaStream_t s) {
-  const int E = c->n_routed, G = c->n_routed + c->n_shared, D = c->dim, I = c->inter;
-  const int rows_routed = (int)(T * c->topk);
-  const int rows_total = rows_routed + (int)(T * c->n_shared);
-  int32_t *tab = reinterpret_cast<int32_t *>(ws + l.tab);
+moe_status tc_up(const Job &j) {
+  const int G = j.G(), D = j.c->dim, I = j.c->inter;
+  int32_t *tab = j.tab();
   Tiling t1{BN_MAX, I / 64, tab, tab + (G + 1)};
-  Tiling t2{BN_MAX, D / tc::BM, tab + (2 * G + 1), tab + (3 * G + 2)};
-  prep_tiles<<<1, 32, 0, s>>>(offsets, E, G, (int)T, t1, t2);
+  Tiling none{0, 0, nullptr, nullptr};
+  prep_tiles<<<1, 32, 0, j.s>>>(j.offsets, j.E(), G, (int)j.T, t1, none);
   moe_status st = launch_status();
   if (st != MOE_OK) return st;
-
-  bf16 *xperm = reinterpret_cast<bf16 *>(ws + l.xperm);
-  bf16 *h = reinterpret_cast<bf16 *>(ws + l.h);
-  {
-    const int vec = D * 2 / 16;
-    const int64_t threads = (int64_t)rows_total * 32;
-    gather_rows<<<(unsigned)((threads + 255) / 256), 256, 0, s>>>(
-        static_cast<const uint4 *>(x), sorted_token, reinterpret_cast<uint4 *>(xperm),
-        rows_routed, rows_total, (int)T, vec);
-    if ((st = launch_status()) != MOE_OK) return st;
-  }
-  CUtensorMap mw1, mw3, mw2, mx, mh;
+  bf16 *xperm = reinterpret_cast<bf16 *>(j.ws + j.l.xperm);
+  bf16 *h = reinterpret_cast<bf16 *>(j.ws + j.l.h);
+  prof(0, j.s);
+  const int64_t threads = (int64_t)j.rows_total() * 32;
+  gather_rows<<<(unsigned)((threads + 255) / 256), 256, 0, j.s>>>(
+      static_cast<const uint4 *>(j.x), j.sorted_token, reinterpret_cast<uint4 *>(xperm),
+      j.rows_routed(), j.rows_total(), (int)j.T, D * 2 / 16);
+  if ((st = launch_status()) != MOE_OK) return st;
+  CUtensorMap mw1, mw3, mx;
   const CUtensorMapDataType BF = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
-  if (!make_tmap(&mw1, w->w1, BF, 2, (uint64_t)G * I, D, 64, 64) ||
-      !make_tmap(&mw3, w->w3, BF, 2, (uint64_t)G * I, D, 64, 64) ||
-      !make_tmap(&mw2, w->w2, BF, 2, (uint64_t)G * D, I, tc::BM, 64) ||
-      !make_tmap(&mx, xperm, BF, 2, (uint64_t)l.rows_pad, D, BOXN, 64) ||
-      !make_tmap(&mh, h, BF, 2, (uint64_t)l.rows_pad, I, BOXN, 64))
+  if (!make_tmap(&mw1, j.w->w1, BF, 2, (uint64_t)G * I, D, 64, 64) ||
+      !make_tmap(&mw3, j.w->w3, BF, 2, (uint64_t)G * I, D, 64, 64) ||
+      !make_tmap(&mx, xperm, BF, 2, (uint64_t)j.l.rows_pad, D, BOXN, 64))
     return MOE_ERR_CUDA;
-
-  tc::Params p;
-  p.offsets = offsets;
-  p.E = E;
-  p.G = G;
-  p.T = (int)T;
-  p.I = I;
-  p.D = D;
-  p.rows_routed = rows_routed;
-  p.out_shared = out_shared;
-  p.status = dev_status;
-  p.timeout_ns = 1000000000LL;
-
+  tc::Params p = tc_params(j);
   p.tile_start = t1.tile_start;
   p.tile_base = t1.tile_base;
   p.KB = D / tc::BK;
   p.out = h;
-  if ((st = launch_tc<1, BN_MAX, BOXN, STAGES>(mw1, mw3, mx, p, s)) != MOE_OK) return st;
+  prof(1, j.s);
+  st = launch_tc<1, BN_MAX, BOXN, STAGES>(mw1, mw3, mx, p, j.s);
+  prof(2, j.s);
+  return st;
+}
 
+template <int BN_MAX, int BOXN, int STAGES>
+moe_status tc_down(const Job &j) {
+  const int G = j.G(), D = j.c->dim, I = j.c->inter;
+  int32_t *tab = j.tab();
+  Tiling t2{BN_MAX, D / tc::BM, tab + (2 * G + 1), tab + (3 * G + 2)};
+  Tiling none{0, 0, nullptr, nullptr};
+  prep_tiles<<<1, 32, 0, j.s>>>(j.offsets, j.E(), G, (int)j.T, t2, none);
+  moe_status st = launch_status();
+  if (st != MOE_OK) return st;
+  bf16 *h = reinterpret_cast<bf16 *>(j.ws + j.l.h);
+  CUtensorMap mw2, mh;
+  const CUtensorMapDataType BF = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  if (!make_tmap(&mw2, j.w->w2, BF, 2, (uint64_t)G * D, I, tc::BM, 64) ||
+      !make_tmap(&mh, h, BF, 2, (uint64_t)j.l.rows_pad, I, BOXN, 64))
+    return MOE_ERR_CUDA;
+  tc::Params p = tc_params(j);
   p.tile_start = t2.tile_start;
   p.tile_base = t2.tile_base;
   p.KB = I / tc::BK;
-  p.out = out_perm;
-  return launch_tc<2, BN_MAX, BOXN, STAGES>(mw2, mw2, mh, p, s);
+  p.out = j.out_perm;
+  prof(3, j.s);
+  st = launch_tc<2, BN_MAX, BOXN, STAGES>(mw2, mw2, mh, p, j.s);
+  prof(4, j.s);
+  return st;
 }
 
+SimtArgs simt_args(const Job &j, const Tiling &t) {
+  SimtArgs a;
+  a.offsets = j.offsets;
+  a.sorted_token = j.sorted_token;
+  a.E = j.E();
+  a.G = j.G();
+  a.T = (int)j.T;
+  a.D = j.c->dim;
+  a.I = j.c->inter;
+  a.rows_routed = j.rows_routed();
+  a.act_bf16 = j.x_dt == MOE_BF16;
+  a.h = reinterpret_cast<float *>(j.ws + j.l.h);
+  a.out_perm = j.out_perm;
+  a.out_shared = j.out_shared;
+  a.tile_start = t.tile_start;
+  a.tile_base = t.tile_base;
+  return a;
+}
+
+// upper bound on CUDA-core tiles: sum over groups of ceil(n_g / 16) times feature tiles
+int64_t simt_tile_bound(const Job &j, int ft) { return ((int64_t)j.rows_total() / 16 + j.G()) * ft; }
+
 template <typename XT, typename WT>
-moe_status run_simt_t(const moe_cfg *c, int64_t T, const void *x, const moe_expert_weights *w,
-                      const int32_t *offsets, const int32_t *sorted_token, float *out_perm,
-                      float *out_shared, uint8_t *ws, const WsLayout &l, int act_bf16,
-                      cudaStream_t s) {
-  const int E = c->n_routed, G = c->n_routed + c->n_shared, D = c->dim, I = c->inter;
-  int32_t *tab = reinterpret_cast<int32_t *>(ws + l.tab);
-  Tiling t1{ST, (I + ST - 1) / ST, tab, tab + (G + 1)};
-  Tiling t2{ST, (D + ST - 1) / ST, tab + (2 * G + 1), tab + (3 * G + 2)};
-  prep_tiles<<<1, 32, 0, s>>>(offsets, E, G, (int)T, t1, t2);
+moe_status simt_up(const Job &j) {
+  const int G = j.G();
+  int32_t *tab = j.tab();
+  Tiling t1{ST, (j.c->inter + ST - 1) / ST, tab, tab + (G + 1)};
+  Tiling none{0, 0, nullptr, nullptr};
+  prep_tiles<<<1, 32, 0, j.s>>>(j.offsets, j.E(), G, (int)j.T, t1, none);
   moe_status st = launch_status();
   if (st != MOE_OK) return st;
-  SimtArgs a;
-  a.offsets = offsets;
-  a.sorted_token = sorted_token;
-  a.E = E;
-  a.G = G;
-  a.T = (int)T;
-  a.D = D;
-  a.I = I;
-  a.rows_routed = (int)(T * c->topk);
-  a.act_bf16 = act_bf16;
-  a.h = reinterpret_cast<float *>(ws + l.h);
-  a.out_perm = out_perm;
-  a.out_shared = out_shared;
-  // upper bound on tiles: sum over groups of ceil(n_g / 16) times feature tiles
-  const int64_t rows = T * c->topk + T * c->n_shared;
-  const int64_t ub1 = (rows / 16 + G) * t1.ft, ub2 = (rows / 16 + G) * t2.ft;
-  a.tile_start = t1.tile_start;
-  a.tile_base = t1.tile_base;
-  simt_gemm1<XT, WT><<<(unsigned)ub1, 256, 0, s>>>(
-      static_cast<const XT *>(x), static_cast<const WT *>(w->w1), static_cast<const WT *>(w->w3),
-      w->w_dt == MOE_E4M3 ? w->s1 : nullptr, w->w_dt == MOE_E4M3 ? w->s3 : nullptr, a);
-  if ((st = launch_status()) != MOE_OK) return st;
-  a.tile_start = t2.tile_start;
-  a.tile_base = t2.tile_base;
-  simt_gemm2<WT><<<(unsigned)ub2, 256, 0, s>>>(static_cast<const WT *>(w->w2),
-                                               w->w_dt == MOE_E4M3 ? w->s2 : nullptr, a);
-  return launch_status();
+  const SimtArgs a = simt_args(j, t1);
+  const bool e4 = j.w->w_dt == MOE_E4M3;
+  prof(0, j.s);
+  prof(1, j.s);
+  simt_gemm1<XT, WT><<<(unsigned)simt_tile_bound(j, t1.ft), 256, 0, j.s>>>(
+      static_cast<const XT *>(j.x), static_cast<const WT *>(j.w->w1),
+      static_cast<const WT *>(j.w->w3), e4 ? j.w->s1 : nullptr, e4 ? j.w->s3 : nullptr, a);
+  st = launch_status();
+  prof(2, j.s);
+  return st;
+}
+
+template <typename WT>
+moe_status simt_down(const Job &j) {
+  const int G = j.G();
+  int32_t *tab = j.tab();
+  Tiling t2{ST, (j.c->dim + ST - 1) / ST, tab + (2 * G + 1), tab + (3 * G + 2)};
+  Tiling none{0, 0, nullptr, nullptr};
+  prep_tiles<<<1, 32, 0, j.s>>>(j.offsets, j.E(), G, (int)j.T, t2, none);
+  moe_status st = launch_status();
+  if (st != MOE_OK) return st;
+  const SimtArgs a = simt_args(j, t2);
+  prof(3, j.s);
+  simt_gemm2<WT><<<(unsigned)simt_tile_bound(j, t2.ft), 256, 0, j.s>>>(
+      static_cast<const WT *>(j.w->w2), j.w->w_dt == MOE_E4M3 ? j.w->s2 : nullptr, a);
+  st = launch_status();
+  prof(4, j.s);
+  return st;
 }
 
 template <typename XT>
-moe_status run_simt_x(const moe_cfg *c, int64_t T, const void *x, const moe_expert_weights *w,
-                      const int32_t *offsets, const int32_t *sorted_token, float *out_perm,
-                      float *out_shared, uint8_t *ws, const WsLayout &l, int act_bf16,
-                      cudaStream_t s) {
-  switch (w->w_dt) {
-    case MOE_F32:
-      return run_simt_t<XT, float>(c, T, x, w, offsets, sorted_token, out_perm, out_shared, ws, l,
-                                   act_bf16, s);
-    case MOE_BF16:
-      return run_simt_t<XT, bf16>(c, T, x, w, offsets, sorted_token, out_perm, out_shared, ws, l,
-                                  act_bf16, s);
-    case MOE_E4M3:
-      return run_simt_t<XT, __nv_fp8_e4m3>(c, T, x, w, offsets, sorted_token, out_perm,
-                                           out_shared, ws, l, act_bf16, s);
+moe_status simt_up_x(const Job &j) {
+  switch (j.w->w_dt) {
+    case MOE_F32: return simt_up<XT, float>(j);
+    case MOE_BF16: return simt_up<XT, bf16>(j);
+    case MOE_E4M3: return simt_up<XT, __nv_fp8_e4m3>(j);
   }
   return MOE_ERR_UNSUPPORTED;
+}
+
+moe_status simt_down_w(const Job &j) {
+  switch (j.w->w_dt) {
+    case MOE_F32: return simt_down<float>(j);
+    case MOE_BF16: return simt_down<bf16>(j);
+    case MOE_E4M3: return simt_down<__nv_fp8_e4m3>(j);
+  }
+  return MOE_ERR_UNSUPPORTED;
+}
+
+// few rows per expert (decode): narrow token tiles and a deep ring so that
+// enough weight bytes are in flight; otherwise token tiles of up to 256
+bool decode_variant(const Job &j) { return j.T * j.c->topk <= (int64_t)16 * j.c->n_routed; }
+
+moe_status run_up(const Job &j) {
+  if (tc_path(j.c, j.x_dt, j.w->w_dt))
+    return decode_variant(j) ? tc_up<32, 32, 10>(j) : tc_up<256, 32, 4>(j);
+  return j.x_dt == MOE_BF16 ? simt_up_x<bf16>(j) : simt_up_x<float>(j);
+}
+
+moe_status run_down(const Job &j) {
+  if (tc_path(j.c, j.x_dt, j.w->w_dt))
+    return decode_variant(j) ? tc_down<32, 32, 10>(j) : tc_down<256, 32, 4>(j);
+  return simt_down_w(j);
+}
+
+// Checks shared by the entry points; fills the job on success.
+moe_status make_job(Job &j, const moe_cfg *cfg, int64_t T, const void *x, moe_dtype x_dt,
+                    const moe_expert_weights *w, const int32_t *offsets,
+                    const int32_t *sorted_token, float *out_perm, float *out_shared, void *ws,
+                    size_t ws_bytes, int32_t *dev_status, moe_stream_t stream, bool need_up,
+                    bool need_down) {
+  moe_status st = check_cfg(cfg);
+  if (st != MOE_OK) return st;
+  if (T < 0 || (T * (int64_t)cfg->topk + T) >= ((int64_t)1 << 31)) return MOE_ERR_INVALID;
+  if (!w || !w->w1 || !w->w3 || !w->w2 || !offsets || !ws) return MOE_ERR_INVALID;
+  if (need_up && (!x || !sorted_token)) return MOE_ERR_INVALID;
+  if (need_down && !out_perm) return MOE_ERR_INVALID;
+  if (cfg->n_shared > 1) return MOE_ERR_UNSUPPORTED;
+  if (need_down && cfg->n_shared == 1 && !out_shared) return MOE_ERR_INVALID;
+  if (x_dt != MOE_F32 && x_dt != MOE_BF16) return MOE_ERR_UNSUPPORTED;
+  if (w->w_dt != MOE_F32 && w->w_dt != MOE_BF16 && w->w_dt != MOE_E4M3) return MOE_ERR_UNSUPPORTED;
+  if (w->w_dt == MOE_E4M3) {
+    if (!w->s1 || !w->s3 || !w->s2) return MOE_ERR_INVALID;
+    if (cfg->dim % 128 != 0 || cfg->inter % 128 != 0) return MOE_ERR_UNSUPPORTED;
+  }
+  j.l = ws_layout(cfg, T, x_dt, w->w_dt);
+  if (ws_bytes < j.l.total) return MOE_ERR_WORKSPACE;
+  j.c = cfg;
+  j.T = T;
+  j.x = x;
+  j.x_dt = x_dt;
+  j.w = w;
+  j.offsets = offsets;
+  j.sorted_token = sorted_token;
+  j.out_perm = out_perm;
+  j.out_shared = out_shared;
+  j.ws = static_cast<uint8_t *>(ws);
+  j.status = dev_status;
+  j.s = as_stream(stream);
+  return MOE_OK;
 }
 
 }  // namespace
@@ -771,45 +892,48 @@ MOE_EXPORT size_t moe_experts_workspace_size(const moe_cfg *cfg, int64_t T, moe_
   return ws_layout(cfg, T, x_dt, w_dt).total;
 }
 
+MOE_EXPORT moe_status moe_experts_up(const moe_cfg *cfg, int64_t T, const void *x, moe_dtype x_dt,
+                                     const moe_expert_weights *w, const int32_t *offsets,
+                                     const int32_t *sorted_token, void *ws, size_t ws_bytes,
+                                     int32_t *dev_status, moe_stream_t stream) {
+  Job j;
+  moe_status st = make_job(j, cfg, T, x, x_dt, w, offsets, sorted_token, nullptr, nullptr, ws,
+                           ws_bytes, dev_status, stream, true, false);
+  if (st != MOE_OK || T == 0) return st;
+  return run_up(j);
+}
+
+MOE_EXPORT moe_status moe_experts_down(const moe_cfg *cfg, int64_t T, moe_dtype x_dt,
+                                       const moe_expert_weights *w, const int32_t *offsets,
+                                       float *out_perm, float *out_shared, void *ws,
+                                       size_t ws_bytes, int32_t *dev_status,
+                                       moe_stream_t stream) {
+  Job j;
+  moe_status st = make_job(j, cfg, T, nullptr, x_dt, w, offsets, nullptr, out_perm, out_shared,
+                           ws, ws_bytes, dev_status, stream, false, true);
+  if (st != MOE_OK || T == 0) return st;
+  return run_down(j);
+}
+
 MOE_EXPORT moe_status moe_experts_forward(const moe_cfg *cfg, int64_t T, const void *x,
                                           moe_dtype x_dt, const moe_expert_weights *w,
                                           const int32_t *offsets, const int32_t *sorted_token,
                                           float *out_perm, float *out_shared, void *ws,
                                           size_t ws_bytes, int32_t *dev_status,
                                           moe_stream_t stream) {
-  moe_status st = check_cfg(cfg);
-  if (st != MOE_OK) return st;
-  if (T < 0 || (T * (int64_t)cfg->topk + T) >= ((int64_t)1 << 31)) return MOE_ERR_INVALID;
-  if (T == 0) return MOE_OK;
-  if (!x || !w || !w->w1 || !w->w3 || !w->w2 || !offsets || !sorted_token || !out_perm || !ws)
-    return MOE_ERR_INVALID;
-  if (cfg->n_shared > 1) return MOE_ERR_UNSUPPORTED;
-  if (cfg->n_shared == 1 && !out_shared) return MOE_ERR_INVALID;
-  if (x_dt != MOE_F32 && x_dt != MOE_BF16) return MOE_ERR_UNSUPPORTED;
-  if (w->w_dt != MOE_F32 && w->w_dt != MOE_BF16 && w->w_dt != MOE_E4M3) return MOE_ERR_UNSUPPORTED;
-  if (w->w_dt == MOE_E4M3) {
-    if (!w->s1 || !w->s3 || !w->s2) return MOE_ERR_INVALID;
-    if (cfg->dim % 128 != 0 || cfg->inter % 128 != 0) return MOE_ERR_UNSUPPORTED;
-  }
-  const WsLayout l = ws_layout(cfg, T, x_dt, w->w_dt);
-  if (ws_bytes < l.total) return MOE_ERR_WORKSPACE;
-  cudaStream_t s = as_stream(stream);
-  uint8_t *wsb = static_cast<uint8_t *>(ws);
-  if (tc_path(cfg, x_dt, w->w_dt)) {
-    // few rows per expert (decode): narrow token tiles and a deep ring so
-    // that enough weight bytes are in flight; otherwise up to 256 tokens
-    if (T * cfg->topk <= (int64_t)16 * cfg->n_routed)
-      return run_tc<32, 32, 10>(cfg, T, x, w, offsets, sorted_token, out_perm, out_shared, wsb,
-                                l, dev_status, s);
-    return run_tc<256, 32, 4>(cfg, T, x, w, offsets, sorted_token, out_perm, out_shared, wsb, l,
-                              dev_status, s);
-  }
-  const int act_bf16 = x_dt == MOE_BF16;
-  if (x_dt == MOE_BF16)
-    return run_simt_x<bf16>(cfg, T, x, w, offsets, sorted_token, out_perm, out_shared, wsb, l,
-                            act_bf16, s);
-  return run_simt_x<float>(cfg, T, x, w, offsets, sorted_token, out_perm, out_shared, wsb, l,
-                           act_bf16, s);
+  Job j;
+  moe_status st = make_job(j, cfg, T, x, x_dt, w, offsets, sorted_token, out_perm, out_shared,
+                           ws, ws_bytes, dev_status, stream, true, true);
+  if (st != MOE_OK || T == 0) return st;
+  if ((st = run_up(j)) != MOE_OK) return st;
+  return run_down(j);
+}
+
+MOE_EXPORT moe_status moe_experts_set_profile_events(void *const *events, int32_t n) {
+  if (n < 0 || n > 5 || (n > 0 && !events)) return MOE_ERR_INVALID;
+  for (int i = 0; i < 5; ++i) g_prof[i] = i < n ? static_cast<cudaEvent_t>(events[i]) : nullptr;
+  g_nprof = n;
+  return MOE_OK;
 }
 
 MOE_EXPORT moe_status moe_experts_selftest_wait(int64_t limit_ns, int32_t *dev_status,

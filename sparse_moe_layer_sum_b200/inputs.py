@@ -79,11 +79,10 @@ def make_block(w: Workload, device="cuda", x_seed_offset: int = 0):
     dev = torch.device(device)
     g = torch.Generator(device=dev).manual_seed(w.seed)
     D, E, I, S = sh.dim, sh.n_routed, sh.inter, sh.n_shared
-    if x_seed_offset:
+    x = torch.randn(w.T, D, generator=g, device=dev, dtype=torch.float32).to(w.x_dtype)
+    if x_seed_offset:  # another batch of the same distribution, same weights
         gx = torch.Generator(device=dev).manual_seed(w.seed + 7919 * x_seed_offset)
-    else:
-        gx = g
-    x = torch.randn(w.T, D, generator=gx, device=dev, dtype=torch.float32).to(w.x_dtype)
+        x = torch.randn(w.T, D, generator=gx, device=dev, dtype=torch.float32).to(w.x_dtype)
     w_r = torch.randn(E, D, generator=g, device=dev, dtype=torch.float32) / math.sqrt(D)
     bias = None
     if sh.has_bias:

@@ -212,29 +212,76 @@ class MoEBlock:
         self.y = torch.empty(T, D, dtype=f32, device=dev)
         self.status = torch.zeros(1, dtype=i32, device=dev)
 
+    # kernels one forward launches: router 2, dispatch 3, experts 5, combine 1
+    LAUNCHES_PER_FORWARD = 11
+
+    def _router(self, x, cfgp, s):
+        p = self.p
+        check(fn("moe_router", "moe_router_forward")(
+            cfgp, self.T, x.data_ptr(), _dt(x), p.w_r.data_ptr(), _ptr(p.bias),
+            self.weights.data_ptr(), self.indices.data_ptr(), self.sel_gap.data_ptr(),
+            self.ws_router.data_ptr(), self.ws_router.numel(), self.status.data_ptr(), s),
+            "moe_router_forward")
+
+    def _dispatch(self, cfgp, s):
+        check(fn("moe_dispatch", "moe_dispatch_build")(
+            cfgp, self.T, self.indices.data_ptr(), self.counts.data_ptr(),
+            self.offsets.data_ptr(), self.sorted_token.data_ptr(), self.slot_of.data_ptr(),
+            self.ws_dispatch.data_ptr(), self.ws_dispatch.numel(), self.status.data_ptr(), s),
+            "moe_dispatch_build")
+
+    def _experts(self, x, cfgp, s):
+        check(fn("moe_experts", "moe_experts_forward")(
+            cfgp, self.T, x.data_ptr(), _dt(x), ctypes.byref(self.wstruct),
+            self.offsets.data_ptr(), self.sorted_token.data_ptr(), self.out_perm.data_ptr(),
+            _ptr(self.out_shared), self.ws_experts.data_ptr(), self.ws_experts.numel(),
+            self.status.data_ptr(), s), "moe_experts_forward")
+
+    def _combine(self, cfgp, s):
+        check(fn("moe_combine", "moe_combine")(
+            cfgp, self.T, self.weights.data_ptr(), self.slot_of.data_ptr(),
+            self.out_perm.data_ptr(), _ptr(self.out_shared), self.y.data_ptr(),
+            self.status.data_ptr(), s), "moe_combine")
+
     def forward(self, x: torch.Tensor) -> torch.Tensor:
         """Enqueue the four libraries for x [T, dim]; returns self.y (fp32)."""
         assert x.shape == (self.T, self.shape.dim) and x.is_cuda and x.is_contiguous()
-        cfgp = ctypes.byref(self.cfg)
-        s = _stream()
-        T, st = self.T, self.status.data_ptr()
-        p = self.p
-        check(fn("moe_router", "moe_router_forward")(
-            cfgp, T, x.data_ptr(), _dt(x), p.w_r.data_ptr(), _ptr(p.bias),
-            self.weights.data_ptr(), self.indices.data_ptr(), self.sel_gap.data_ptr(),
-            self.ws_router.data_ptr(), self.ws_router.numel(), st, s), "moe_router_forward")
-        check(fn("moe_dispatch", "moe_dispatch_build")(
-            cfgp, T, self.indices.data_ptr(), self.counts.data_ptr(), self.offsets.data_ptr(),
-            self.sorted_token.data_ptr(), self.slot_of.data_ptr(), self.ws_dispatch.data_ptr(),
-            self.ws_dispatch.numel(), st, s), "moe_dispatch_build")
-        check(fn("moe_experts", "moe_experts_forward")(
-            cfgp, T, x.data_ptr(), _dt(x), ctypes.byref(self.wstruct), self.offsets.data_ptr(),
-            self.sorted_token.data_ptr(), self.out_perm.data_ptr(), _ptr(self.out_shared),
-            self.ws_experts.data_ptr(), self.ws_experts.numel(), st, s), "moe_experts_forward")
-        check(fn("moe_combine", "moe_combine")(
-            cfgp, T, self.weights.data_ptr(), self.slot_of.data_ptr(), self.out_perm.data_ptr(),
-            _ptr(self.out_shared), self.y.data_ptr(), st, s), "moe_combine")
+        cfgp, s = ctypes.byref(self.cfg), _stream()
+        self._router(x, cfgp, s)
+        self._dispatch(cfgp, s)
+        self._experts(x, cfgp, s)
+        self._combine(cfgp, s)
         return self.y
+
+    def forward_profiled(self, x: torch.Tensor, ev) -> torch.Tensor:
+        """forward() with 10 CUDA events recorded on the stream: around the
+        router [0,1], dispatch [1,2], the row gather [3,4], the two expert
+        GEMMs [4,5] and [6,7], and the combine [8,9]."""
+        cfgp, s = ctypes.byref(self.cfg), _stream()
+        ev[0].record()
+        self._router(x, cfgp, s)
+        ev[1].record()
+        self._dispatch(cfgp, s)
+        ev[2].record()
+        handles = (ctypes.c_void_p * 5)(*[e.cuda_event for e in ev[3:8]])
+        check(fn("moe_experts", "moe_experts_set_profile_events")(handles, 5), "profile events")
+        try:
+            self._experts(x, cfgp, s)
+        finally:
+            fn("moe_experts", "moe_experts_set_profile_events")(None, 0)
+        ev[8].record()
+        self._combine(cfgp, s)
+        ev[9].record()
+        return self.y
+
+    def forward_host(self, x_host: torch.Tensor, y_host: torch.Tensor, x_dev: torch.Tensor):
+        """End to end from host memory: copy x (pinned host) to the device,
+        run the block, copy y back into y_host (pinned), all on the current
+        stream; the caller synchronises."""
+        x_dev.copy_(x_host, non_blocking=True)
+        self.forward(x_dev)
+        y_host.copy_(self.y, non_blocking=True)
+        return y_host
 
     def device_status(self) -> int:
         """The first device-side error of the forwards so far (0 = none); syncs."""

@@ -1,0 +1,63 @@
+"""Algorithmic work of the MoE block and of each of its kernels.
+
+"Algorithmic" bytes are the bytes any implementation must move from or to
+HBM, and flops the multiply-adds it must do, given the routing (which experts
+received tokens).  Intermediate buffers an implementation chooses to keep in
+HBM (the permuted rows, h, the per-slot expert outputs) are counted only for
+the kernel that reads or writes them, never for the block as a whole.
+"""
+from __future__ import annotations
+
+import json
+import os
+from dataclasses import dataclass
+
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks(root: str) -> tuple[dict, str]:
+    """Measured peaks (MEASURED_PEAKS.json at the repo root), else the fallback."""
+    path = os.path.join(root, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+@dataclass
+class Work:
+    bytes: float
+    flops: float
+
+
+def block_work(D, E, I, k, S, T, n_touched, w_bytes, x_bytes, scale_bytes_per_expert=0.0,
+               has_bias=True) -> Work:
+    """Whole block: weights of the touched experts and the shared expert, the
+    fp32 router matrix and bias, x in and fp32 y out; expert and router flops."""
+    weights = (n_touched + S) * (3 * D * I * w_bytes + scale_bytes_per_expert)
+    router = E * D * 4 + (E * 4 if has_bias else 0)
+    io = T * D * x_bytes + T * D * 4
+    flops = T * (k + S) * 2 * 3 * D * I + T * 2 * D * E
+    return Work(weights + router + io, flops)
+
+
+def kernel_work(D, E, I, k, S, T, n_touched, w_bytes, x_bytes, scale_bytes_per_expert=0.0):
+    """Per kernel of one forward: the bytes it must move and flops it must do."""
+    rows = T * k + T * S                       # expert-contiguous rows incl. the shared expert
+    n_w = n_touched + S                        # weight matrices actually streamed
+    sc = scale_bytes_per_expert / 3.0          # per matrix
+    return {
+        "router": Work(E * D * 4 + E * 4 + T * D * x_bytes + T * k * 8, T * 2 * D * E),
+        "dispatch": Work(T * k * 4 * 3 + (E + 1) * 8, 0.0),
+        "gather": Work(T * k * D * x_bytes * 2 + T * D * x_bytes * 2, 0.0),
+        # W1 and W3 of each touched expert, the rows in, h out
+        "gemm1": Work(n_w * (2 * D * I * w_bytes + 2 * sc) + rows * D * 2 + rows * I * 2,
+                      rows * 2 * 2 * D * I),
+        # W2 of each touched expert, h in, fp32 expert outputs out
+        "gemm2": Work(n_w * (D * I * w_bytes + sc) + rows * I * 2 + rows * D * 4,
+                      rows * 2 * D * I),
+        # k expert rows and the shared row in, y out (all fp32)
+        "combine": Work(rows * D * 4 + T * D * 4 + T * k * 8, T * (k + S) * D * 2),
+    }
