@@ -51,6 +51,13 @@ WORKLOADS = {
     "v3_fp8_t8192": Workload("v3_fp8_t8192", BlockShape(**V3), 8192, torch.bfloat16, "e4m3", 1005,
                              note="T=8192, e4m3 expert weights with fp32 128x128 block scales, "
                                   "bf16 activations"),
+    # profiling-sized stand-in for the T=4096 prefill: same dim/inter and the
+    # same ~128 rows per expert, but 32 experts (2.9 GB of weights) so that a
+    # multi-pass ncu capture stays small
+    "prof_prefill_e32_t512": Workload("prof_prefill_e32_t512",
+                                      BlockShape(dim=7168, n_routed=32, n_groups=8, topk_groups=4,
+                                                 topk=8, inter=2048), 512, torch.bfloat16,
+                                      "bf16", 1006, note="V3 dims, 32 experts, T=512"),
 }
 
 

@@ -263,6 +263,8 @@ class MoEBlock:
         ev[1].record()
         self._dispatch(cfgp, s)
         ev[2].record()
+        for e in ev[3:8]:   # mark them recorded for torch; the library re-records them
+            e.record()
         handles = (ctypes.c_void_p * 5)(*[e.cuda_event for e in ev[3:8]])
         check(fn("moe_experts", "moe_experts_set_profile_events")(handles, 5), "profile events")
         try:
