@@ -184,13 +184,14 @@ struct Layout {
   static constexpr int XBUF_OFF = (MISC_OFF + MISC_BYTES + 127) / 128 * 128;
   static constexpr int XBUF_BYTES = MODE == 1 ? 2 * 2 * 32 * XB_STRIDE * 4 : 0;
   static constexpr int TAB_OFF = XBUF_OFF + XBUF_BYTES;
-  static constexpr uint32_t TMEM_COLS = 2 * BN_MAX < 32 ? 32 : 2 * BN_MAX;
+  static constexpr uint32_t TMEM_COLS =
+      2 * BN_MAX <= 32 ? 32 : 2 * BN_MAX <= 64 ? 64 : 2 * BN_MAX <= 128 ? 128
+                                                : 2 * BN_MAX <= 256 ? 256 : 512;
   static size_t smem_bytes(int G, int E) {
     return 1024 + TAB_OFF + sizeof(int32_t) * (size_t)((G + 1) + G + (E + 1));
   }
   static_assert(BN_MAX % 16 == 0 && BN_MAX >= 16 && BN_MAX <= 256, "MMA N range");
   static_assert(BOXN % 16 == 0 && BN_MAX % BOXN == 0, "B box rows");
-  static_assert((2 * BN_MAX & (2 * BN_MAX - 1)) == 0, "TMEM columns must be a power of two");
 };
 
 // Waits for a barrier phase with a time limit but ignores the abort flag;
@@ -828,19 +829,35 @@ moe_status simt_down_w(const Job &j) {
   return MOE_ERR_UNSUPPORTED;
 }
 
+// Tile shapes of the two instantiations (compile-time tunables).
+#ifndef MOE_TC_PREFILL_BN
+#define MOE_TC_PREFILL_BN 256
+#endif
+#ifndef MOE_TC_PREFILL_STAGES
+#define MOE_TC_PREFILL_STAGES 4
+#endif
+#ifndef MOE_TC_DECODE_BN
+#define MOE_TC_DECODE_BN 32
+#endif
+#ifndef MOE_TC_DECODE_STAGES
+#define MOE_TC_DECODE_STAGES 10
+#endif
+constexpr int PF_BN = MOE_TC_PREFILL_BN, PF_ST = MOE_TC_PREFILL_STAGES;
+constexpr int DC_BN = MOE_TC_DECODE_BN, DC_ST = MOE_TC_DECODE_STAGES;
+
 // few rows per expert (decode): narrow token tiles and a deep ring so that
-// enough weight bytes are in flight; otherwise token tiles of up to 256
+// enough weight bytes are in flight; otherwise token tiles of up to PF_BN
 bool decode_variant(const Job &j) { return j.T * j.c->topk <= (int64_t)16 * j.c->n_routed; }
 
 moe_status run_up(const Job &j) {
   if (tc_path(j.c, j.x_dt, j.w->w_dt))
-    return decode_variant(j) ? tc_up<32, 32, 10>(j) : tc_up<256, 32, 4>(j);
+    return decode_variant(j) ? tc_up<DC_BN, 32, DC_ST>(j) : tc_up<PF_BN, 32, PF_ST>(j);
   return j.x_dt == MOE_BF16 ? simt_up_x<bf16>(j) : simt_up_x<float>(j);
 }
 
 moe_status run_down(const Job &j) {
   if (tc_path(j.c, j.x_dt, j.w->w_dt))
-    return decode_variant(j) ? tc_down<32, 32, 10>(j) : tc_down<256, 32, 4>(j);
+    return decode_variant(j) ? tc_down<DC_BN, 32, DC_ST>(j) : tc_down<PF_BN, 32, PF_ST>(j);
   return simt_down_w(j);
 }
 

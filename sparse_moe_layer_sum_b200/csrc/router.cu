@@ -17,8 +17,11 @@
 #include <cuda_bf16.h>
 #include <math.h>
 
+#include <cudaTypedefs.h>
+
 #include "common.cuh"
 #include "moe_router.h"
+#include "sm100.cuh"
 
 namespace moe {
 namespace {
@@ -233,6 +236,296 @@ __global__ void __launch_bounds__(SEL_WARPS * 32) router_select(SelectArgs a) {
   if (a.sel_gap && lane == 0) a.sel_gap[t] = gap;
 }
 
+// ------------------------------------------------ tensor-core scores (bf16 x)
+//
+// z = x W_r^T with x in bf16 (exact in fp32) and W_r in fp32: W_r is split
+// once per call into three bf16 matrices with W_r = hi + mid + lo exactly
+// (each term holds the next 8 significant bits; the remainders are exact in
+// fp32), and z = x hi^T + x mid^T + x lo^T runs as three tcgen05 bf16 MMAs
+// per k-step into one fp32 TMEM accumulator.  The products are exact, so z
+// carries only fp32 accumulation error, as an fp32 dot product would.
+
+__global__ void __launch_bounds__(256) split_w3(const float *__restrict__ w, __nv_bfloat16 *w3,
+                                                int64_t n) {
+  const int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+  if (i >= n) return;
+  const float v = w[i];
+  const __nv_bfloat16 hi = __float2bfloat16_rn(v);
+  const float r1 = v - __bfloat162float(hi);
+  const __nv_bfloat16 mid = __float2bfloat16_rn(r1);
+  const float r2 = r1 - __bfloat162float(mid);
+  w3[i] = hi;
+  w3[n + i] = mid;
+  w3[2 * n + i] = __float2bfloat16_rn(r2);
+}
+
+namespace tcr {
+
+constexpr int BK = 64, BM = 128, THREADS = 192, EPI_WARPS = 4;
+constexpr int A_BYTES = BM * BK * 2;  // one of the three weight terms
+
+struct Params {
+  int T, E, nsplit, kb_per_split, KB, mt, nt;
+  float *z_part;  // [nsplit][T][E]
+  int32_t *status;
+  int64_t timeout_ns;
+};
+
+template <int BN, int STAGES>
+struct Layout {
+  static constexpr int B_BYTES = BN * BK * 2;
+  static constexpr int STAGE_BYTES = 3 * A_BYTES + B_BYTES;
+  static constexpr int BAR_OFF = STAGES * STAGE_BYTES;
+  static constexpr int MISC_OFF = BAR_OFF + (2 * STAGES + 5) * 8;
+  static constexpr size_t SMEM = 1024 + MISC_OFF + 16 + 4 * STAGES;
+  static constexpr uint32_t TMEM_COLS = 2 * BN;
+};
+
+__device__ __forceinline__ void drain_wait(uint64_t *bar, uint32_t parity, int64_t limit_ns) {
+  const uint64_t t0 = sm100::globaltimer_ns();
+  while (!sm100::mbar_try_wait(bar, parity))
+    if ((int64_t)(sm100::globaltimer_ns() - t0) > limit_ns) break;
+}
+
+// tile -> (split, token tile, expert tile); expert tiles innermost so the
+// CTAs sharing an x tile run together
+template <int BN, int STAGES>
+__global__ void __launch_bounds__(THREADS, 1)
+    router_scores_tc(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
+                     const Params p) {
+  using L = Layout<BN, STAGES>;
+  using namespace sm100;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                            ~static_cast<uintptr_t>(1023));
+  uint64_t *full = reinterpret_cast<uint64_t *>(sm + L::BAR_OFF);
+  uint64_t *empty = full + STAGES;
+  uint64_t *accf = empty + STAGES;
+  uint64_t *acce = accf + 2;
+  uint64_t *drain = acce + 2;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + L::MISC_OFF);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + L::MISC_OFF + 4);
+  volatile int *pending = reinterpret_cast<volatile int *>(sm + L::MISC_OFF + 16);
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(full + s, 1);
+      mbar_init(empty + s, 1);
+      pending[s] = -1;
+    }
+    mbar_init(accf, 1);
+    mbar_init(accf + 1, 1);
+    mbar_init(acce, EPI_WARPS);
+    mbar_init(acce + 1, EPI_WARPS);
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&tmW);
+    tma_prefetch_desc(&tmX);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, L::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int total = p.nsplit * p.nt * p.mt;
+
+  auto decode = [&](int tile, int &split, int &n0, int &m0, int &kb0, int &kb1, int &nvalid) {
+    const int mt = tile % p.mt;
+    const int rest = tile / p.mt;
+    const int nt = rest % p.nt;
+    split = rest / p.nt;
+    m0 = mt * BM;
+    n0 = nt * BN;
+    nvalid = min(BN, p.T - n0);
+    kb0 = split * p.kb_per_split;
+    kb1 = min(p.KB, kb0 + p.kb_per_split);
+  };
+
+  if (warp == 0) {
+    if (lane == 0) {
+      const uint64_t pol_w = policy_evict_first();
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
+        int split, n0, m0, kb0, kb1, nvalid;
+        decode(tile, split, n0, m0, kb0, kb1, nvalid);
+        const int nbox = (nvalid + 31) / 32;
+        const uint32_t bytes = (uint32_t)(3 * A_BYTES + nbox * 32 * BK * 2);
+        for (int kb = kb0; kb < kb1; ++kb) {
+          if (!wait_bounded(empty + stage, phase ^ 1u, abort_flag, p.timeout_ns, p.status)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(full + stage, bytes);
+          pending[stage] = (int)phase;
+          uint8_t *dst = sm + stage * L::STAGE_BYTES;
+          for (int t3 = 0; t3 < 3; ++t3)
+            tma_load_2d_hint(&tmW, dst + t3 * A_BYTES, full + stage, kb * BK, t3 * p.E + m0,
+                             pol_w);
+          for (int i = 0; i < nbox; ++i)
+            tma_load_2d(&tmX, dst + 3 * A_BYTES + i * 32 * BK * 2, full + stage, kb * BK,
+                        n0 + i * 32);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      int stage = 0, acc = 0;
+      uint32_t phase = 0, acc_phase = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
+        int split, n0, m0, kb0, kb1, nvalid;
+        decode(tile, split, n0, m0, kb0, kb1, nvalid);
+        if (!wait_bounded(acce + acc, acc_phase ^ 1u, abort_flag, p.timeout_ns, p.status)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
+        const uint32_t idesc = idesc_bf16_f32(BM, (nvalid + 15) & ~15);
+        for (int kb = kb0; kb < kb1; ++kb) {
+          if (!wait_bounded(full + stage, phase, abort_flag, p.timeout_ns, p.status)) {
+            ok = false;
+            break;
+          }
+          pending[stage] = -1;
+          tc_fence_after();
+          const uint32_t a_addr = smem_u32(sm + stage * L::STAGE_BYTES);
+          const uint32_t b_addr = a_addr + 3 * A_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk)
+#pragma unroll
+            for (int t3 = 0; t3 < 3; ++t3)
+              mma_bf16(d_tmem, sdesc_sw128(a_addr + t3 * A_BYTES + kk * 32),
+                       sdesc_sw128(b_addr + kk * 32), idesc,
+                       (kb > kb0 || kk > 0 || t3 > 0) ? 1u : 0u);
+          mma_commit(empty + stage);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        mma_commit(accf + acc);
+        acc ^= 1;
+        if (acc == 0) acc_phase ^= 1u;
+      }
+      if (!ok) {
+        mma_commit(drain);
+        drain_wait(drain, 0, p.timeout_ns);
+      }
+    }
+  } else {
+    const int q = warp & 3;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
+      int split, n0, m0, kb0, kb1, nvalid;
+      decode(tile, split, n0, m0, kb0, kb1, nvalid);
+      if (!wait_bounded(accf + acc, acc_phase, abort_flag, p.timeout_ns, p.status)) break;
+      tc_fence_after();
+      const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
+      float *out = p.z_part + (size_t)split * p.T * p.E;
+      const int e = m0 + q * 32 + lane;
+      for (int c0 = 0; c0 < nvalid; c0 += 32) {
+        uint32_t v[32];
+        tmem_ld_32x32b_x32(tb + (uint32_t)c0, v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+          if (c0 + j < nvalid) out[(size_t)(n0 + c0 + j) * p.E + e] = __uint_as_float(v[j]);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(acce + acc);
+      acc ^= 1;
+      if (acc == 0) acc_phase ^= 1u;
+    }
+  }
+  __syncthreads();
+  if (threadIdx.x == 0 && *abort_flag)
+    for (int s = 0; s < STAGES; ++s)
+      if (pending[s] >= 0) drain_wait(full + s, (uint32_t)pending[s], p.timeout_ns);
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, L::TMEM_COLS);
+  }
+}
+
+}  // namespace tcr
+
+constexpr int TC_BN = 128, TC_STAGES = 3;
+
+bool tc_router(const moe_cfg *c, moe_dtype x_dt) {
+  return x_dt == MOE_BF16 && c->n_routed % tcr::BM == 0 && c->dim % tcr::BK == 0;
+}
+
+struct TcPlan {
+  int mt, nt, nsplit, kb_per_split, KB;
+};
+
+TcPlan plan_tc(const moe_cfg *c, int64_t T) {
+  TcPlan p;
+  p.KB = c->dim / tcr::BK;
+  p.mt = c->n_routed / tcr::BM;
+  p.nt = (int)((T + TC_BN - 1) / TC_BN);
+  const int tiles = p.mt * p.nt;
+  int ns = (148 + tiles - 1) / tiles;  // fill the SMs of a B200 at small T
+  ns = ns < 1 ? 1 : (ns > p.KB ? p.KB : ns);
+  p.kb_per_split = (p.KB + ns - 1) / ns;
+  p.nsplit = (p.KB + p.kb_per_split - 1) / p.kb_per_split;
+  return p;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void *ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  }
+  return fn;
+}
+
+bool make_tmap_bf16(CUtensorMap *m, const void *base, uint64_t rows, uint64_t cols,
+                    uint32_t box_rows) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t gdim[2] = {cols, rows};
+  cuuint64_t gstride[1] = {cols * 2};
+  cuuint32_t box[2] = {64, box_rows};
+  cuuint32_t estride[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), gdim, gstride, box,
+            estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+  return n;
+}
+
+size_t tc_ws_bytes(const moe_cfg *c, int64_t T) {
+  const TcPlan p = plan_tc(c, T);
+  return align_up((size_t)3 * c->n_routed * c->dim * 2, 1024) +
+         align_up((size_t)p.nsplit * T * c->n_routed * 4, 256);
+}
+
 struct Plan {
   int nsplit, cols_per_split;
 };
@@ -261,7 +554,9 @@ using namespace moe;
 MOE_EXPORT size_t moe_router_workspace_size(const moe_cfg *cfg, int64_t T) {
   if (check_cfg(cfg) != MOE_OK || T < 0) return 0;
   const Plan p = plan_scores(cfg, T);
-  return align_up((size_t)p.nsplit * (size_t)T * cfg->n_routed * sizeof(float), 256);
+  const size_t simt = align_up((size_t)p.nsplit * (size_t)T * cfg->n_routed * sizeof(float), 256);
+  const size_t tc = tc_ws_bytes(cfg, T);
+  return simt > tc ? simt : tc;
 }
 
 MOE_EXPORT moe_status moe_router_forward(const moe_cfg *cfg, int64_t T, const void *x,
@@ -281,8 +576,45 @@ MOE_EXPORT moe_status moe_router_forward(const moe_cfg *cfg, int64_t T, const vo
   if (ws_bytes < moe_router_workspace_size(cfg, T)) return MOE_ERR_WORKSPACE;
 
   cudaStream_t s = as_stream(stream);
-  const Plan p = plan_scores(cfg, T);
   float *z_part = static_cast<float *>(ws);
+  int nsplit;
+  if (tc_router(cfg, x_dt) && T >= 32) {
+    const TcPlan tp = plan_tc(cfg, T);
+    const int64_t nw = (int64_t)cfg->n_routed * cfg->dim;
+    __nv_bfloat16 *w3 = static_cast<__nv_bfloat16 *>(ws);
+    z_part = reinterpret_cast<float *>(static_cast<uint8_t *>(ws) +
+                                       align_up((size_t)3 * nw * 2, 1024));
+    split_w3<<<(unsigned)((nw + 255) / 256), 256, 0, s>>>(w_r, w3, nw);
+    if ((st = launch_status()) != MOE_OK) return st;
+    CUtensorMap mw, mx;
+    if (!make_tmap_bf16(&mw, w3, (uint64_t)3 * cfg->n_routed, cfg->dim, tcr::BM) ||
+        !make_tmap_bf16(&mx, x, (uint64_t)T, cfg->dim, 32))
+      return MOE_ERR_CUDA;
+    tcr::Params pp;
+    pp.T = (int)T;
+    pp.E = cfg->n_routed;
+    pp.nsplit = tp.nsplit;
+    pp.kb_per_split = tp.kb_per_split;
+    pp.KB = tp.KB;
+    pp.mt = tp.mt;
+    pp.nt = tp.nt;
+    pp.z_part = z_part;
+    pp.status = dev_status;
+    pp.timeout_ns = 1000000000LL;
+    using L = tcr::Layout<TC_BN, TC_STAGES>;
+    auto kern = tcr::router_scores_tc<TC_BN, TC_STAGES>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L::SMEM) !=
+        cudaSuccess)
+      return MOE_ERR_CUDA;
+    const int total = tp.nsplit * tp.nt * tp.mt;
+    const int nsm = sm_count();
+    if (nsm <= 0) return MOE_ERR_CUDA;
+    kern<<<total < nsm ? total : nsm, tcr::THREADS, L::SMEM, s>>>(mw, mx, pp);
+    if ((st = launch_status()) != MOE_OK) return st;
+    nsplit = tp.nsplit;
+  } else {
+  const Plan p = plan_scores(cfg, T);
+  nsplit = p.nsplit;
   dim3 grid((unsigned)((T + SC_BM - 1) / SC_BM), (unsigned)((cfg->n_routed + SC_BN - 1) / SC_BN),
             (unsigned)p.nsplit);
   if (x_dt == MOE_BF16)
@@ -294,10 +626,11 @@ MOE_EXPORT moe_status moe_router_forward(const moe_cfg *cfg, int64_t T, const vo
                                                      (int)T, cfg->n_routed, cfg->dim,
                                                      p.cols_per_split);
   if ((st = launch_status()) != MOE_OK) return st;
+  }
 
   SelectArgs a;
   a.z_part = z_part;
-  a.nsplit = p.nsplit;
+  a.nsplit = nsplit;
   a.bias = cfg->has_bias ? bias : nullptr;
   a.weights = weights;
   a.indices = indices;

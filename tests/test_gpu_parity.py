@@ -33,6 +33,10 @@ DECODE_SMALL = custom("decode_small", 40, dim=1024, n_routed=64, n_groups=8, top
                       topk=8, inter=256, seed=18)
 ONE_TOKEN = custom("one_token", 1, dim=256, n_routed=16, n_groups=4, topk_groups=2, topk=4,
                    inter=128, seed=19)
+ROUTER_TC = custom("router_tc", 200, dim=512, n_routed=128, n_groups=8, topk_groups=4, topk=8,
+                   inter=128, seed=20)
+ROUTER_TC_SPLIT = custom("router_tc_split", 40, dim=2048, n_routed=256, n_groups=8,
+                         topk_groups=4, topk=8, inter=128, seed=21)
 FP8_SMALL = custom("fp8_small", 260, w_format="e4m3", dim=512, n_routed=16, n_groups=4,
                    topk_groups=2, topk=4, inter=256, seed=17)
 
@@ -56,7 +60,8 @@ def run_block(w, x, params):
 
 
 @pytest.mark.parametrize("w", [WORKLOADS["tiny_f32"], TINY_BF16, MID, MID_F32, SOFTMAX_NOBIAS,
-                               NOBIAS_SIGMOID, ONE_GROUP], ids=lambda w: w.name)
+                               NOBIAS_SIGMOID, ONE_GROUP, ROUTER_TC, ROUTER_TC_SPLIT],
+                         ids=lambda w: w.name)
 def test_router_matches_oracle(w):
     x, p = make_block(w)
     weights, indices, gap = moe.router_forward(w.shape, x, p.w_r, p.bias, gap=True)
