@@ -173,9 +173,12 @@ struct Params {
   int64_t timeout_ns;
 };
 
-template <int MODE, int BN_MAX, int BOXN, int STAGES>
+// CG = CTA group: 1 = one SM per tile; 2 = an SM pair per tile (cta_group::2),
+// where each CTA holds 128 weight rows and half of the token tile.
+template <int MODE, int CG, int BN_MAX, int BOXN, int STAGES>
 struct Layout {
-  static constexpr int B_BYTES = BN_MAX * BK * 2;
+  static constexpr int B_ROWS = BN_MAX / CG;  // token rows one CTA holds per stage
+  static constexpr int B_BYTES = B_ROWS * BK * 2;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int BAR_OFF = STAGES * STAGE_BYTES;
   static constexpr int NBARS = 2 * STAGES + 5;  // full, empty, acc_full x2, acc_empty x2, drain
@@ -187,11 +190,15 @@ struct Layout {
   static constexpr uint32_t TMEM_COLS =
       2 * BN_MAX <= 32 ? 32 : 2 * BN_MAX <= 64 ? 64 : 2 * BN_MAX <= 128 ? 128
                                                 : 2 * BN_MAX <= 256 ? 256 : 512;
+  // weight rows one tile covers: GEMM1 pairs 64 rows of w1 with the same 64
+  // rows of w3 per CTA; GEMM2 takes 128 rows of w2 per CTA
+  static constexpr int FEAT = (MODE == 1 ? 64 : BM) * CG;
   static size_t smem_bytes(int G, int E) {
     return 1024 + TAB_OFF + sizeof(int32_t) * (size_t)((G + 1) + G + (E + 1));
   }
+  static_assert(CG == 1 || CG == 2, "CTA group");
   static_assert(BN_MAX % 16 == 0 && BN_MAX >= 16 && BN_MAX <= 256, "MMA N range");
-  static_assert(BOXN % 16 == 0 && BN_MAX % BOXN == 0, "B box rows");
+  static_assert(BOXN % 16 == 0 && B_ROWS % BOXN == 0, "B box rows");
 };
 
 // Waits for a barrier phase with a time limit but ignores the abort flag;
@@ -203,11 +210,17 @@ __device__ __forceinline__ void drain_wait(uint64_t *bar, uint32_t parity, int64
   }
 }
 
-template <int MODE, int BN_MAX, int BOXN, int STAGES>
+__device__ __forceinline__ void sleep_ns(int64_t ns) {
+  const uint64_t t0 = sm100::globaltimer_ns();
+  while ((int64_t)(sm100::globaltimer_ns() - t0) < ns) {
+  }
+}
+
+template <int MODE, int CG, int BN_MAX, int BOXN, int STAGES>
 __global__ void __launch_bounds__(THREADS, 1)
     tc_expert_gemm(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA1,
                    const __grid_constant__ CUtensorMap tmB, const Params p) {
-  using L = Layout<MODE, BN_MAX, BOXN, STAGES>;
+  using L = Layout<MODE, CG, BN_MAX, BOXN, STAGES>;
   using namespace sm100;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -226,6 +239,12 @@ __global__ void __launch_bounds__(THREADS, 1)
   int32_t *s_off = s_tbase + p.G;
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  // this CTA's rank in its pair, the tile-unit (pair or CTA) index and count
+  const uint32_t rank = CG == 2 ? cluster_rank() : 0u;
+  const bool leader = rank == 0;
+  const int unit = CG == 2 ? (int)cluster_id_x() : (int)blockIdx.x;
+  const int nunits = CG == 2 ? (int)cluster_count_x() : (int)gridDim.x;
+
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(full + s, 1);
@@ -234,8 +253,8 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
     mbar_init(accf + 0, 1);
     mbar_init(accf + 1, 1);
-    mbar_init(acce + 0, EPI_WARPS);
-    mbar_init(acce + 1, EPI_WARPS);
+    mbar_init(acce + 0, EPI_WARPS * CG);
+    mbar_init(acce + 1, EPI_WARPS * CG);
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -247,11 +266,17 @@ __global__ void __launch_bounds__(THREADS, 1)
   for (int i = threadIdx.x; i < p.G; i += THREADS) s_tbase[i] = p.tile_base[i];
   for (int i = threadIdx.x; i <= p.E; i += THREADS) s_off[i] = p.offsets[i];
   if (warp == 1) {
-    tmem_alloc(tmem_slot, L::TMEM_COLS);
-    tmem_relinquish();
+    if (CG == 2) {
+      tmem_alloc_pair(tmem_slot, L::TMEM_COLS);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(tmem_slot, L::TMEM_COLS);
+      tmem_relinquish();
+    }
   }
   tc_fence_before();
   __syncthreads();
+  if (CG == 2) cluster_sync();  // the pair's barriers exist before any remote arrive
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   const int total = s_tstart[p.G];
@@ -264,29 +289,46 @@ __global__ void __launch_bounds__(THREADS, 1)
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
+      for (int tile = unit; ok && tile < total; tile += nunits) {
         const Tile t = decode_tile(tile, s_tstart, s_tbase, s_off, p.G, p.E, p.T, p.rows_routed);
-        const int arow = MODE == 1 ? t.g * p.I + t.ft * 64 : t.g * p.D + t.ft * BM;
-        const int nbox = (t.nvalid + BOXN - 1) / BOXN;
+        const int nmma = (t.nvalid + 15) & ~15;
+        const int brows = nmma / CG;  // this CTA's share of the token rows
+        const int b0 = t.rowbase + t.n0 + (int)rank * brows;
+        const int arow = MODE == 1 ? t.g * p.I + t.ft * L::FEAT + (int)rank * 64
+                                   : t.g * p.D + t.ft * L::FEAT + (int)rank * BM;
+        const int nbox = (brows + BOXN - 1) / BOXN;
         const uint32_t bytes = (uint32_t)(A_BYTES + nbox * BOXN * BK * 2);
         for (int kb = 0; kb < p.KB; ++kb) {
           if (!wait_bounded(empty + stage, phase ^ 1u, abort_flag, p.timeout_ns, p.status)) {
             ok = false;
             break;
           }
-          mbar_arrive_expect_tx(full + stage, bytes);
+          // the leader's full barrier counts the bytes of both CTAs
+          if (leader) mbar_arrive_expect_tx(full + stage, bytes * CG);
           pending[stage] = (int)phase;
           uint8_t *a_dst = sm + stage * L::STAGE_BYTES;
           uint8_t *b_dst = a_dst + A_BYTES;
-          if (MODE == 1) {
-            tma_load_2d_hint(&tmA0, a_dst, full + stage, kb * BK, arow, pol_w);
-            tma_load_2d_hint(&tmA1, a_dst + A_BYTES / 2, full + stage, kb * BK, arow, pol_w);
+          if (CG == 2) {
+            const uint32_t fb = mapa_shared(smem_u32(full + stage), 0);
+            if (MODE == 1) {
+              tma_load_2d_pair(&tmA0, a_dst, fb, kb * BK, arow, pol_w);
+              tma_load_2d_pair(&tmA1, a_dst + A_BYTES / 2, fb, kb * BK, arow, pol_w);
+            } else {
+              tma_load_2d_pair(&tmA0, a_dst, fb, kb * BK, arow, pol_w);
+            }
+            for (int i = 0; i < nbox; ++i)
+              tma_load_2d_pair(&tmB, b_dst + i * BOXN * BK * 2, fb, kb * BK, b0 + i * BOXN, pol_x);
           } else {
-            tma_load_2d_hint(&tmA0, a_dst, full + stage, kb * BK, arow, pol_w);
+            if (MODE == 1) {
+              tma_load_2d_hint(&tmA0, a_dst, full + stage, kb * BK, arow, pol_w);
+              tma_load_2d_hint(&tmA1, a_dst + A_BYTES / 2, full + stage, kb * BK, arow, pol_w);
+            } else {
+              tma_load_2d_hint(&tmA0, a_dst, full + stage, kb * BK, arow, pol_w);
+            }
+            for (int i = 0; i < nbox; ++i)
+              tma_load_2d_hint(&tmB, b_dst + i * BOXN * BK * 2, full + stage, kb * BK,
+                               b0 + i * BOXN, pol_x);
           }
-          for (int i = 0; i < nbox; ++i)
-            tma_load_2d_hint(&tmB, b_dst + i * BOXN * BK * 2, full + stage, kb * BK,
-                             t.rowbase + t.n0 + i * BOXN, pol_x);
           if (++stage == STAGES) {
             stage = 0;
             phase ^= 1u;
@@ -295,12 +337,12 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
     }
   } else if (warp == 1) {
-    if (lane == 0) {
+    if (lane == 0 && leader) {
       // ------------------------------------------------------ MMA issuer
       int stage = 0, acc = 0;
       uint32_t phase = 0, acc_phase = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
+      for (int tile = unit; ok && tile < total; tile += nunits) {
         const Tile t = decode_tile(tile, s_tstart, s_tbase, s_off, p.G, p.E, p.T, p.rows_routed);
         if (!wait_bounded(acce + acc, acc_phase ^ 1u, abort_flag, p.timeout_ns, p.status)) {
           ok = false;
@@ -309,7 +351,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN_MAX);
         const int nmma = (t.nvalid + 15) & ~15;
-        const uint32_t idesc = idesc_bf16_f32(BM, nmma);
+        const uint32_t idesc = idesc_bf16_f32(BM * CG, nmma);
         for (int kb = 0; kb < p.KB; ++kb) {
           if (!wait_bounded(full + stage, phase, abort_flag, p.timeout_ns, p.status)) {
             ok = false;
@@ -320,23 +362,37 @@ __global__ void __launch_bounds__(THREADS, 1)
           const uint32_t a_addr = smem_u32(sm + stage * L::STAGE_BYTES);
           const uint32_t b_addr = a_addr + A_BYTES;
 #pragma unroll
-          for (int kk = 0; kk < BK / 16; ++kk)
-            mma_bf16(d_tmem, sdesc_sw128(a_addr + kk * 32), sdesc_sw128(b_addr + kk * 32), idesc,
-                     (kb | kk) != 0 ? 1u : 0u);
-          mma_commit(empty + stage);
+          for (int kk = 0; kk < BK / 16; ++kk) {
+            const uint64_t ad = sdesc_sw128(a_addr + kk * 32), bd = sdesc_sw128(b_addr + kk * 32);
+            const uint32_t accum = (kb | kk) != 0 ? 1u : 0u;
+            if (CG == 2)
+              mma_bf16_pair(d_tmem, ad, bd, idesc, accum);
+            else
+              mma_bf16(d_tmem, ad, bd, idesc, accum);
+          }
+          if (CG == 2)
+            mma_commit_pair_mc(empty + stage, 0x3);
+          else
+            mma_commit(empty + stage);
           if (++stage == STAGES) {
             stage = 0;
             phase ^= 1u;
           }
         }
         if (!ok) break;
-        mma_commit(accf + acc);
+        if (CG == 2)
+          mma_commit_pair_mc(accf + acc, 0x3);
+        else
+          mma_commit(accf + acc);
         acc ^= 1;
         if (acc == 0) acc_phase ^= 1u;
       }
       if (!ok) {
         // make sure no MMA is still writing TMEM before it is freed
-        mma_commit(drain);
+        if (CG == 2)
+          mma_commit_pair(drain);
+        else
+          mma_commit(drain);
         drain_wait(drain, 0, p.timeout_ns);
       }
     }
@@ -345,7 +401,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     const int q = warp & 3;  // TMEM lane quarter this warp may access
     int acc = 0;
     uint32_t acc_phase = 0;
-    for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
+    for (int tile = unit; tile < total; tile += nunits) {
       const Tile t = decode_tile(tile, s_tstart, s_tbase, s_off, p.G, p.E, p.T, p.rows_routed);
       if (!wait_bounded(accf + acc, acc_phase, abort_flag, p.timeout_ns, p.status)) break;
       tc_fence_after();
@@ -361,7 +417,7 @@ __global__ void __launch_bounds__(THREADS, 1)
           out = p.out_shared;
           row0 = (size_t)(t.g - p.E) * p.T + t.n0;
         }
-        const int d = t.ft * BM + q * 32 + lane;
+        const int d = t.ft * L::FEAT + (int)rank * BM + q * 32 + lane;
         for (int c0 = 0; c0 < t.nvalid; c0 += 32) {
           uint32_t v[32];
           tmem_ld_32x32b_x32(tb + (uint32_t)c0, v);
@@ -379,7 +435,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         float *buf_a = xbuf + pr * 2 * 32 * XB_STRIDE;  // a, columns 16-31 of the chunk
         float *buf_u = buf_a + 32 * XB_STRIDE;          // u, columns 0-15 of the chunk
         bf16 *out = static_cast<bf16 *>(p.out);
-        const int f = t.ft * 64 + pr * 32 + lane;
+        const int f = t.ft * L::FEAT + (int)rank * 64 + pr * 32 + lane;
         const size_t row0 = (size_t)t.rowbase + t.n0;
         for (int c0 = 0; c0 < t.nvalid; c0 += 32) {
           uint32_t v[32];
@@ -404,7 +460,12 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(acce + acc);
+      if (lane == 0) {
+        if (CG == 2)
+          mbar_arrive_cluster(mapa_shared(smem_u32(acce + acc), 0));  // the leader's barrier
+        else
+          mbar_arrive(acce + acc);
+      }
       acc ^= 1;
       if (acc == 0) acc_phase ^= 1u;
     }
@@ -412,14 +473,24 @@ __global__ void __launch_bounds__(THREADS, 1)
 
   __syncthreads();
   if (threadIdx.x == 0 && *abort_flag) {
-    // a stalled pipeline stopped early: let copies already issued land
-    for (int s = 0; s < STAGES; ++s)
-      if (pending[s] >= 0) drain_wait(full + s, (uint32_t)pending[s], p.timeout_ns);
+    // a stalled pipeline stopped early: let copies already issued land.  The
+    // leader's full barriers count both CTAs' copies; the other CTA of a pair
+    // cannot wait on them and just allows its copies time to land.
+    if (leader) {
+      for (int s = 0; s < STAGES; ++s)
+        if (pending[s] >= 0) drain_wait(full + s, (uint32_t)pending[s], p.timeout_ns);
+    } else {
+      sleep_ns(200000);
+    }
   }
   __syncthreads();
+  if (CG == 2) cluster_sync();  // neither CTA leaves while the other may touch its memory
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, L::TMEM_COLS);
+    if (CG == 2)
+      tmem_dealloc_pair(tmem_base, L::TMEM_COLS);
+    else
+      tmem_dealloc(tmem_base, L::TMEM_COLS);
   }
 }
 
@@ -627,18 +698,40 @@ WsLayout ws_layout(const moe_cfg *c, int64_t T, moe_dtype x_dt, moe_dtype w_dt) 
   return l;
 }
 
-template <int MODE, int BN_MAX, int BOXN, int STAGES>
+template <int MODE, int CG, int BN_MAX, int BOXN, int STAGES>
 moe_status launch_tc(const CUtensorMap &a0, const CUtensorMap &a1, const CUtensorMap &b,
                      const tc::Params &p, cudaStream_t s) {
-  using L = tc::Layout<MODE, BN_MAX, BOXN, STAGES>;
-  auto kern = tc::tc_expert_gemm<MODE, BN_MAX, BOXN, STAGES>;
+  using L = tc::Layout<MODE, CG, BN_MAX, BOXN, STAGES>;
+  auto kern = tc::tc_expert_gemm<MODE, CG, BN_MAX, BOXN, STAGES>;
   const size_t smem = L::smem_bytes(p.G, p.E);
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
       cudaSuccess)
     return MOE_ERR_CUDA;
   const int nsm = sm_count();
-  if (nsm <= 0) return MOE_ERR_CUDA;
-  kern<<<nsm, tc::THREADS, smem, s>>>(a0, a1, b, p);
+  if (nsm < 2) return MOE_ERR_CUDA;
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  cfg.blockDim = dim3(tc::THREADS);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cfg.gridDim = dim3(nsm);
+  if (CG == 2) {
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    // one persistent pair per co-resident SM pair
+    int pairs = nsm / 2;
+    cfg.gridDim = dim3(2 * pairs);
+    int active = 0;
+    if (cudaOccupancyMaxActiveClusters(&active, kern, &cfg) == cudaSuccess && active > 0 &&
+        active < pairs)
+      pairs = active;
+    cfg.gridDim = dim3(2 * pairs);
+  }
+  if (cudaLaunchKernelEx(&cfg, kern, a0, a1, b, p) != cudaSuccess) return MOE_ERR_CUDA;
   return launch_status();
 }
 
@@ -689,11 +782,11 @@ tc::Params tc_params(const Job &j) {
   return p;
 }
 
-template <int BN_MAX, int BOXN, int STAGES>
+template <int CG, int BN_MAX, int BOXN, int STAGES>
 moe_status tc_up(const Job &j) {
   const int G = j.G(), D = j.c->dim, I = j.c->inter;
   int32_t *tab = j.tab();
-  Tiling t1{BN_MAX, I / 64, tab, tab + (G + 1)};
+  Tiling t1{BN_MAX, I / (64 * CG), tab, tab + (G + 1)};
   Tiling none{0, 0, nullptr, nullptr};
   prep_tiles<<<1, 32, 0, j.s>>>(j.offsets, j.E(), G, (int)j.T, t1, none);
   moe_status st = launch_status();
@@ -718,16 +811,16 @@ moe_status tc_up(const Job &j) {
   p.KB = D / tc::BK;
   p.out = h;
   prof(1, j.s);
-  st = launch_tc<1, BN_MAX, BOXN, STAGES>(mw1, mw3, mx, p, j.s);
+  st = launch_tc<1, CG, BN_MAX, BOXN, STAGES>(mw1, mw3, mx, p, j.s);
   prof(2, j.s);
   return st;
 }
 
-template <int BN_MAX, int BOXN, int STAGES>
+template <int CG, int BN_MAX, int BOXN, int STAGES>
 moe_status tc_down(const Job &j) {
   const int G = j.G(), D = j.c->dim, I = j.c->inter;
   int32_t *tab = j.tab();
-  Tiling t2{BN_MAX, D / tc::BM, tab + (2 * G + 1), tab + (3 * G + 2)};
+  Tiling t2{BN_MAX, D / (tc::BM * CG), tab + (2 * G + 1), tab + (3 * G + 2)};
   Tiling none{0, 0, nullptr, nullptr};
   prep_tiles<<<1, 32, 0, j.s>>>(j.offsets, j.E(), G, (int)j.T, t2, none);
   moe_status st = launch_status();
@@ -744,7 +837,7 @@ moe_status tc_down(const Job &j) {
   p.KB = I / tc::BK;
   p.out = j.out_perm;
   prof(3, j.s);
-  st = launch_tc<2, BN_MAX, BOXN, STAGES>(mw2, mw2, mh, p, j.s);
+  st = launch_tc<2, CG, BN_MAX, BOXN, STAGES>(mw2, mw2, mh, p, j.s);
   prof(4, j.s);
   return st;
 }
@@ -834,7 +927,7 @@ moe_status simt_down_w(const Job &j) {
 #define MOE_TC_PREFILL_BN 256
 #endif
 #ifndef MOE_TC_PREFILL_STAGES
-#define MOE_TC_PREFILL_STAGES 4
+#define MOE_TC_PREFILL_STAGES 6
 #endif
 #ifndef MOE_TC_DECODE_BN
 #define MOE_TC_DECODE_BN 32
@@ -845,19 +938,27 @@ moe_status simt_down_w(const Job &j) {
 constexpr int PF_BN = MOE_TC_PREFILL_BN, PF_ST = MOE_TC_PREFILL_STAGES;
 constexpr int DC_BN = MOE_TC_DECODE_BN, DC_ST = MOE_TC_DECODE_STAGES;
 
-// few rows per expert (decode): narrow token tiles and a deep ring so that
-// enough weight bytes are in flight; otherwise token tiles of up to PF_BN
+// few rows per expert (decode): one SM per tile, narrow token tiles and a deep
+// ring so that enough weight bytes are in flight; otherwise SM pairs with
+// token tiles of up to PF_BN rows, each SM holding half of them
 bool decode_variant(const Job &j) { return j.T * j.c->topk <= (int64_t)16 * j.c->n_routed; }
+
+// an SM pair per tile (cta_group::2) covers 128 features of w1/w3 and 256 rows of w2
+bool pair_ok(const Job &j) { return j.c->inter % 128 == 0 && j.c->dim % 256 == 0; }
 
 moe_status run_up(const Job &j) {
   if (tc_path(j.c, j.x_dt, j.w->w_dt))
-    return decode_variant(j) ? tc_up<DC_BN, 32, DC_ST>(j) : tc_up<PF_BN, 32, PF_ST>(j);
+    return decode_variant(j) ? tc_up<1, DC_BN, 32, DC_ST>(j)
+           : pair_ok(j)      ? tc_up<2, PF_BN, 32, PF_ST>(j)
+                             : tc_up<1, 256, 32, 4>(j);
   return j.x_dt == MOE_BF16 ? simt_up_x<bf16>(j) : simt_up_x<float>(j);
 }
 
 moe_status run_down(const Job &j) {
   if (tc_path(j.c, j.x_dt, j.w->w_dt))
-    return decode_variant(j) ? tc_down<DC_BN, 32, DC_ST>(j) : tc_down<PF_BN, 32, PF_ST>(j);
+    return decode_variant(j) ? tc_down<1, DC_BN, 32, DC_ST>(j)
+           : pair_ok(j)      ? tc_down<2, PF_BN, 32, PF_ST>(j)
+                             : tc_down<1, 256, 32, 4>(j);
   return simt_down_w(j);
 }
 

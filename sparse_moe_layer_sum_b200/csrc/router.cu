@@ -521,6 +521,7 @@ int sm_count() {
 }
 
 size_t tc_ws_bytes(const moe_cfg *c, int64_t T) {
+  if (c->n_routed % tcr::BM != 0 || c->dim % tcr::BK != 0) return 0;  // CUDA-core path only
   const TcPlan p = plan_tc(c, T);
   return align_up((size_t)3 * c->n_routed * c->dim * 2, 1024) +
          align_up((size_t)p.nsplit * T * c->n_routed * 4, 256);

@@ -86,6 +86,11 @@ def test_workspace_sizes_grow_with_tokens():
     assert g(ctypes.byref(c), 4096, 1, 1) > g(ctypes.byref(c), 64, 1, 1) > 0
     assert fn("moe_dispatch", "moe_dispatch_workspace_size")(ctypes.byref(c), 16384) >= 256 * 4
     assert f(ctypes.byref(v3_cfg(topk=200)), 8) == 0            # invalid config -> 0
+    # shapes that only the CUDA-core paths take (no tensor-core tiling)
+    for E, G in ((16, 4), (24, 4), (64, 8)):
+        small = v3_cfg(dim=256, n_routed=E, n_groups=G, topk_groups=2, topk=4, inter=96)
+        assert f(ctypes.byref(small), 300) > 0
+        assert g(ctypes.byref(small), 300, 0, 0) > 0
 
 
 def test_dispatch_validation():

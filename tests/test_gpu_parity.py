@@ -37,6 +37,9 @@ ROUTER_TC = custom("router_tc", 200, dim=512, n_routed=128, n_groups=8, topk_gro
                    inter=128, seed=20)
 ROUTER_TC_SPLIT = custom("router_tc_split", 40, dim=2048, n_routed=256, n_groups=8,
                          topk_groups=4, topk=8, inter=128, seed=21)
+# dim % 256 != 0: the prefill path falls back to one SM per tile
+CG1_PREFILL = custom("cg1_prefill", 230, dim=384, n_routed=16, n_groups=4, topk_groups=2, topk=4,
+                     inter=128, seed=22)
 FP8_SMALL = custom("fp8_small", 260, w_format="e4m3", dim=512, n_routed=16, n_groups=4,
                    topk_groups=2, topk=4, inter=256, seed=17)
 
@@ -113,7 +116,7 @@ def test_dispatch_reports_out_of_range():
 
 
 @pytest.mark.parametrize("w", [WORKLOADS["tiny_f32"], TINY_BF16, MID, MID_F32, DECODE_SMALL,
-                               ONE_TOKEN, FP8_SMALL], ids=lambda w: w.name)
+                               ONE_TOKEN, CG1_PREFILL, FP8_SMALL], ids=lambda w: w.name)
 def test_experts_rows_match_oracle(w):
     """Expert outputs row by row, on a seeded index set (routing held fixed)."""
     x, p = make_block(w)
