@@ -101,8 +101,15 @@ __global__ void __launch_bounds__(32) prep_tiles(const int32_t *__restrict__ off
 }
 
 struct Tile {
-  int g, ft, n0, nvalid, rowbase;
+  int g, ft, tt, n0, nvalid, rowbase;
 };
+
+// First k-block of a tile.  Tiles that run at the same time share operands
+// (the feature tiles of one expert read the same token rows; the token tiles
+// of one expert read the same weight rows); starting them at different
+// k-blocks spreads those concurrent reads over different L2 lines instead of
+// sending every SM to the same lines at once.
+__device__ __forceinline__ int k_rotation(const Tile &t, int KB) { return (t.ft * 7 + t.tt * 5) % KB; }
 
 // rowbase: first row of the group in the expert-contiguous activation
 // buffers (routed: offsets[g]; shared: after the T*k routed rows).
@@ -124,8 +131,8 @@ __device__ __forceinline__ Tile decode_tile(int tile, const int32_t *tstart, con
   const int ntt = (n + base - 1) / base;
   const int local = tile - tstart[lo];
   t.ft = local / ntt;
-  const int tt = local - t.ft * ntt;
-  t.n0 = tt * base;
+  t.tt = local - t.ft * ntt;
+  t.n0 = t.tt * base;
   t.nvalid = min(base, n - t.n0);
   t.rowbase = lo < E ? off[lo] : rows_routed + (lo - E) * T;
   return t;
@@ -298,7 +305,9 @@ __global__ void __launch_bounds__(THREADS, 1)
                                    : t.g * p.D + t.ft * L::FEAT + (int)rank * BM;
         const int nbox = (brows + BOXN - 1) / BOXN;
         const uint32_t bytes = (uint32_t)(A_BYTES + nbox * BOXN * BK * 2);
-        for (int kb = 0; kb < p.KB; ++kb) {
+        const int k0 = k_rotation(t, p.KB);
+        for (int i = 0; i < p.KB; ++i) {
+          const int kb = k0 + i < p.KB ? k0 + i : k0 + i - p.KB;
           if (!wait_bounded(empty + stage, phase ^ 1u, abort_flag, p.timeout_ns, p.status)) {
             ok = false;
             break;
@@ -929,6 +938,9 @@ moe_status simt_down_w(const Job &j) {
 #ifndef MOE_TC_PREFILL_STAGES
 #define MOE_TC_PREFILL_STAGES 6
 #endif
+#ifndef MOE_TC_PREFILL_CG
+#define MOE_TC_PREFILL_CG 2
+#endif
 #ifndef MOE_TC_DECODE_BN
 #define MOE_TC_DECODE_BN 32
 #endif
@@ -944,7 +956,9 @@ constexpr int DC_BN = MOE_TC_DECODE_BN, DC_ST = MOE_TC_DECODE_STAGES;
 bool decode_variant(const Job &j) { return j.T * j.c->topk <= (int64_t)16 * j.c->n_routed; }
 
 // an SM pair per tile (cta_group::2) covers 128 features of w1/w3 and 256 rows of w2
-bool pair_ok(const Job &j) { return j.c->inter % 128 == 0 && j.c->dim % 256 == 0; }
+bool pair_ok(const Job &j) {
+  return MOE_TC_PREFILL_CG == 2 && j.c->inter % 128 == 0 && j.c->dim % 256 == 0;
+}
 
 moe_status run_up(const Job &j) {
   if (tc_path(j.c, j.x_dt, j.w->w_dt))
