@@ -45,6 +45,9 @@ def parse():
     ap.add_argument("--cpu-sample", type=int, default=8,
                     help="tokens the oracle pushes through the block for cpu_baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--combine", choices=["scatter", "ordered"], default="scatter",
+                    help="weighted sum into y inside the second matmul, or ordered and "
+                         "bit-reproducible in a separate pass")
     return ap.parse_args()
 
 
@@ -190,7 +193,7 @@ def run_ours(args, rank, local_rank, world):
     for i in range(1, N_X_BATCHES):
         gx.manual_seed(w.seed + 104729 * (1 + rank * N_X_BATCHES + i))
         xs.append(torch.randn(w.T, sh.dim, generator=gx, device=dev).to(w.x_dtype))
-    blk = moe.MoEBlock(sh, params, w.T, w.x_dtype, device=dev)
+    blk = moe.MoEBlock(sh, params, w.T, w.x_dtype, device=dev, combine=args.combine)
 
     for i in range(max(args.warmup, 1)):
         blk.forward(xs[i % N_X_BATCHES])
@@ -240,7 +243,7 @@ def run_ours(args, rank, local_rank, world):
     scale_b = (3 * (sh.dim // 128) * (sh.inter // 128) * 4) if w.w_format == "e4m3" else 0
     touched = [int((c > 0).sum()) for c in counts]
     kw = [kernel_work(sh.dim, sh.n_routed, sh.inter, sh.topk, sh.n_shared, w.T, n, w_bytes,
-                      x_bytes, scale_b) for n in touched]
+                      x_bytes, scale_b, scatter=blk.combine_mode == "scatter") for n in touched]
     bw = [block_work(sh.dim, sh.n_routed, sh.inter, sh.topk, sh.n_shared, w.T, n, w_bytes,
                      x_bytes, scale_b, sh.has_bias) for n in touched]
     steps_per_batch = [sum(1 for i in range(K) if i % N_X_BATCHES == b) for b in range(N_X_BATCHES)]
@@ -322,6 +325,7 @@ def run_ours(args, rank, local_rank, world):
         "dtype": "bf16" if w.w_format != "f32" else "f32",
         "data": "synthetic (seeded N(0,1) activations, N(0,1/fan_in) weights, U(-0.1,0.1) bias)",
         "config": {"workload": w.name, "T": w.T, "dim": sh.dim, "n_routed": sh.n_routed,
+                   "combine": blk.combine_mode,
                    "topk": sh.topk, "inter": sh.inter, "weights": w.w_format,
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                    "l2": f"inputs larger than L2: {N_X_BATCHES} rotating x batches and "
@@ -329,7 +333,7 @@ def run_ours(args, rank, local_rank, world):
                          "of expert weights per step"},
         "roofline": roof, "step_roofline": step_roof,
         "kernels_ms": dur, "cpu_baseline": cpu, "e2e": e2e,
-        "gpu_launches": K * moe.MoEBlock.LAUNCHES_PER_FORWARD,
+        "gpu_launches": K * blk.launches_per_forward,
         "clocks": clk, "touched_experts": touched, "hot_share": hot,
     }
     if rank == 0:

@@ -66,6 +66,26 @@ moe_status moe_experts_forward(const moe_cfg *cfg, int64_t T, const void *x, moe
                                moe_stream_t stream);
 
 /*
+ * The experts and the weighted combine in one pass: the second matmul's
+ * epilogue adds gate(t, e) * expert_e(x[t]) for every routed row, and the
+ * shared expert's output with gate 1, straight into the fp32 block output
+ *   y[t,:] = sum_j weights[t,j] * expert_{indices[t,j]}(x[t,:]) + shared(x[t,:])
+ * with fp32 reductions (the "y[idx] += expert(x[idx]) * weight" accumulation
+ * of the moe-forward excerpt, run for all experts at once).  y is zeroed by
+ * the call first.  No per-slot expert outputs are written, which saves their
+ * round trip through memory; in exchange the order of the fp32 additions
+ * into y is not fixed, so results may differ in the last bits from run to
+ * run (use moe_experts_forward + moe_combine for bit-reproducible sums).
+ * indices, weights [T, topk] from moe_router_forward; y [T, dim] fp32 out.
+ */
+moe_status moe_experts_forward_combine(const moe_cfg *cfg, int64_t T, const void *x,
+                                       moe_dtype x_dt, const moe_expert_weights *w,
+                                       const int32_t *offsets, const int32_t *sorted_token,
+                                       const int32_t *indices, const float *weights, float *y,
+                                       void *ws, size_t ws_bytes, int32_t *dev_status,
+                                       moe_stream_t stream);
+
+/*
  * The two halves of moe_experts_forward, for callers that schedule them
  * separately (moe_experts_forward(...) == moe_experts_up(...) followed by
  * moe_experts_down(...) on the same stream and workspace).

@@ -52,6 +52,9 @@ SIGNATURES = {
     ("moe_experts", "moe_experts_forward"): (
         _i32, [_cfgp, _i64, _vp, _i32, ctypes.POINTER(MoEExpertWeights), _vp, _vp, _vp, _vp,
                _vp, _sz, _vp, _vp]),
+    ("moe_experts", "moe_experts_forward_combine"): (
+        _i32, [_cfgp, _i64, _vp, _i32, ctypes.POINTER(MoEExpertWeights), _vp, _vp, _vp, _vp, _vp,
+               _vp, _sz, _vp, _vp]),
     ("moe_experts", "moe_experts_up"): (
         _i32, [_cfgp, _i64, _vp, _i32, ctypes.POINTER(MoEExpertWeights), _vp, _vp, _vp, _sz, _vp,
                _vp]),

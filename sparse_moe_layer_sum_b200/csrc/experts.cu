@@ -178,6 +178,12 @@ struct Params {
   float *out_shared;
   int32_t *status;
   int64_t timeout_ns;
+  // MODE 3 (second GEMM with the weighted scatter into y)
+  const int32_t *sorted_token;
+  const int32_t *indices;  // [T, k]
+  const float *weights;    // [T, k]
+  int k;
+  float *y;                // [T, D], zeroed before the launch
 };
 
 // CG = CTA group: 1 = one SM per tile; 2 = an SM pair per tile (cta_group::2),
@@ -192,14 +198,15 @@ struct Layout {
   static constexpr int MISC_OFF = BAR_OFF + NBARS * 8;
   static constexpr int MISC_BYTES = 16 + 4 * STAGES;
   static constexpr int XBUF_OFF = (MISC_OFF + MISC_BYTES + 127) / 128 * 128;
-  static constexpr int XBUF_BYTES = MODE == 1 ? 2 * 2 * 32 * XB_STRIDE * 4 : 0;
+  // GEMM1: SwiGLU exchange buffers; MODE 3: the tile's (token, gate) list
+  static constexpr int XBUF_BYTES = MODE == 1 ? 2 * 2 * 32 * XB_STRIDE * 4 : MODE == 3 ? BN_MAX * 8 : 0;
   static constexpr int TAB_OFF = XBUF_OFF + XBUF_BYTES;
   static constexpr uint32_t TMEM_COLS =
       2 * BN_MAX <= 32 ? 32 : 2 * BN_MAX <= 64 ? 64 : 2 * BN_MAX <= 128 ? 128
                                                 : 2 * BN_MAX <= 256 ? 256 : 512;
   // weight rows one tile covers: GEMM1 pairs 64 rows of w1 with the same 64
   // rows of w3 per CTA; GEMM2 takes 128 rows of w2 per CTA
-  static constexpr int FEAT = (MODE == 1 ? 64 : BM) * CG;
+  static constexpr int FEAT = (MODE == 1 ? 64 : BM) * CG;  // MODE 2 and 3: rows of w2
   static size_t smem_bytes(int G, int E) {
     return 1024 + TAB_OFF + sizeof(int32_t) * (size_t)((G + 1) + G + (E + 1));
   }
@@ -415,7 +422,38 @@ __global__ void __launch_bounds__(THREADS, 1)
       if (!wait_bounded(accf + acc, acc_phase, abort_flag, p.timeout_ns, p.status)) break;
       tc_fence_after();
       const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN_MAX);
-      if (MODE == 2) {
+      if (MODE == 3) {
+        // weighted scatter into y: y[t, d] += gate(t) * o[t, d] (gate 1 for the
+        // shared expert), with fp32 reductions; first the tile's token list
+        int32_t *s_tok = reinterpret_cast<int32_t *>(xbuf);
+        float *s_gate = reinterpret_cast<float *>(s_tok + BN_MAX);
+        const int et = threadIdx.x - 64;  // 0..127 over the four epilogue warps
+        named_bar_sync(3, 128);            // the previous tile's readers are done
+        for (int c = et; c < t.nvalid; c += 128) {
+          int tok;
+          float gate = 1.0f;
+          if (t.g < p.E) {
+            tok = p.sorted_token[t.rowbase + t.n0 + c];
+            for (int jj = 0; jj < p.k; ++jj)
+              if (p.indices[(size_t)tok * p.k + jj] == t.g) gate = p.weights[(size_t)tok * p.k + jj];
+          } else {
+            tok = t.n0 + c;
+          }
+          s_tok[c] = tok;
+          s_gate[c] = gate;
+        }
+        named_bar_sync(3, 128);
+        const int d = t.ft * L::FEAT + (int)rank * BM + q * 32 + lane;
+        for (int c0 = 0; c0 < t.nvalid; c0 += 32) {
+          uint32_t v[32];
+          tmem_ld_32x32b_x32(tb + (uint32_t)c0, v);
+          tmem_wait_ld();
+#pragma unroll
+          for (int j = 0; j < 32; ++j)
+            if (c0 + j < t.nvalid)
+              atomicAdd(p.y + (size_t)s_tok[c0 + j] * p.D + d, s_gate[c0 + j] * __uint_as_float(v[j]));
+        }
+      } else if (MODE == 2) {
         // lanes are output features d, columns are tokens
         float *out;
         size_t row0;
@@ -547,6 +585,11 @@ struct SimtArgs {
   int E, G, T, D, I, rows_routed, act_bf16;
   float *h;  // [rows, I] fp32 (values rounded to bf16 when act_bf16)
   float *out_perm, *out_shared;
+  // weighted scatter into y instead of out_perm / out_shared (when y != NULL)
+  const int32_t *indices;
+  const float *weights;
+  int k;
+  float *y;
 };
 
 template <typename XT, typename WT>
@@ -626,6 +669,21 @@ __global__ void __launch_bounds__(256) simt_gemm2(const WT *w2, const float *s2,
     }
   }
   if (r < t.nvalid) {
+    if (a.y) {
+      int tok = t.n0 + r;
+      float gate = 1.0f;
+      if (t.g < a.E) {
+        tok = a.sorted_token[t.rowbase + t.n0 + r];
+        for (int jj = 0; jj < a.k; ++jj)
+          if (a.indices[(size_t)tok * a.k + jj] == t.g) gate = a.weights[(size_t)tok * a.k + jj];
+      }
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int d = t.ft * ST + dq + j;
+        if (d < a.D) atomicAdd(a.y + (size_t)tok * a.D + d, gate * acc[j]);
+      }
+      return;
+    }
     float *out;
     size_t row;
     if (t.g < a.E) {
@@ -764,6 +822,10 @@ struct Job {
   const int32_t *sorted_token;
   float *out_perm;
   float *out_shared;
+  // weighted scatter into y (moe_experts_forward_combine); y == NULL otherwise
+  const int32_t *indices;
+  const float *weights;
+  float *y;
   uint8_t *ws;
   WsLayout l;
   int32_t *status;
@@ -788,6 +850,11 @@ tc::Params tc_params(const Job &j) {
   p.out_shared = j.out_shared;
   p.status = j.status;
   p.timeout_ns = 1000000000LL;
+  p.sorted_token = j.sorted_token;
+  p.indices = j.indices;
+  p.weights = j.weights;
+  p.k = j.c->topk;
+  p.y = j.y;
   return p;
 }
 
@@ -846,7 +913,10 @@ moe_status tc_down(const Job &j) {
   p.KB = I / tc::BK;
   p.out = j.out_perm;
   prof(3, j.s);
-  st = launch_tc<2, CG, BN_MAX, BOXN, STAGES>(mw2, mw2, mh, p, j.s);
+  if (j.y)
+    st = launch_tc<3, CG, BN_MAX, BOXN, STAGES>(mw2, mw2, mh, p, j.s);
+  else
+    st = launch_tc<2, CG, BN_MAX, BOXN, STAGES>(mw2, mw2, mh, p, j.s);
   prof(4, j.s);
   return st;
 }
@@ -867,6 +937,10 @@ SimtArgs simt_args(const Job &j, const Tiling &t) {
   a.out_shared = j.out_shared;
   a.tile_start = t.tile_start;
   a.tile_base = t.tile_base;
+  a.indices = j.indices;
+  a.weights = j.weights;
+  a.k = j.c->topk;
+  a.y = j.y;
   return a;
 }
 
@@ -1007,6 +1081,9 @@ moe_status make_job(Job &j, const moe_cfg *cfg, int64_t T, const void *x, moe_dt
   j.sorted_token = sorted_token;
   j.out_perm = out_perm;
   j.out_shared = out_shared;
+  j.indices = nullptr;
+  j.weights = nullptr;
+  j.y = nullptr;
   j.ws = static_cast<uint8_t *>(ws);
   j.status = dev_status;
   j.s = as_stream(stream);
@@ -1057,6 +1134,30 @@ MOE_EXPORT moe_status moe_experts_forward(const moe_cfg *cfg, int64_t T, const v
   moe_status st = make_job(j, cfg, T, x, x_dt, w, offsets, sorted_token, out_perm, out_shared,
                            ws, ws_bytes, dev_status, stream, true, true);
   if (st != MOE_OK || T == 0) return st;
+  if ((st = run_up(j)) != MOE_OK) return st;
+  return run_down(j);
+}
+
+MOE_EXPORT moe_status moe_experts_forward_combine(const moe_cfg *cfg, int64_t T, const void *x,
+                                                  moe_dtype x_dt, const moe_expert_weights *w,
+                                                  const int32_t *offsets,
+                                                  const int32_t *sorted_token,
+                                                  const int32_t *indices, const float *weights,
+                                                  float *y, void *ws, size_t ws_bytes,
+                                                  int32_t *dev_status, moe_stream_t stream) {
+  Job j;
+  // out_perm / out_shared are not used on this path; y stands in for the checks
+  moe_status st = make_job(j, cfg, T, x, x_dt, w, offsets, sorted_token, y, y, ws, ws_bytes,
+                           dev_status, stream, true, true);
+  if (st != MOE_OK || T == 0) return st;
+  if (!indices || !weights || !y) return MOE_ERR_INVALID;
+  j.out_perm = nullptr;
+  j.out_shared = nullptr;
+  j.indices = indices;
+  j.weights = weights;
+  j.y = y;
+  if (cudaMemsetAsync(y, 0, (size_t)T * cfg->dim * sizeof(float), j.s) != cudaSuccess)
+    return MOE_ERR_CUDA;
   if ((st = run_up(j)) != MOE_OK) return st;
   return run_down(j);
 }

@@ -139,6 +139,28 @@ def experts_forward(shape: BlockShape, x: torch.Tensor, wstruct: MoEExpertWeight
     return out_perm, out_shared
 
 
+def experts_forward_combine(shape: BlockShape, x: torch.Tensor, wstruct: MoEExpertWeights,
+                            offsets: torch.Tensor, sorted_token: torch.Tensor,
+                            indices: torch.Tensor, weights: torch.Tensor, *, y=None, ws=None,
+                            status=None):
+    """moe_experts_forward_combine: y [T, dim] fp32 (experts + weighted scatter)."""
+    _check_cuda(x, offsets, sorted_token, indices, weights)
+    cfg = shape.cfg()
+    T = x.shape[0]
+    if y is None:
+        y = torch.empty(T, shape.dim, dtype=torch.float32, device=x.device)
+    need = fn("moe_experts", "moe_experts_workspace_size")(ctypes.byref(cfg), T, _dt(x),
+                                                            wstruct.w_dt)
+    if ws is None or ws.numel() < need:
+        ws = _ws(need, x.device)
+    st = fn("moe_experts", "moe_experts_forward_combine")(
+        ctypes.byref(cfg), T, x.data_ptr(), _dt(x), ctypes.byref(wstruct), offsets.data_ptr(),
+        sorted_token.data_ptr(), indices.data_ptr(), weights.data_ptr(), y.data_ptr(),
+        ws.data_ptr(), ws.numel(), _ptr(status), _stream())
+    check(st, "moe_experts_forward_combine")
+    return y
+
+
 def combine(shape: BlockShape, weights: torch.Tensor, slot_of: torch.Tensor,
             out_perm: torch.Tensor, out_shared: Optional[torch.Tensor], *, y=None, status=None):
     """moe_combine: y [T, dim] fp32."""
@@ -183,10 +205,19 @@ class MoEBlock:
     forward() enqueues router -> dispatch -> experts -> combine on the current
     stream with no host synchronisation; all buffers are preallocated, so the
     call can be captured in a CUDA graph.
+
+    combine="scatter" (default) adds the gated expert outputs straight into y
+    from the second matmul (moe_experts_forward_combine); "ordered" writes
+    the per-slot outputs and sums them in a fixed order (moe_experts_forward
+    + moe_combine), bit-reproducible run to run.
     """
 
     def __init__(self, shape: BlockShape, params: BlockParams, T: int, x_dtype: torch.dtype,
-                 device=None):
+                 device=None, combine: str = "scatter"):
+        if combine not in ("scatter", "ordered"):
+            raise ValueError(combine)
+        self.combine_mode = combine
+        self.x_dtype = x_dtype
         self.shape, self.p, self.T = shape, params, T
         dev = torch.device(device or params.w1.device)
         self.cfg = shape.cfg()
@@ -207,13 +238,23 @@ class MoEBlock:
         self.offsets = torch.empty(shape.n_routed + 1, dtype=i32, device=dev)
         self.sorted_token = torch.empty(T * k, dtype=i32, device=dev)
         self.slot_of = torch.empty(T * k, dtype=i32, device=dev)
-        self.out_perm = torch.empty(T * k, D, dtype=f32, device=dev)
-        self.out_shared = torch.empty(T, D, dtype=f32, device=dev) if shape.n_shared else None
+        ordered = combine == "ordered"
+        self.out_perm = torch.empty(T * k if ordered else 0, D, dtype=f32, device=dev)
+        self.out_shared = (torch.empty(T if ordered else 0, D, dtype=f32, device=dev)
+                           if shape.n_shared else None)
         self.y = torch.empty(T, D, dtype=f32, device=dev)
         self.status = torch.zeros(1, dtype=i32, device=dev)
 
-    # kernels one forward launches: router 2, dispatch 3, experts 5, combine 1
-    LAUNCHES_PER_FORWARD = 11
+    # kernels one forward launches: router 3 (bf16 x on the tensor-core path:
+    # weight split, scores, selection), dispatch 3, experts 5 (two tile tables,
+    # row gather, two GEMMs), then combine 1 (ordered) or the zeroing of y
+    # (scatter, a memset node)
+    @property
+    def launches_per_forward(self) -> int:
+        sh = self.shape
+        tc_router = (self.x_dtype == torch.bfloat16 and sh.n_routed % 128 == 0
+                     and sh.dim % 64 == 0 and self.T >= 32)
+        return (3 if tc_router else 2) + 3 + 5 + (1 if self.combine_mode == "ordered" else 0)
 
     def _router(self, x, cfgp, s):
         p = self.p
@@ -231,6 +272,14 @@ class MoEBlock:
             "moe_dispatch_build")
 
     def _experts(self, x, cfgp, s):
+        if self.combine_mode == "scatter":
+            check(fn("moe_experts", "moe_experts_forward_combine")(
+                cfgp, self.T, x.data_ptr(), _dt(x), ctypes.byref(self.wstruct),
+                self.offsets.data_ptr(), self.sorted_token.data_ptr(), self.indices.data_ptr(),
+                self.weights.data_ptr(), self.y.data_ptr(), self.ws_experts.data_ptr(),
+                self.ws_experts.numel(), self.status.data_ptr(), s),
+                "moe_experts_forward_combine")
+            return
         check(fn("moe_experts", "moe_experts_forward")(
             cfgp, self.T, x.data_ptr(), _dt(x), ctypes.byref(self.wstruct),
             self.offsets.data_ptr(), self.sorted_token.data_ptr(), self.out_perm.data_ptr(),
@@ -238,6 +287,8 @@ class MoEBlock:
             self.status.data_ptr(), s), "moe_experts_forward")
 
     def _combine(self, cfgp, s):
+        if self.combine_mode == "scatter":
+            return  # done inside the experts' second matmul
         check(fn("moe_combine", "moe_combine")(
             cfgp, self.T, self.weights.data_ptr(), self.slot_of.data_ptr(),
             self.out_perm.data_ptr(), _ptr(self.out_shared), self.y.data_ptr(),

@@ -43,8 +43,11 @@ def block_work(D, E, I, k, S, T, n_touched, w_bytes, x_bytes, scale_bytes_per_ex
     return Work(weights + router + io, flops)
 
 
-def kernel_work(D, E, I, k, S, T, n_touched, w_bytes, x_bytes, scale_bytes_per_expert=0.0):
-    """Per kernel of one forward: the bytes it must move and flops it must do."""
+def kernel_work(D, E, I, k, S, T, n_touched, w_bytes, x_bytes, scale_bytes_per_expert=0.0,
+                scatter=False):
+    """Per kernel of one forward: the bytes it must move and flops it must do.
+    With scatter=True the second matmul adds the gated outputs into y itself
+    (y written once, no per-slot outputs) and there is no combine pass."""
     rows = T * k + T * S                       # expert-contiguous rows incl. the shared expert
     n_w = n_touched + S                        # weight matrices actually streamed
     sc = scale_bytes_per_expert / 3.0          # per matrix
@@ -55,9 +58,9 @@ def kernel_work(D, E, I, k, S, T, n_touched, w_bytes, x_bytes, scale_bytes_per_e
         # W1 and W3 of each touched expert, the rows in, h out
         "gemm1": Work(n_w * (2 * D * I * w_bytes + 2 * sc) + rows * D * 2 + rows * I * 2,
                       rows * 2 * 2 * D * I),
-        # W2 of each touched expert, h in, fp32 expert outputs out
-        "gemm2": Work(n_w * (D * I * w_bytes + sc) + rows * I * 2 + rows * D * 4,
-                      rows * 2 * D * I),
+        # W2 of each touched expert, h in, fp32 expert outputs (or y) out
+        "gemm2": Work(n_w * (D * I * w_bytes + sc) + rows * I * 2 +
+                      (T * D * 4 if scatter else rows * D * 4), rows * 2 * D * I),
         # k expert rows and the shared row in, y out (all fp32)
         "combine": Work(rows * D * 4 + T * D * 4 + T * k * 8, T * (k + S) * D * 2),
     }

@@ -117,6 +117,14 @@ def test_experts_validation():
     assert call(wt=fp8) == INVALID                             # e4m3 needs block scales
     bad = MoEExpertWeights(0x1000, 0x1000, 0x1000, 7, None, None, None)
     assert call(wt=bad) == UNSUPPORTED
+    fc = fn("moe_experts", "moe_experts_forward_combine")
+    # missing router outputs or y
+    assert fc(ctypes.byref(c), 8, P, 1, ctypes.byref(w), P, P, None, P, P, P, 1 << 40, None,
+              None) == INVALID
+    assert fc(ctypes.byref(c), 8, P, 1, ctypes.byref(w), P, P, P, P, None, P, 1 << 40, None,
+              None) == INVALID
+    assert fc(ctypes.byref(c), 8, P, 1, ctypes.byref(w), P, P, P, P, P, P, 8, None,
+              None) == WORKSPACE
 
 
 def test_combine_and_selftest_validation():

@@ -54,8 +54,8 @@ def built():
     assert torch.cuda.is_available()
 
 
-def run_block(w, x, params):
-    blk = moe.MoEBlock(w.shape, params, w.T, x.dtype)
+def run_block(w, x, params, combine="scatter"):
+    blk = moe.MoEBlock(w.shape, params, w.T, x.dtype, combine=combine)
     y = blk.forward(x).clone()
     torch.cuda.synchronize()
     assert blk.device_status() == 0
@@ -154,12 +154,13 @@ def test_experts_rows_match_oracle(w):
     assert mean_sum / n <= MEAN_TOL[w.w_format], mean_sum / n
 
 
+@pytest.mark.parametrize("combine", ["scatter", "ordered"])
 @pytest.mark.parametrize("w", [WORKLOADS["tiny_f32"], TINY_BF16, MID, MID_F32, SOFTMAX_NOBIAS,
-                               ONE_GROUP, DECODE_SMALL, ONE_TOKEN, FP8_SMALL],
+                               ONE_GROUP, DECODE_SMALL, ONE_TOKEN, CG1_PREFILL, FP8_SMALL],
                          ids=lambda w: w.name)
-def test_block_matches_oracle(w):
+def test_block_matches_oracle(w, combine):
     x, p = make_block(w)
-    blk, y = run_block(w, x, p)
+    blk, y = run_block(w, x, p, combine)
     r = oracle_route(w, x, p)
     rep = compare_routing(r, blk.weights.cpu().numpy(),
                           blk.indices.cpu().numpy().astype(np.int64),
@@ -173,13 +174,23 @@ def test_block_matches_oracle(w):
         assert np.array_equal(blk.counts.cpu().numpy(), d.counts)
 
 
-def test_block_is_deterministic():
+def test_ordered_combine_is_bit_reproducible():
     x, p = make_block(MID)
-    blk = moe.MoEBlock(MID.shape, p, MID.T, x.dtype)
+    blk = moe.MoEBlock(MID.shape, p, MID.T, x.dtype, combine="ordered")
     y1 = blk.forward(x).clone()
     y2 = blk.forward(x).clone()
     torch.cuda.synchronize()
     assert torch.equal(y1, y2)
+
+
+def test_scatter_and_ordered_combine_agree():
+    x, p = make_block(MID)
+    ys = moe.MoEBlock(MID.shape, p, MID.T, x.dtype, combine="scatter").forward(x).clone()
+    yo = moe.MoEBlock(MID.shape, p, MID.T, x.dtype, combine="ordered").forward(x).clone()
+    torch.cuda.synchronize()
+    rms = yo.pow(2).mean().sqrt()
+    # same fp32 terms, summed in different orders
+    assert float((ys - yo).abs().max() / rms) < 1e-5
 
 
 def test_zero_input_gives_zero_output_and_uniform_gates():
