@@ -201,10 +201,11 @@ def test_zero_input_gives_zero_output_and_uniform_gates():
     assert torch.all(blk.weights == 2.5 / 4)
 
 
-def test_graph_capture_replays():
+@pytest.mark.parametrize("combine", ["scatter", "ordered"])
+def test_graph_capture_replays(combine):
     w = TINY_BF16
     x, p = make_block(w)
-    blk = moe.MoEBlock(w.shape, p, w.T, x.dtype)
+    blk = moe.MoEBlock(w.shape, p, w.T, x.dtype, combine=combine)
     ref = blk.forward(x).clone()
     s = torch.cuda.Stream()
     s.wait_stream(torch.cuda.current_stream())
@@ -217,7 +218,10 @@ def test_graph_capture_replays():
     blk.y.zero_()
     g.replay()
     torch.cuda.synchronize()
-    assert torch.equal(blk.y, ref)
+    if combine == "ordered":
+        assert torch.equal(blk.y, ref)
+    else:  # fp32 reductions in a run-dependent order
+        assert float((blk.y - ref).abs().max() / ref.pow(2).mean().sqrt()) < 1e-5
 
 
 def test_bounded_wait_reports_timeout_and_context_survives():
