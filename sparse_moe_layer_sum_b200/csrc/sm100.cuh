@@ -267,6 +267,31 @@ __device__ __forceinline__ void tma_load_2d_pair(const CUtensorMap *m, void *dst
       : "memory");
 }
 
+// Four rows (row0..row3, each one 128-byte box) of a 2-D tensor into
+// consecutive 128-byte rows of shared memory: the rows are gathered by index.
+__device__ __forceinline__ void tma_gather4(const CUtensorMap *m, void *dst, uint64_t *bar,
+                                            int32_t x, int4 rows, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
+      ".L2::cache_hint [%0], [%1, {%2, %3, %4, %5, %6}], [%7], %8;" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(m)), "r"(x), "r"(rows.x), "r"(rows.y), "r"(rows.z),
+      "r"(rows.w), "r"(smem_u32(bar)), "l"(policy)
+      : "memory");
+}
+
+// Same, counted on an mbarrier of either CTA of the pair.
+__device__ __forceinline__ void tma_gather4_pair(const CUtensorMap *m, void *dst,
+                                                 uint32_t mbar_cluster_addr, int32_t x, int4 rows,
+                                                 uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.tile::gather4.mbarrier::"
+      "complete_tx::bytes.L2::cache_hint [%0], [%1, {%2, %3, %4, %5, %6}], [%7], %8;" ::"r"(
+          smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(m)), "r"(x), "r"(rows.x), "r"(rows.y), "r"(rows.z),
+      "r"(rows.w), "r"(mbar_cluster_addr), "l"(policy)
+      : "memory");
+}
+
 __device__ __forceinline__ void tmem_alloc_pair(uint32_t *slot, uint32_t ncols) {
   asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                    smem_u32(slot)),
