@@ -5,18 +5,16 @@
 // · Mixture of experts" that matches that page's per-expert count of
 // 3 * 7168 * 2048 parameters.  The shared expert runs on every token.
 //
-// Tensor-core path (bf16 activations and weights), sm_100a:
-//   GEMM1         h = silu(X W1^T) * (X W3^T), bf16 out; the token rows of
-//                 each expert are gathered from x by the TMA (tile::gather4)
-//   GEMM2         o = h W2^T, fp32 out (or gated and added into y)
+// Tensor-core path (bf16 activations; bf16 or e4m3 weights), sm_100a:
+//   gather_rows   X_perm[p] = x[sorted_token[p]] (expert-contiguous rows),
+//                 followed by the T rows of x for the shared expert.
+//   GEMM1         h = silu(X W1^T) * (X W3^T), bf16 out
+//   GEMM2         o = h W2^T, fp32 out
 // Both GEMMs are one persistent, warp-specialised kernel template
-// (tc_expert_gemm): warp 0 streams weight tiles from HBM into a deep
-// shared-memory ring, warp 6 streams token rows into a shallower one (they
-// come from L2 at lower latency), one thread of warp 1 issues tcgen05.mma
-// into a double-buffered TMEM accumulator, and warps 2-5 drain the
-// accumulator with tcgen05.ld and run the epilogue while the next tile's
-// MMAs proceed.  At prefill sizes a tile runs on an SM pair (cta_group::2,
-// M = 256): each SM streams its own 128 weight rows and half of the tokens.
+// (tc_expert_gemm): warp 0 issues TMA loads into a shared-memory ring, one
+// thread of warp 1 issues tcgen05.mma into a double-buffered TMEM
+// accumulator, warps 2-5 drain the accumulator with tcgen05.ld and run the
+// epilogue while the next tile's MMAs proceed.
 //
 // The operands are swapped relative to the usual token-major GEMM: the 128
 // rows of an MMA (M) are weight rows and the MMA's N is the expert's tokens.
@@ -140,16 +138,31 @@ __device__ __forceinline__ Tile decode_tile(int tile, const int32_t *tstart, con
   return t;
 }
 
+// ------------------------------------------------------------------ gather
+
+// X_perm[p] = x[sorted_token[p]] for p < rows_routed, then x itself for the
+// shared expert's rows.  One warp per row, 16-byte vectors.
+__global__ void __launch_bounds__(256) gather_rows(const uint4 *__restrict__ x,
+                                                   const int32_t *__restrict__ sorted_token,
+                                                   uint4 *__restrict__ xp, int rows_routed,
+                                                   int rows_total, int T, int vec_per_row) {
+  const int row = (int)((blockIdx.x * (size_t)blockDim.x + threadIdx.x) / 32);
+  const int lane = threadIdx.x % 32;
+  if (row >= rows_total) return;
+  const int src = row < rows_routed ? sorted_token[row] : (row - rows_routed) % T;
+  const uint4 *s = x + (size_t)src * vec_per_row;
+  uint4 *d = xp + (size_t)row * vec_per_row;
+  for (int v = lane; v < vec_per_row; v += 32) d[v] = __ldg(s + v);
+}
+
 // ------------------------------------------------------- tensor-core GEMMs
 
 namespace tc {
 
 constexpr int BK = 64;                 // K elements per ring stage (128 bytes bf16)
-constexpr int BM = 128;                // MMA M per CTA: weight rows per tile
+constexpr int BM = 128;                // MMA M: weight rows per tile
 constexpr int A_BYTES = BM * BK * 2;   // 16 KB
-// warp 0 streams weights (A), warp 1 issues MMAs, warps 2-5 run the
-// epilogue, warp 6 streams token rows (B)
-constexpr int THREADS = 224;
+constexpr int THREADS = 192;           // warp 0 TMA, warp 1 MMA, warps 2-5 epilogue
 constexpr int EPI_WARPS = 4;
 constexpr int XB_STRIDE = 17;          // exchange buffer row stride (floats)
 
@@ -165,7 +178,7 @@ struct Params {
   float *out_shared;
   int32_t *status;
   int64_t timeout_ns;
-  // GEMM1 token rows (gathered from x); MODE 3 gates
+  // MODE 3 (second GEMM with the weighted scatter into y)
   const int32_t *sorted_token;
   const int32_t *indices;  // [T, k]
   const float *weights;    // [T, k]
@@ -173,44 +186,33 @@ struct Params {
   float *y;                // [T, D], zeroed before the launch
 };
 
-constexpr int align_to(int v, int a) { return (v + a - 1) / a * a; }
-
-// MODE 1: h = silu(x w1^T) * (x w3^T), token rows gathered from x.
-// MODE 2: o = h w2^T into out_perm / out_shared.  MODE 3: same GEMM, gated
-// outputs added into y.  CG = CTA group: 1 = one SM per tile; 2 = an SM pair
-// per tile (cta_group::2), each CTA holding 128 weight rows and half of the
-// token rows.  SA / SB: depths of the weight ring and the token ring.
-template <int MODE, int CG, int BN_MAX, int SA, int SB>
+// CG = CTA group: 1 = one SM per tile; 2 = an SM pair per tile (cta_group::2),
+// where each CTA holds 128 weight rows and half of the token tile.
+template <int MODE, int CG, int BN_MAX, int BOXN, int STAGES>
 struct Layout {
-  static constexpr bool GATHER = MODE == 1;
   static constexpr int B_ROWS = BN_MAX / CG;  // token rows one CTA holds per stage
   static constexpr int B_BYTES = B_ROWS * BK * 2;
-  static constexpr int BOXN = 32;             // rows per box load of h (MODE 2, 3)
-  static constexpr int B_OFF = SA * A_BYTES;
-  static constexpr int BAR_OFF = B_OFF + SB * B_BYTES;
-  // fullA, emptyA, fullB, emptyB, acc_full x2, acc_empty x2, drain
-  static constexpr int NBARS = 2 * SA + 2 * SB + 5;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int BAR_OFF = STAGES * STAGE_BYTES;
+  static constexpr int NBARS = 2 * STAGES + 5;  // full, empty, acc_full x2, acc_empty x2, drain
   static constexpr int MISC_OFF = BAR_OFF + NBARS * 8;
-  static constexpr int MISC_BYTES = 16 + 4 * (SA + SB);
-  static constexpr int TOK_OFF = align_to(MISC_OFF + MISC_BYTES, 16);
-  static constexpr int TOK_BYTES = GATHER ? B_ROWS * 4 : 0;
-  static constexpr int XBUF_OFF = align_to(TOK_OFF + TOK_BYTES, 128);
+  static constexpr int MISC_BYTES = 16 + 4 * STAGES;
+  static constexpr int XBUF_OFF = (MISC_OFF + MISC_BYTES + 127) / 128 * 128;
   // GEMM1: SwiGLU exchange buffers; MODE 3: the tile's (token, gate) list
-  static constexpr int XBUF_BYTES =
-      MODE == 1 ? 2 * 2 * 32 * XB_STRIDE * 4 : MODE == 3 ? BN_MAX * 8 : 0;
+  static constexpr int XBUF_BYTES = MODE == 1 ? 2 * 2 * 32 * XB_STRIDE * 4 : MODE == 3 ? BN_MAX * 8 : 0;
   static constexpr int TAB_OFF = XBUF_OFF + XBUF_BYTES;
   static constexpr uint32_t TMEM_COLS =
       2 * BN_MAX <= 32 ? 32 : 2 * BN_MAX <= 64 ? 64 : 2 * BN_MAX <= 128 ? 128
                                                 : 2 * BN_MAX <= 256 ? 256 : 512;
   // weight rows one tile covers: GEMM1 pairs 64 rows of w1 with the same 64
-  // rows of w3 per CTA; the second GEMM takes 128 rows of w2 per CTA
-  static constexpr int FEAT = (MODE == 1 ? 64 : BM) * CG;
+  // rows of w3 per CTA; GEMM2 takes 128 rows of w2 per CTA
+  static constexpr int FEAT = (MODE == 1 ? 64 : BM) * CG;  // MODE 2 and 3: rows of w2
   static size_t smem_bytes(int G, int E) {
     return 1024 + TAB_OFF + sizeof(int32_t) * (size_t)((G + 1) + G + (E + 1));
   }
   static_assert(CG == 1 || CG == 2, "CTA group");
   static_assert(BN_MAX % 16 == 0 && BN_MAX >= 16 && BN_MAX <= 256, "MMA N range");
-  static_assert(GATHER ? B_ROWS % 8 == 0 : B_ROWS % BOXN == 0, "token rows per stage");
+  static_assert(BOXN % 16 == 0 && B_ROWS % BOXN == 0, "B box rows");
 };
 
 // Waits for a barrier phase with a time limit but ignores the abort flag;
@@ -228,27 +230,23 @@ __device__ __forceinline__ void sleep_ns(int64_t ns) {
   }
 }
 
-template <int MODE, int CG, int BN_MAX, int SA, int SB>
+template <int MODE, int CG, int BN_MAX, int BOXN, int STAGES>
 __global__ void __launch_bounds__(THREADS, 1)
     tc_expert_gemm(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA1,
                    const __grid_constant__ CUtensorMap tmB, const Params p) {
-  using L = Layout<MODE, CG, BN_MAX, SA, SB>;
+  using L = Layout<MODE, CG, BN_MAX, BOXN, STAGES>;
   using namespace sm100;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                             ~static_cast<uintptr_t>(1023));
-  uint64_t *fullA = reinterpret_cast<uint64_t *>(sm + L::BAR_OFF);
-  uint64_t *emptyA = fullA + SA;
-  uint64_t *fullB = emptyA + SA;
-  uint64_t *emptyB = fullB + SB;
-  uint64_t *accf = emptyB + SB;
+  uint64_t *full = reinterpret_cast<uint64_t *>(sm + L::BAR_OFF);
+  uint64_t *empty = full + STAGES;
+  uint64_t *accf = empty + STAGES;
   uint64_t *acce = accf + 2;
   uint64_t *drain = acce + 2;
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + L::MISC_OFF);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + L::MISC_OFF + 4);
-  volatile int *pendA = reinterpret_cast<volatile int *>(sm + L::MISC_OFF + 16);
-  volatile int *pendB = pendA + SA;
-  int32_t *s_tok = reinterpret_cast<int32_t *>(sm + L::TOK_OFF);
+  volatile int *pending = reinterpret_cast<volatile int *>(sm + L::MISC_OFF + 16);
   float *xbuf = reinterpret_cast<float *>(sm + L::XBUF_OFF);
   int32_t *s_tstart = reinterpret_cast<int32_t *>(sm + L::TAB_OFF);
   int32_t *s_tbase = s_tstart + p.G + 1;
@@ -262,15 +260,10 @@ __global__ void __launch_bounds__(THREADS, 1)
   const int nunits = CG == 2 ? (int)cluster_count_x() : (int)gridDim.x;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < SA; ++s) {
-      mbar_init(fullA + s, 1);
-      mbar_init(emptyA + s, 1);
-      pendA[s] = -1;
-    }
-    for (int s = 0; s < SB; ++s) {
-      mbar_init(fullB + s, 1);
-      mbar_init(emptyB + s, 1);
-      pendB[s] = -1;
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(full + s, 1);
+      mbar_init(empty + s, 1);
+      pending[s] = -1;
     }
     mbar_init(accf + 0, 1);
     mbar_init(accf + 1, 1);
@@ -304,124 +297,66 @@ __global__ void __launch_bounds__(THREADS, 1)
 
   if (warp == 0) {
     if (lane == 0) {
-      // ------------------------------------------- weight (A) producer
+      // ---------------------------------------------------- TMA producer
       const uint64_t pol_w = policy_evict_first();  // weights: streamed once
+      const uint64_t pol_x = policy_evict_last();   // activations: re-read per feature tile
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
       for (int tile = unit; ok && tile < total; tile += nunits) {
         const Tile t = decode_tile(tile, s_tstart, s_tbase, s_off, p.G, p.E, p.T, p.rows_routed);
+        const int nmma = (t.nvalid + 15) & ~15;
+        const int brows = nmma / CG;  // this CTA's share of the token rows
+        const int b0 = t.rowbase + t.n0 + (int)rank * brows;
         const int arow = MODE == 1 ? t.g * p.I + t.ft * L::FEAT + (int)rank * 64
                                    : t.g * p.D + t.ft * L::FEAT + (int)rank * BM;
+        const int nbox = (brows + BOXN - 1) / BOXN;
+        const uint32_t bytes = (uint32_t)(A_BYTES + nbox * BOXN * BK * 2);
         const int k0 = k_rotation(t, p.KB);
         for (int i = 0; i < p.KB; ++i) {
           const int kb = k0 + i < p.KB ? k0 + i : k0 + i - p.KB;
-          if (!wait_bounded(emptyA + stage, phase ^ 1u, abort_flag, p.timeout_ns, p.status)) {
+          if (!wait_bounded(empty + stage, phase ^ 1u, abort_flag, p.timeout_ns, p.status)) {
             ok = false;
             break;
           }
           // the leader's full barrier counts the bytes of both CTAs
-          if (leader) mbar_arrive_expect_tx(fullA + stage, A_BYTES * CG);
-          pendA[stage] = (int)phase;
-          uint8_t *dst = sm + stage * A_BYTES;
+          if (leader) mbar_arrive_expect_tx(full + stage, bytes * CG);
+          pending[stage] = (int)phase;
+          uint8_t *a_dst = sm + stage * L::STAGE_BYTES;
+          uint8_t *b_dst = a_dst + A_BYTES;
           if (CG == 2) {
-            const uint32_t fb = mapa_shared(smem_u32(fullA + stage), 0);
+            const uint32_t fb = mapa_shared(smem_u32(full + stage), 0);
             if (MODE == 1) {
-              tma_load_2d_pair(&tmA0, dst, fb, kb * BK, arow, pol_w);
-              tma_load_2d_pair(&tmA1, dst + A_BYTES / 2, fb, kb * BK, arow, pol_w);
+              tma_load_2d_pair(&tmA0, a_dst, fb, kb * BK, arow, pol_w);
+              tma_load_2d_pair(&tmA1, a_dst + A_BYTES / 2, fb, kb * BK, arow, pol_w);
             } else {
-              tma_load_2d_pair(&tmA0, dst, fb, kb * BK, arow, pol_w);
+              tma_load_2d_pair(&tmA0, a_dst, fb, kb * BK, arow, pol_w);
             }
+            for (int i = 0; i < nbox; ++i)
+              tma_load_2d_pair(&tmB, b_dst + i * BOXN * BK * 2, fb, kb * BK, b0 + i * BOXN, pol_x);
           } else {
             if (MODE == 1) {
-              tma_load_2d_hint(&tmA0, dst, fullA + stage, kb * BK, arow, pol_w);
-              tma_load_2d_hint(&tmA1, dst + A_BYTES / 2, fullA + stage, kb * BK, arow, pol_w);
+              tma_load_2d_hint(&tmA0, a_dst, full + stage, kb * BK, arow, pol_w);
+              tma_load_2d_hint(&tmA1, a_dst + A_BYTES / 2, full + stage, kb * BK, arow, pol_w);
             } else {
-              tma_load_2d_hint(&tmA0, dst, fullA + stage, kb * BK, arow, pol_w);
+              tma_load_2d_hint(&tmA0, a_dst, full + stage, kb * BK, arow, pol_w);
             }
+            for (int i = 0; i < nbox; ++i)
+              tma_load_2d_hint(&tmB, b_dst + i * BOXN * BK * 2, full + stage, kb * BK,
+                               b0 + i * BOXN, pol_x);
           }
-          if (++stage == SA) {
+          if (++stage == STAGES) {
             stage = 0;
             phase ^= 1u;
           }
         }
       }
     }
-  } else if (warp == 6) {
-    // ---------------------------------------------- token (B) producer
-    const uint64_t pol_x = policy_evict_last();  // token rows: re-read per feature tile
-    int stage = 0;
-    uint32_t phase = 0;
-    bool ok = true;
-    for (int tile = unit; ok && tile < total; tile += nunits) {
-      const Tile t = decode_tile(tile, s_tstart, s_tbase, s_off, p.G, p.E, p.T, p.rows_routed);
-      const int nmma = (t.nvalid + 15) & ~15;
-      const int brows = nmma / CG;  // this CTA's share of the token rows
-      const int r0 = (int)rank * brows;
-      int nload;   // TMA instructions per stage
-      uint32_t bytes;
-      if (L::GATHER) {
-        // this tile's token list; rows past the expert's tokens repeat its last
-        // token (their accumulator columns are never stored)
-        __syncwarp();
-        for (int r = lane; r < brows; r += 32) {
-          const int row = min(r0 + r, t.nvalid - 1);
-          s_tok[r] = t.g < p.E ? p.sorted_token[t.rowbase + t.n0 + row] : t.n0 + row;
-        }
-        __syncwarp();
-        nload = brows / 4;
-        bytes = (uint32_t)(brows * BK * 2);
-      } else {
-        nload = (brows + L::BOXN - 1) / L::BOXN;
-        bytes = (uint32_t)(nload * L::BOXN * BK * 2);
-      }
-      const int b0 = t.rowbase + t.n0 + r0;  // first row in h (MODE 2, 3)
-      const int k0 = k_rotation(t, p.KB);
-      for (int i = 0; i < p.KB; ++i) {
-        const int kb = k0 + i < p.KB ? k0 + i : k0 + i - p.KB;
-        int got = 1;
-        if (lane == 0) {
-          got = wait_bounded(emptyB + stage, phase ^ 1u, abort_flag, p.timeout_ns, p.status);
-          if (got) {
-            if (leader) mbar_arrive_expect_tx(fullB + stage, bytes * CG);
-            pendB[stage] = (int)phase;
-          }
-        }
-        if (!__shfl_sync(0xffffffffu, got, 0)) {
-          ok = false;
-          break;
-        }
-        uint8_t *dst = sm + L::B_OFF + stage * L::B_BYTES;
-        const uint32_t fb = CG == 2 ? mapa_shared(smem_u32(fullB + stage), 0) : 0u;
-        if (L::GATHER) {
-          for (int l = lane; l < nload; l += 32) {
-            const int4 rows = *reinterpret_cast<const int4 *>(s_tok + 4 * l);
-            if (CG == 2)
-              tma_gather4_pair(&tmB, dst + l * 4 * BK * 2, fb, kb * BK, rows, pol_x);
-            else
-              tma_gather4(&tmB, dst + l * 4 * BK * 2, fullB + stage, kb * BK, rows, pol_x);
-          }
-        } else if (lane == 0) {
-          for (int l = 0; l < nload; ++l) {
-            if (CG == 2)
-              tma_load_2d_pair(&tmB, dst + l * L::BOXN * BK * 2, fb, kb * BK, b0 + l * L::BOXN,
-                               pol_x);
-            else
-              tma_load_2d_hint(&tmB, dst + l * L::BOXN * BK * 2, fullB + stage, kb * BK,
-                               b0 + l * L::BOXN, pol_x);
-          }
-        }
-        if (++stage == SB) {
-          stage = 0;
-          phase ^= 1u;
-        }
-      }
-    }
   } else if (warp == 1) {
     if (lane == 0 && leader) {
       // ------------------------------------------------------ MMA issuer
-      int sa = 0, sb = 0, acc = 0;
-      uint32_t pa = 0, pb = 0, acc_phase = 0;
+      int stage = 0, acc = 0;
+      uint32_t phase = 0, acc_phase = 0;
       bool ok = true;
       for (int tile = unit; ok && tile < total; tile += nunits) {
         const Tile t = decode_tile(tile, s_tstart, s_tbase, s_off, p.G, p.E, p.T, p.rows_routed);
@@ -434,16 +369,14 @@ __global__ void __launch_bounds__(THREADS, 1)
         const int nmma = (t.nvalid + 15) & ~15;
         const uint32_t idesc = idesc_bf16_f32(BM * CG, nmma);
         for (int kb = 0; kb < p.KB; ++kb) {
-          if (!wait_bounded(fullA + sa, pa, abort_flag, p.timeout_ns, p.status) ||
-              !wait_bounded(fullB + sb, pb, abort_flag, p.timeout_ns, p.status)) {
+          if (!wait_bounded(full + stage, phase, abort_flag, p.timeout_ns, p.status)) {
             ok = false;
             break;
           }
-          pendA[sa] = -1;
-          pendB[sb] = -1;
+          pending[stage] = -1;
           tc_fence_after();
-          const uint32_t a_addr = smem_u32(sm + sa * A_BYTES);
-          const uint32_t b_addr = smem_u32(sm + L::B_OFF + sb * L::B_BYTES);
+          const uint32_t a_addr = smem_u32(sm + stage * L::STAGE_BYTES);
+          const uint32_t b_addr = a_addr + A_BYTES;
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk) {
             const uint64_t ad = sdesc_sw128(a_addr + kk * 32), bd = sdesc_sw128(b_addr + kk * 32);
@@ -453,20 +386,13 @@ __global__ void __launch_bounds__(THREADS, 1)
             else
               mma_bf16(d_tmem, ad, bd, idesc, accum);
           }
-          if (CG == 2) {
-            mma_commit_pair_mc(emptyA + sa, 0x3);
-            mma_commit_pair_mc(emptyB + sb, 0x3);
-          } else {
-            mma_commit(emptyA + sa);
-            mma_commit(emptyB + sb);
-          }
-          if (++sa == SA) {
-            sa = 0;
-            pa ^= 1u;
-          }
-          if (++sb == SB) {
-            sb = 0;
-            pb ^= 1u;
+          if (CG == 2)
+            mma_commit_pair_mc(empty + stage, 0x3);
+          else
+            mma_commit(empty + stage);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
           }
         }
         if (!ok) break;
@@ -499,8 +425,8 @@ __global__ void __launch_bounds__(THREADS, 1)
       if (MODE == 3) {
         // weighted scatter into y: y[t, d] += gate(t) * o[t, d] (gate 1 for the
         // shared expert), with fp32 reductions; first the tile's token list
-        int32_t *l_tok = reinterpret_cast<int32_t *>(xbuf);
-        float *l_gate = reinterpret_cast<float *>(l_tok + BN_MAX);
+        int32_t *s_tok = reinterpret_cast<int32_t *>(xbuf);
+        float *s_gate = reinterpret_cast<float *>(s_tok + BN_MAX);
         const int et = threadIdx.x - 64;  // 0..127 over the four epilogue warps
         named_bar_sync(3, 128);            // the previous tile's readers are done
         for (int c = et; c < t.nvalid; c += 128) {
@@ -513,8 +439,8 @@ __global__ void __launch_bounds__(THREADS, 1)
           } else {
             tok = t.n0 + c;
           }
-          l_tok[c] = tok;
-          l_gate[c] = gate;
+          s_tok[c] = tok;
+          s_gate[c] = gate;
         }
         named_bar_sync(3, 128);
         const int d = t.ft * L::FEAT + (int)rank * BM + q * 32 + lane;
@@ -525,7 +451,7 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
           for (int j = 0; j < 32; ++j)
             if (c0 + j < t.nvalid)
-              atomicAdd(p.y + (size_t)l_tok[c0 + j] * p.D + d, l_gate[c0 + j] * __uint_as_float(v[j]));
+              atomicAdd(p.y + (size_t)s_tok[c0 + j] * p.D + d, s_gate[c0 + j] * __uint_as_float(v[j]));
         }
       } else if (MODE == 2) {
         // lanes are output features d, columns are tokens
@@ -598,10 +524,8 @@ __global__ void __launch_bounds__(THREADS, 1)
     // leader's full barriers count both CTAs' copies; the other CTA of a pair
     // cannot wait on them and just allows its copies time to land.
     if (leader) {
-      for (int s = 0; s < SA; ++s)
-        if (pendA[s] >= 0) drain_wait(fullA + s, (uint32_t)pendA[s], p.timeout_ns);
-      for (int s = 0; s < SB; ++s)
-        if (pendB[s] >= 0) drain_wait(fullB + s, (uint32_t)pendB[s], p.timeout_ns);
+      for (int s = 0; s < STAGES; ++s)
+        if (pending[s] >= 0) drain_wait(full + s, (uint32_t)pending[s], p.timeout_ns);
     } else {
       sleep_ns(200000);
     }
@@ -816,7 +740,7 @@ int sm_count() {
 }
 
 struct WsLayout {
-  size_t tab, h, total;
+  size_t tab, xperm, h, total;
   int64_t rows_pad;
 };
 
@@ -833,19 +757,20 @@ WsLayout ws_layout(const moe_cfg *c, int64_t T, moe_dtype x_dt, moe_dtype w_dt) 
   l.tab = 0;
   size_t off = align_up(sizeof(int32_t) * (size_t)(4 * G + 4), 1024);
   const bool tc = tc_path(c, x_dt, w_dt);
+  l.xperm = off;
+  if (tc) off = align_up(off + (size_t)l.rows_pad * c->dim * 2, 1024);
   l.h = off;
   off = align_up(off + (size_t)l.rows_pad * c->inter * (tc ? 2 : 4), 1024);
   l.total = off;
   return l;
 }
 
-template <int MODE, int CG, int BN_MAX, int SA, int SB>
+template <int MODE, int CG, int BN_MAX, int BOXN, int STAGES>
 moe_status launch_tc(const CUtensorMap &a0, const CUtensorMap &a1, const CUtensorMap &b,
                      const tc::Params &p, cudaStream_t s) {
-  using L = tc::Layout<MODE, CG, BN_MAX, SA, SB>;
-  auto kern = tc::tc_expert_gemm<MODE, CG, BN_MAX, SA, SB>;
+  using L = tc::Layout<MODE, CG, BN_MAX, BOXN, STAGES>;
+  auto kern = tc::tc_expert_gemm<MODE, CG, BN_MAX, BOXN, STAGES>;
   const size_t smem = L::smem_bytes(p.G, p.E);
-  if (smem > 232448) return MOE_ERR_UNSUPPORTED;  // too many experts for the tile tables
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
       cudaSuccess)
     return MOE_ERR_CUDA;
@@ -933,7 +858,7 @@ tc::Params tc_params(const Job &j) {
   return p;
 }
 
-template <int CG, int BN_MAX, int SA, int SB>
+template <int CG, int BN_MAX, int BOXN, int STAGES>
 moe_status tc_up(const Job &j) {
   const int G = j.G(), D = j.c->dim, I = j.c->inter;
   int32_t *tab = j.tab();
@@ -942,27 +867,32 @@ moe_status tc_up(const Job &j) {
   prep_tiles<<<1, 32, 0, j.s>>>(j.offsets, j.E(), G, (int)j.T, t1, none);
   moe_status st = launch_status();
   if (st != MOE_OK) return st;
+  bf16 *xperm = reinterpret_cast<bf16 *>(j.ws + j.l.xperm);
   bf16 *h = reinterpret_cast<bf16 *>(j.ws + j.l.h);
+  prof(0, j.s);
+  const int64_t threads = (int64_t)j.rows_total() * 32;
+  gather_rows<<<(unsigned)((threads + 255) / 256), 256, 0, j.s>>>(
+      static_cast<const uint4 *>(j.x), j.sorted_token, reinterpret_cast<uint4 *>(xperm),
+      j.rows_routed(), j.rows_total(), (int)j.T, D * 2 / 16);
+  if ((st = launch_status()) != MOE_OK) return st;
   CUtensorMap mw1, mw3, mx;
   const CUtensorMapDataType BF = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
-  // x rows are gathered four at a time: a box is one row of 64 columns
   if (!make_tmap(&mw1, j.w->w1, BF, 2, (uint64_t)G * I, D, 64, 64) ||
       !make_tmap(&mw3, j.w->w3, BF, 2, (uint64_t)G * I, D, 64, 64) ||
-      !make_tmap(&mx, j.x, BF, 2, (uint64_t)j.T, D, 1, 64))
+      !make_tmap(&mx, xperm, BF, 2, (uint64_t)j.l.rows_pad, D, BOXN, 64))
     return MOE_ERR_CUDA;
   tc::Params p = tc_params(j);
   p.tile_start = t1.tile_start;
   p.tile_base = t1.tile_base;
   p.KB = D / tc::BK;
   p.out = h;
-  prof(0, j.s);
   prof(1, j.s);
-  st = launch_tc<1, CG, BN_MAX, SA, SB>(mw1, mw3, mx, p, j.s);
+  st = launch_tc<1, CG, BN_MAX, BOXN, STAGES>(mw1, mw3, mx, p, j.s);
   prof(2, j.s);
   return st;
 }
 
-template <int CG, int BN_MAX, int SA, int SB>
+template <int CG, int BN_MAX, int BOXN, int STAGES>
 moe_status tc_down(const Job &j) {
   const int G = j.G(), D = j.c->dim, I = j.c->inter;
   int32_t *tab = j.tab();
@@ -975,7 +905,7 @@ moe_status tc_down(const Job &j) {
   CUtensorMap mw2, mh;
   const CUtensorMapDataType BF = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   if (!make_tmap(&mw2, j.w->w2, BF, 2, (uint64_t)G * D, I, tc::BM, 64) ||
-      !make_tmap(&mh, h, BF, 2, (uint64_t)j.l.rows_pad, I, 32, 64))
+      !make_tmap(&mh, h, BF, 2, (uint64_t)j.l.rows_pad, I, BOXN, 64))
     return MOE_ERR_CUDA;
   tc::Params p = tc_params(j);
   p.tile_start = t2.tile_start;
@@ -984,9 +914,9 @@ moe_status tc_down(const Job &j) {
   p.out = j.out_perm;
   prof(3, j.s);
   if (j.y)
-    st = launch_tc<3, CG, BN_MAX, SA, SB>(mw2, mw2, mh, p, j.s);
+    st = launch_tc<3, CG, BN_MAX, BOXN, STAGES>(mw2, mw2, mh, p, j.s);
   else
-    st = launch_tc<2, CG, BN_MAX, SA, SB>(mw2, mw2, mh, p, j.s);
+    st = launch_tc<2, CG, BN_MAX, BOXN, STAGES>(mw2, mw2, mh, p, j.s);
   prof(4, j.s);
   return st;
 }
@@ -1075,16 +1005,12 @@ moe_status simt_down_w(const Job &j) {
   return MOE_ERR_UNSUPPORTED;
 }
 
-// Tile shapes and ring depths (weight ring SA, token ring SB) of the
-// instantiations (compile-time tunables).
+// Tile shapes of the two instantiations (compile-time tunables).
 #ifndef MOE_TC_PREFILL_BN
 #define MOE_TC_PREFILL_BN 256
 #endif
-#ifndef MOE_TC_PREFILL_SA
-#define MOE_TC_PREFILL_SA 9
-#endif
-#ifndef MOE_TC_PREFILL_SB
-#define MOE_TC_PREFILL_SB 4
+#ifndef MOE_TC_PREFILL_STAGES
+#define MOE_TC_PREFILL_STAGES 6
 #endif
 #ifndef MOE_TC_PREFILL_CG
 #define MOE_TC_PREFILL_CG 2
@@ -1092,14 +1018,11 @@ moe_status simt_down_w(const Job &j) {
 #ifndef MOE_TC_DECODE_BN
 #define MOE_TC_DECODE_BN 32
 #endif
-#ifndef MOE_TC_DECODE_SA
-#define MOE_TC_DECODE_SA 12
+#ifndef MOE_TC_DECODE_STAGES
+#define MOE_TC_DECODE_STAGES 10
 #endif
-#ifndef MOE_TC_DECODE_SB
-#define MOE_TC_DECODE_SB 4
-#endif
-constexpr int PF_BN = MOE_TC_PREFILL_BN, PF_SA = MOE_TC_PREFILL_SA, PF_SB = MOE_TC_PREFILL_SB;
-constexpr int DC_BN = MOE_TC_DECODE_BN, DC_SA = MOE_TC_DECODE_SA, DC_SB = MOE_TC_DECODE_SB;
+constexpr int PF_BN = MOE_TC_PREFILL_BN, PF_ST = MOE_TC_PREFILL_STAGES;
+constexpr int DC_BN = MOE_TC_DECODE_BN, DC_ST = MOE_TC_DECODE_STAGES;
 
 // few rows per expert (decode): one SM per tile, narrow token tiles and a deep
 // ring so that enough weight bytes are in flight; otherwise SM pairs with
@@ -1113,17 +1036,17 @@ bool pair_ok(const Job &j) {
 
 moe_status run_up(const Job &j) {
   if (tc_path(j.c, j.x_dt, j.w->w_dt))
-    return decode_variant(j) ? tc_up<1, DC_BN, DC_SA, DC_SB>(j)
-           : pair_ok(j)      ? tc_up<2, PF_BN, PF_SA, PF_SB>(j)
-                             : tc_up<1, 256, 6, 3>(j);
+    return decode_variant(j) ? tc_up<1, DC_BN, 32, DC_ST>(j)
+           : pair_ok(j)      ? tc_up<2, PF_BN, 32, PF_ST>(j)
+                             : tc_up<1, 256, 32, 4>(j);
   return j.x_dt == MOE_BF16 ? simt_up_x<bf16>(j) : simt_up_x<float>(j);
 }
 
 moe_status run_down(const Job &j) {
   if (tc_path(j.c, j.x_dt, j.w->w_dt))
-    return decode_variant(j) ? tc_down<1, DC_BN, DC_SA, DC_SB>(j)
-           : pair_ok(j)      ? tc_down<2, PF_BN, PF_SA, PF_SB>(j)
-                             : tc_down<1, 256, 6, 3>(j);
+    return decode_variant(j) ? tc_down<1, DC_BN, 32, DC_ST>(j)
+           : pair_ok(j)      ? tc_down<2, PF_BN, 32, PF_ST>(j)
+                             : tc_down<1, 256, 32, 4>(j);
   return simt_down_w(j);
 }
 

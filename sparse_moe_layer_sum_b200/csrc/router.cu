@@ -263,6 +263,7 @@ namespace tcr {
 
 constexpr int BK = 64, BM = 128, THREADS = 192, EPI_WARPS = 4;
 constexpr int A_BYTES = BM * BK * 2;  // one of the three weight terms
+constexpr int NCHUNK = 3;             // TMEM buffers for per-k-block partial sums
 
 struct Params {
   int T, E, nsplit, kb_per_split, KB, mt, nt;
@@ -276,9 +277,11 @@ struct Layout {
   static constexpr int B_BYTES = BN * BK * 2;
   static constexpr int STAGE_BYTES = 3 * A_BYTES + B_BYTES;
   static constexpr int BAR_OFF = STAGES * STAGE_BYTES;
-  static constexpr int MISC_OFF = BAR_OFF + (2 * STAGES + 5) * 8;
+  // full, empty, chunk_full, chunk_empty, drain
+  static constexpr int MISC_OFF = BAR_OFF + (2 * STAGES + 2 * NCHUNK + 1) * 8;
   static constexpr size_t SMEM = 1024 + MISC_OFF + 16 + 4 * STAGES;
-  static constexpr uint32_t TMEM_COLS = 2 * BN;
+  static constexpr uint32_t TMEM_COLS = 512;
+  static_assert(NCHUNK * BN <= 512, "TMEM chunk buffers");
 };
 
 __device__ __forceinline__ void drain_wait(uint64_t *bar, uint32_t parity, int64_t limit_ns) {
@@ -287,6 +290,12 @@ __device__ __forceinline__ void drain_wait(uint64_t *bar, uint32_t parity, int64
     if ((int64_t)(sm100::globaltimer_ns() - t0) > limit_ns) break;
 }
 
+// Tensor cores add in fp32 with a rounding that drifts with the number of
+// additions into one accumulator, so the MMAs of each k-block (x times the
+// three weight terms, 64 columns of dim) go into a fresh TMEM buffer and the
+// epilogue warps add that partial into fp32 running sums in registers:
+// every accumulation chain stays a dozen additions long.
+//
 // tile -> (split, token tile, expert tile); expert tiles innermost so the
 // CTAs sharing an x tile run together
 template <int BN, int STAGES>
@@ -300,9 +309,9 @@ __global__ void __launch_bounds__(THREADS, 1)
                                             ~static_cast<uintptr_t>(1023));
   uint64_t *full = reinterpret_cast<uint64_t *>(sm + L::BAR_OFF);
   uint64_t *empty = full + STAGES;
-  uint64_t *accf = empty + STAGES;
-  uint64_t *acce = accf + 2;
-  uint64_t *drain = acce + 2;
+  uint64_t *cfull = empty + STAGES;
+  uint64_t *cempty = cfull + NCHUNK;
+  uint64_t *drain = cempty + NCHUNK;
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + L::MISC_OFF);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + L::MISC_OFF + 4);
   volatile int *pending = reinterpret_cast<volatile int *>(sm + L::MISC_OFF + 16);
@@ -313,10 +322,10 @@ __global__ void __launch_bounds__(THREADS, 1)
       mbar_init(empty + s, 1);
       pending[s] = -1;
     }
-    mbar_init(accf, 1);
-    mbar_init(accf + 1, 1);
-    mbar_init(acce, EPI_WARPS);
-    mbar_init(acce + 1, EPI_WARPS);
+    for (int c = 0; c < NCHUNK; ++c) {
+      mbar_init(cfull + c, 1);
+      mbar_init(cempty + c, EPI_WARPS);
+    }
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -347,7 +356,7 @@ __global__ void __launch_bounds__(THREADS, 1)
 
   if (warp == 0) {
     if (lane == 0) {
-      const uint64_t pol_w = policy_evict_first();
+      const uint64_t pol_w = policy_evict_last();  // the weight terms are re-read per token tile
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
@@ -379,26 +388,22 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      int stage = 0, acc = 0;
-      uint32_t phase = 0, acc_phase = 0;
+      int stage = 0, c = 0;
+      uint32_t phase = 0, cphase = 0;
       bool ok = true;
       for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
         int split, n0, m0, kb0, kb1, nvalid;
         decode(tile, split, n0, m0, kb0, kb1, nvalid);
-        if (!wait_bounded(acce + acc, acc_phase ^ 1u, abort_flag, p.timeout_ns, p.status)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
         const uint32_t idesc = idesc_bf16_f32(BM, (nvalid + 15) & ~15);
         for (int kb = kb0; kb < kb1; ++kb) {
-          if (!wait_bounded(full + stage, phase, abort_flag, p.timeout_ns, p.status)) {
+          if (!wait_bounded(cempty + c, cphase ^ 1u, abort_flag, p.timeout_ns, p.status) ||
+              !wait_bounded(full + stage, phase, abort_flag, p.timeout_ns, p.status)) {
             ok = false;
             break;
           }
           pending[stage] = -1;
           tc_fence_after();
+          const uint32_t d_tmem = tmem_base + (uint32_t)(c * BN);
           const uint32_t a_addr = smem_u32(sm + stage * L::STAGE_BYTES);
           const uint32_t b_addr = a_addr + 3 * A_BYTES;
 #pragma unroll
@@ -406,18 +411,18 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
             for (int t3 = 0; t3 < 3; ++t3)
               mma_bf16(d_tmem, sdesc_sw128(a_addr + t3 * A_BYTES + kk * 32),
-                       sdesc_sw128(b_addr + kk * 32), idesc,
-                       (kb > kb0 || kk > 0 || t3 > 0) ? 1u : 0u);
+                       sdesc_sw128(b_addr + kk * 32), idesc, (kk > 0 || t3 > 0) ? 1u : 0u);
           mma_commit(empty + stage);
+          mma_commit(cfull + c);
           if (++stage == STAGES) {
             stage = 0;
             phase ^= 1u;
           }
+          if (++c == NCHUNK) {
+            c = 0;
+            cphase ^= 1u;
+          }
         }
-        if (!ok) break;
-        mma_commit(accf + acc);
-        acc ^= 1;
-        if (acc == 0) acc_phase ^= 1u;
       }
       if (!ok) {
         mma_commit(drain);
@@ -425,30 +430,49 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
     }
   } else {
+    // epilogue: running fp32 sums of the per-k-block partials; lane = expert,
+    // the 128 columns (tokens) of the tile in four groups of 32
     const int q = warp & 3;
-    int acc = 0;
-    uint32_t acc_phase = 0;
+    int c = 0;
+    uint32_t cphase = 0;
     for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
       int split, n0, m0, kb0, kb1, nvalid;
       decode(tile, split, n0, m0, kb0, kb1, nvalid);
-      if (!wait_bounded(accf + acc, acc_phase, abort_flag, p.timeout_ns, p.status)) break;
-      tc_fence_after();
-      const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
+      float run[BN];
+#pragma unroll
+      for (int j = 0; j < BN; ++j) run[j] = 0.f;
+      bool ok = true;
+      for (int kb = kb0; kb < kb1; ++kb) {
+        if (!wait_bounded(cfull + c, cphase, abort_flag, p.timeout_ns, p.status)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(c * BN);
+#pragma unroll
+        for (int g = 0; g < BN / 32; ++g) {
+          if (g * 32 < nvalid) {
+            uint32_t v[32];
+            tmem_ld_32x32b_x32(tb + (uint32_t)(g * 32), v);
+            tmem_wait_ld();
+#pragma unroll
+            for (int j = 0; j < 32; ++j) run[g * 32 + j] += __uint_as_float(v[j]);
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(cempty + c);
+        if (++c == NCHUNK) {
+          c = 0;
+          cphase ^= 1u;
+        }
+      }
+      if (!ok) break;
       float *out = p.z_part + (size_t)split * p.T * p.E;
       const int e = m0 + q * 32 + lane;
-      for (int c0 = 0; c0 < nvalid; c0 += 32) {
-        uint32_t v[32];
-        tmem_ld_32x32b_x32(tb + (uint32_t)c0, v);
-        tmem_wait_ld();
 #pragma unroll
-        for (int j = 0; j < 32; ++j)
-          if (c0 + j < nvalid) out[(size_t)(n0 + c0 + j) * p.E + e] = __uint_as_float(v[j]);
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(acce + acc);
-      acc ^= 1;
-      if (acc == 0) acc_phase ^= 1u;
+      for (int j = 0; j < BN; ++j)
+        if (j < nvalid) out[(size_t)(n0 + j) * p.E + e] = run[j];
     }
   }
   __syncthreads();

@@ -246,15 +246,18 @@ class MoEBlock:
         self.status = torch.zeros(1, dtype=i32, device=dev)
 
     # kernels one forward launches: router 3 (bf16 x on the tensor-core path:
-    # weight split, scores, selection) or 2, dispatch 3, experts 4 (two tile
-    # tables, two GEMMs), then combine 1 (ordered) or nothing (scatter; y is
-    # zeroed by a memset node)
+    # weight split, scores, selection) or 2, dispatch 3, experts 5 on the
+    # tensor-core path (two tile tables, row gather, two GEMMs) or 4, then
+    # combine 1 (ordered) or nothing (scatter; y is zeroed by a memset node)
     @property
     def launches_per_forward(self) -> int:
         sh = self.shape
         tc_router = (self.x_dtype == torch.bfloat16 and sh.n_routed % 128 == 0
                      and sh.dim % 64 == 0 and self.T >= 32)
-        return (3 if tc_router else 2) + 3 + 4 + (1 if self.combine_mode == "ordered" else 0)
+        tc_experts = (self.x_dtype == torch.bfloat16 and self.p.w1.dtype == torch.bfloat16
+                      and sh.dim % 128 == 0 and sh.inter % 128 == 0)
+        return ((3 if tc_router else 2) + 3 + (5 if tc_experts else 4)
+                + (1 if self.combine_mode == "ordered" else 0))
 
     def _router(self, x, cfgp, s):
         p = self.p
