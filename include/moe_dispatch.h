@@ -39,6 +39,30 @@ moe_status moe_dispatch_build(const moe_cfg *cfg, int64_t T, const int32_t *indi
                               int32_t *slot_of, void *ws, size_t ws_bytes,
                               int32_t *dev_status, moe_stream_t stream);
 
+/*
+ * moe_dispatch_build without a workspace argument, for callers that hold
+ * only their input and output buffers and have no way to obtain device
+ * memory for scratch space -- for instance a host framework that hands a
+ * kernel its tensors but no allocator, or a process whose device memory is
+ * entirely owned by another allocator.  (The pages have no counterpart; this
+ * is a convenience of this library.)
+ *
+ * The scratch space is a fixed array of 1 MiB inside this library, which
+ * every GPU that loads the library holds until the process exits.  It covers
+ * ceil(T / 64) * n_routed <= 262144 (for example T up to 65536 tokens with
+ * 256 experts); larger calls return MOE_ERR_WORKSPACE and launch nothing.
+ * The first call on a device looks up the array's device address with that
+ * device current (and caches it), so make that first call before any stream
+ * capture.  This entry point allocates and frees no memory.  All calls share
+ * the one array: calls that may overlap on the GPU (other streams, other
+ * threads) race on it and must be serialised by the caller.  Outputs,
+ * limits and errors are those of moe_dispatch_build.
+ */
+moe_status moe_dispatch_build_noalloc(const moe_cfg *cfg, int64_t T, const int32_t *indices,
+                                      int32_t *counts, int32_t *offsets, int32_t *sorted_token,
+                                      int32_t *slot_of, int32_t *dev_status,
+                                      moe_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -48,6 +48,8 @@ SIGNATURES = {
     ("moe_dispatch", "moe_dispatch_workspace_size"): (_sz, [_cfgp, _i64]),
     ("moe_dispatch", "moe_dispatch_build"): (
         _i32, [_cfgp, _i64, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp, _vp]),
+    ("moe_dispatch", "moe_dispatch_build_noalloc"): (
+        _i32, [_cfgp, _i64, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
     ("moe_experts", "moe_experts_workspace_size"): (_sz, [_cfgp, _i64, _i32, _i32]),
     ("moe_experts", "moe_experts_forward"): (
         _i32, [_cfgp, _i64, _vp, _i32, ctypes.POINTER(MoEExpertWeights), _vp, _vp, _vp, _vp,

@@ -14,6 +14,8 @@
 //                       time; lanes holding the same expert rank themselves
 //                       with __match_any_sync, so the order inside an expert
 //                       is the pair order (token ascending) -- deterministic.
+#include <mutex>
+
 #include "common.cuh"
 #include "moe_dispatch.h"
 
@@ -123,6 +125,34 @@ __global__ void __launch_bounds__(32) dispatch_scatter(const int32_t *__restrict
   }
 }
 
+// ------------------------------------------------- no-allocation variant
+//
+// Scratch for moe_dispatch_build_noalloc: the per-chunk histograms live in
+// this file-scope device array instead of a caller-provided workspace.  Every
+// GPU that loads the library holds it until the process exits.
+constexpr int64_t NOALLOC_SCRATCH_INTS = (int64_t)1 << 18;  // 1 MiB
+__device__ __align__(256) int32_t g_noalloc_scratch[NOALLOC_SCRATCH_INTS];
+
+constexpr int MAX_DEVICES = 64;
+std::mutex g_noalloc_mu;
+int32_t *g_noalloc_ptr[MAX_DEVICES] = {};
+
+// Device address of the scratch array on the current device.  In host code the
+// array's name only stands for a host-side symbol, so the address is looked up
+// once per device (with that device current) and cached.
+moe_status noalloc_scratch(int32_t **out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= MAX_DEVICES) return MOE_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void *ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || !ptr) return MOE_ERR_CUDA;
+    g_noalloc_ptr[dev] = static_cast<int32_t *>(ptr);
+  }
+  *out = g_noalloc_ptr[dev];
+  return MOE_OK;
+}
+
 }  // namespace
 }  // namespace moe
 
@@ -164,4 +194,22 @@ MOE_EXPORT moe_status moe_dispatch_build(const moe_cfg *cfg, int64_t T, const in
     if ((st = launch_status()) != MOE_OK) return st;
   }
   return MOE_OK;
+}
+
+MOE_EXPORT moe_status moe_dispatch_build_noalloc(const moe_cfg *cfg, int64_t T,
+                                                 const int32_t *indices, int32_t *counts,
+                                                 int32_t *offsets, int32_t *sorted_token,
+                                                 int32_t *slot_of, int32_t *dev_status,
+                                                 moe_stream_t stream) {
+  moe_status st = check_cfg(cfg);
+  if (st != MOE_OK) return st;
+  if (T < 0) return MOE_ERR_INVALID;
+  const size_t need = moe_dispatch_workspace_size(cfg, T);
+  if (need > (size_t)NOALLOC_SCRATCH_INTS * sizeof(int32_t)) return MOE_ERR_WORKSPACE;
+  int32_t *scratch = nullptr;
+  if ((st = noalloc_scratch(&scratch)) != MOE_OK) return st;
+  // the histogram pass writes every scratch entry the later passes read, so
+  // nothing has to be cleared between calls
+  return moe_dispatch_build(cfg, T, indices, counts, offsets, sorted_token, slot_of, scratch,
+                            (size_t)NOALLOC_SCRATCH_INTS * sizeof(int32_t), dev_status, stream);
 }
