@@ -162,7 +162,10 @@ namespace tc {
 constexpr int BK = 64;                 // K elements per ring stage (128 bytes bf16)
 constexpr int BM = 128;                // MMA M: weight rows per tile
 constexpr int A_BYTES = BM * BK * 2;   // 16 KB
-constexpr int THREADS = 192;           // warp 0 TMA, warp 1 MMA, warps 2-5 epilogue
+// warp 0 issues TMA loads, warp 1 MMAs, warps 2-5 run the epilogue, warps 6-7
+// convert e4m3 weight tiles to bf16 (idle with bf16 weights)
+constexpr int THREADS = 256;
+constexpr int CONV_WARPS = 2;
 constexpr int EPI_WARPS = 4;
 constexpr int XB_STRIDE = 17;          // exchange buffer row stride (floats)
 
@@ -184,19 +187,26 @@ struct Params {
   const float *weights;    // [T, k]
   int k;
   float *y;                // [T, D], zeroed before the launch
+  // e4m3 weights: fp32 scales of 128 x 128 blocks, [G, rows/128, cols/128]
+  const float *sA0, *sA1;  // GEMM1: w1, w3; second GEMM: w2 (sA1 unused)
 };
 
 // CG = CTA group: 1 = one SM per tile; 2 = an SM pair per tile (cta_group::2),
 // where each CTA holds 128 weight rows and half of the token tile.
-template <int MODE, int CG, int BN_MAX, int BOXN, int STAGES>
+// F8: the weights arrive as e4m3 tiles (A8, 64 bytes per row) that the
+// converter warps expand into the bf16 tile the MMA reads.
+template <int MODE, int CG, int BN_MAX, int BOXN, int STAGES, bool F8>
 struct Layout {
   static constexpr int B_ROWS = BN_MAX / CG;  // token rows one CTA holds per stage
   static constexpr int B_BYTES = B_ROWS * BK * 2;
-  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int A8_BYTES = F8 ? BM * BK : 0;
+  static constexpr int A8_OFF = A_BYTES + B_BYTES;  // within a stage
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + A8_BYTES;
   static constexpr int BAR_OFF = STAGES * STAGE_BYTES;
-  static constexpr int NBARS = 2 * STAGES + 5;  // full, empty, acc_full x2, acc_empty x2, drain
+  // full, empty, [a8_full, converted], acc_full x2, acc_empty x2, drain
+  static constexpr int NBARS = (F8 ? 4 : 2) * STAGES + 5;
   static constexpr int MISC_OFF = BAR_OFF + NBARS * 8;
-  static constexpr int MISC_BYTES = 16 + 4 * STAGES;
+  static constexpr int MISC_BYTES = 16 + 8 * STAGES;
   static constexpr int XBUF_OFF = (MISC_OFF + MISC_BYTES + 127) / 128 * 128;
   // GEMM1: SwiGLU exchange buffers; MODE 3: the tile's (token, gate) list
   static constexpr int XBUF_BYTES = MODE == 1 ? 2 * 2 * 32 * XB_STRIDE * 4 : MODE == 3 ? BN_MAX * 8 : 0;
@@ -230,23 +240,26 @@ __device__ __forceinline__ void sleep_ns(int64_t ns) {
   }
 }
 
-template <int MODE, int CG, int BN_MAX, int BOXN, int STAGES>
+template <int MODE, int CG, int BN_MAX, int BOXN, int STAGES, bool F8>
 __global__ void __launch_bounds__(THREADS, 1)
     tc_expert_gemm(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA1,
                    const __grid_constant__ CUtensorMap tmB, const Params p) {
-  using L = Layout<MODE, CG, BN_MAX, BOXN, STAGES>;
+  using L = Layout<MODE, CG, BN_MAX, BOXN, STAGES, F8>;
   using namespace sm100;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                             ~static_cast<uintptr_t>(1023));
   uint64_t *full = reinterpret_cast<uint64_t *>(sm + L::BAR_OFF);
   uint64_t *empty = full + STAGES;
-  uint64_t *accf = empty + STAGES;
+  uint64_t *a8full = empty + STAGES;                 // F8 only
+  uint64_t *conv = a8full + (F8 ? STAGES : 0);       // F8 only
+  uint64_t *accf = conv + (F8 ? STAGES : 0);
   uint64_t *acce = accf + 2;
   uint64_t *drain = acce + 2;
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + L::MISC_OFF);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + L::MISC_OFF + 4);
   volatile int *pending = reinterpret_cast<volatile int *>(sm + L::MISC_OFF + 16);
+  volatile int *pend8 = pending + STAGES;  // e4m3 loads in flight (F8)
   float *xbuf = reinterpret_cast<float *>(sm + L::XBUF_OFF);
   int32_t *s_tstart = reinterpret_cast<int32_t *>(sm + L::TAB_OFF);
   int32_t *s_tbase = s_tstart + p.G + 1;
@@ -264,6 +277,11 @@ __global__ void __launch_bounds__(THREADS, 1)
       mbar_init(full + s, 1);
       mbar_init(empty + s, 1);
       pending[s] = -1;
+      pend8[s] = -1;
+      if (F8) {
+        mbar_init(a8full + s, 1);
+        mbar_init(conv + s, CONV_WARPS * CG);
+      }
     }
     mbar_init(accf + 0, 1);
     mbar_init(accf + 1, 1);
@@ -311,7 +329,9 @@ __global__ void __launch_bounds__(THREADS, 1)
         const int arow = MODE == 1 ? t.g * p.I + t.ft * L::FEAT + (int)rank * 64
                                    : t.g * p.D + t.ft * L::FEAT + (int)rank * BM;
         const int nbox = (brows + BOXN - 1) / BOXN;
-        const uint32_t bytes = (uint32_t)(A_BYTES + nbox * BOXN * BK * 2);
+        // with e4m3 weights the full barrier counts only the token rows; the
+        // weight tile arrives on this CTA's own a8_full barrier
+        const uint32_t bytes = (uint32_t)((F8 ? 0 : A_BYTES) + nbox * BOXN * BK * 2);
         const int k0 = k_rotation(t, p.KB);
         for (int i = 0; i < p.KB; ++i) {
           const int kb = k0 + i < p.KB ? k0 + i : k0 + i - p.KB;
@@ -324,7 +344,26 @@ __global__ void __launch_bounds__(THREADS, 1)
           pending[stage] = (int)phase;
           uint8_t *a_dst = sm + stage * L::STAGE_BYTES;
           uint8_t *b_dst = a_dst + A_BYTES;
-          if (CG == 2) {
+          if (F8) {
+            uint8_t *a8 = a_dst + L::A8_OFF;
+            mbar_arrive_expect_tx(a8full + stage, L::A8_BYTES);
+            pend8[stage] = (int)phase;
+            if (MODE == 1) {
+              tma_load_2d_hint(&tmA0, a8, a8full + stage, kb * BK, arow, pol_w);
+              tma_load_2d_hint(&tmA1, a8 + L::A8_BYTES / 2, a8full + stage, kb * BK, arow, pol_w);
+            } else {
+              tma_load_2d_hint(&tmA0, a8, a8full + stage, kb * BK, arow, pol_w);
+            }
+            if (CG == 2) {
+              const uint32_t fb = mapa_shared(smem_u32(full + stage), 0);
+              for (int i = 0; i < nbox; ++i)
+                tma_load_2d_pair(&tmB, b_dst + i * BOXN * BK * 2, fb, kb * BK, b0 + i * BOXN, pol_x);
+            } else {
+              for (int i = 0; i < nbox; ++i)
+                tma_load_2d_hint(&tmB, b_dst + i * BOXN * BK * 2, full + stage, kb * BK,
+                                 b0 + i * BOXN, pol_x);
+            }
+          } else if (CG == 2) {
             const uint32_t fb = mapa_shared(smem_u32(full + stage), 0);
             if (MODE == 1) {
               tma_load_2d_pair(&tmA0, a_dst, fb, kb * BK, arow, pol_w);
@@ -369,7 +408,9 @@ __global__ void __launch_bounds__(THREADS, 1)
         const int nmma = (t.nvalid + 15) & ~15;
         const uint32_t idesc = idesc_bf16_f32(BM * CG, nmma);
         for (int kb = 0; kb < p.KB; ++kb) {
-          if (!wait_bounded(full + stage, phase, abort_flag, p.timeout_ns, p.status)) {
+          if (!wait_bounded(full + stage, phase, abort_flag, p.timeout_ns, p.status) ||
+              (F8 && !wait_bounded<CG == 2>(conv + stage, phase, abort_flag, p.timeout_ns,
+                                            p.status))) {
             ok = false;
             break;
           }
@@ -410,6 +451,70 @@ __global__ void __launch_bounds__(THREADS, 1)
         else
           mma_commit(drain);
         drain_wait(drain, 0, p.timeout_ns);
+      }
+    }
+  } else if (warp >= 2 + EPI_WARPS) {
+    if (F8) {
+      // ----------------------------------------------- e4m3 -> bf16 converter
+      // A8 row r (64 codes) becomes A row r (64 bf16) in the 128-byte swizzled
+      // layout: 16-byte chunk c of row r lands at chunk c ^ (r % 8).  Each code
+      // is multiplied by the fp32 scale of its 128 x 128 block and rounded
+      // once to bf16.
+      const int ct = threadIdx.x - 32 * (2 + EPI_WARPS);  // 0 .. 63
+      const int rows_w = MODE == 1 ? p.I : p.D;            // rows of one expert's matrix
+      const int cols_w = MODE == 1 ? p.D : p.I;
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int tile = unit; ok && tile < total; tile += nunits) {
+        const Tile t = decode_tile(tile, s_tstart, s_tbase, s_off, p.G, p.E, p.T, p.rows_routed);
+        const int r0 = MODE == 1 ? t.ft * L::FEAT + (int)rank * 64 : t.ft * L::FEAT + (int)rank * BM;
+        const size_t srow = ((size_t)t.g * (rows_w / 128) + r0 / 128) * (cols_w / 128);
+        const int k0 = k_rotation(t, p.KB);
+        for (int i = 0; i < p.KB; ++i) {
+          const int kb = k0 + i < p.KB ? k0 + i : k0 + i - p.KB;
+          if (!wait_bounded(a8full + stage, phase, abort_flag, p.timeout_ns, p.status)) {
+            ok = false;
+            break;
+          }
+          pend8[stage] = -1;
+          const float sc0 = p.sA0[srow + kb / 2];
+          const float sc1 = MODE == 1 ? p.sA1[srow + kb / 2] : sc0;
+          const uint8_t *a8 = sm + stage * L::STAGE_BYTES + L::A8_OFF;
+          uint8_t *a16 = sm + stage * L::STAGE_BYTES;
+#pragma unroll 4
+          for (int it = 0; it < BM * 8 / (32 * CONV_WARPS); ++it) {
+            const int idx = ct + it * 32 * CONV_WARPS;
+            const int r = idx >> 3, c = idx & 7;
+            const float sc = (MODE == 1 && r >= 64) ? sc1 : sc0;
+            const uint2 q = *reinterpret_cast<const uint2 *>(a8 + r * 64 + c * 8);
+            uint32_t w[4];
+            const uint32_t qq[2] = {q.x, q.y};
+#pragma unroll
+            for (int h = 0; h < 4; ++h) {
+              const __nv_fp8x2_storage_t pair =
+                  static_cast<__nv_fp8x2_storage_t>((qq[h >> 1] >> ((h & 1) * 16)) & 0xffffu);
+              const __half2_raw hr = __nv_cvt_fp8x2_to_halfraw2(pair, __NV_E4M3);
+              const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&hr));
+              const __nv_bfloat162 b = __floats2bfloat162_rn(f.x * sc, f.y * sc);
+              w[h] = *reinterpret_cast<const uint32_t *>(&b);
+            }
+            *reinterpret_cast<uint4 *>(a16 + r * 128 + ((c ^ (r & 7)) << 4)) =
+                make_uint4(w[0], w[1], w[2], w[3]);
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            if (CG == 2)
+              mbar_arrive_cluster(mapa_shared(smem_u32(conv + stage), 0));  // the leader's barrier
+            else
+              mbar_arrive(conv + stage);
+          }
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
       }
     }
   } else {
@@ -523,6 +628,9 @@ __global__ void __launch_bounds__(THREADS, 1)
     // a stalled pipeline stopped early: let copies already issued land.  The
     // leader's full barriers count both CTAs' copies; the other CTA of a pair
     // cannot wait on them and just allows its copies time to land.
+    if (F8)  // the e4m3 tiles land on this CTA's own barriers
+      for (int s = 0; s < STAGES; ++s)
+        if (pend8[s] >= 0) drain_wait(a8full + s, (uint32_t)pend8[s], p.timeout_ns);
     if (leader) {
       for (int s = 0; s < STAGES; ++s)
         if (pending[s] >= 0) drain_wait(full + s, (uint32_t)pending[s], p.timeout_ns);
@@ -717,9 +825,11 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 }
 
 // 2-D row-major [rows, cols] matrix of `elem` bytes, box of box_rows rows x
-// box_cols columns, 128-byte swizzle (box_cols * elem must be 128).
+// box_cols columns, 128-byte swizzle (box_cols * elem must be 128) unless
+// `plain` (rows of the box stored back to back, as the e4m3 tiles are).
 bool make_tmap(CUtensorMap *m, const void *base, CUtensorMapDataType dt, size_t elem,
-               uint64_t rows, uint64_t cols, uint32_t box_rows, uint32_t box_cols) {
+               uint64_t rows, uint64_t cols, uint32_t box_rows, uint32_t box_cols,
+               bool plain = false) {
   auto fn = encode_fn();
   if (!fn) return false;
   cuuint64_t gdim[2] = {cols, rows};
@@ -727,7 +837,8 @@ bool make_tmap(CUtensorMap *m, const void *base, CUtensorMapDataType dt, size_t 
   cuuint32_t box[2] = {box_cols, box_rows};
   cuuint32_t estride[2] = {1, 1};
   return fn(m, dt, 2, const_cast<void *>(base), gdim, gstride, box, estride,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_INTERLEAVE_NONE,
+            plain ? CU_TENSOR_MAP_SWIZZLE_NONE : CU_TENSOR_MAP_SWIZZLE_128B,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -747,7 +858,8 @@ struct WsLayout {
 constexpr int ROW_PAD = 256;  // spare rows so a TMA box never starts past a buffer
 
 bool tc_path(const moe_cfg *c, moe_dtype x_dt, moe_dtype w_dt) {
-  return x_dt == MOE_BF16 && (w_dt == MOE_BF16) && c->dim % 128 == 0 && c->inter % 128 == 0;
+  return x_dt == MOE_BF16 && (w_dt == MOE_BF16 || w_dt == MOE_E4M3) && c->dim % 128 == 0 &&
+         c->inter % 128 == 0;
 }
 
 WsLayout ws_layout(const moe_cfg *c, int64_t T, moe_dtype x_dt, moe_dtype w_dt) {
@@ -765,11 +877,13 @@ WsLayout ws_layout(const moe_cfg *c, int64_t T, moe_dtype x_dt, moe_dtype w_dt) 
   return l;
 }
 
-template <int MODE, int CG, int BN_MAX, int BOXN, int STAGES>
+template <int MODE, int CG, int BN_MAX, int BOXN, int STAGES, bool F8>
 moe_status launch_tc(const CUtensorMap &a0, const CUtensorMap &a1, const CUtensorMap &b,
                      const tc::Params &p, cudaStream_t s) {
-  using L = tc::Layout<MODE, CG, BN_MAX, BOXN, STAGES>;
-  auto kern = tc::tc_expert_gemm<MODE, CG, BN_MAX, BOXN, STAGES>;
+  using L = tc::Layout<MODE, CG, BN_MAX, BOXN, STAGES, F8>;
+  auto kern = tc::tc_expert_gemm<MODE, CG, BN_MAX, BOXN, STAGES, F8>;
+  const size_t smem_max = 232448;
+  if (L::smem_bytes(p.G, p.E) > smem_max) return MOE_ERR_UNSUPPORTED;
   const size_t smem = L::smem_bytes(p.G, p.E);
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
       cudaSuccess)
@@ -855,10 +969,20 @@ tc::Params tc_params(const Job &j) {
   p.weights = j.weights;
   p.k = j.c->topk;
   p.y = j.y;
+  p.sA0 = nullptr;
+  p.sA1 = nullptr;
   return p;
 }
 
-template <int CG, int BN_MAX, int BOXN, int STAGES>
+// Weight tensor map: bf16 tiles in the 128-byte swizzled layout the MMA reads,
+// or e4m3 tiles stored plainly (64 bytes per row) for the converter warps.
+bool weight_tmap(CUtensorMap *m, const void *w, bool f8, uint64_t rows, uint64_t cols,
+                 uint32_t box_rows) {
+  if (f8) return make_tmap(m, w, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, rows, cols, box_rows, 64, true);
+  return make_tmap(m, w, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, rows, cols, box_rows, 64);
+}
+
+template <int CG, int BN_MAX, int BOXN, int STAGES, bool F8>
 moe_status tc_up(const Job &j) {
   const int G = j.G(), D = j.c->dim, I = j.c->inter;
   int32_t *tab = j.tab();
@@ -877,8 +1001,8 @@ moe_status tc_up(const Job &j) {
   if ((st = launch_status()) != MOE_OK) return st;
   CUtensorMap mw1, mw3, mx;
   const CUtensorMapDataType BF = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
-  if (!make_tmap(&mw1, j.w->w1, BF, 2, (uint64_t)G * I, D, 64, 64) ||
-      !make_tmap(&mw3, j.w->w3, BF, 2, (uint64_t)G * I, D, 64, 64) ||
+  if (!weight_tmap(&mw1, j.w->w1, F8, (uint64_t)G * I, D, 64) ||
+      !weight_tmap(&mw3, j.w->w3, F8, (uint64_t)G * I, D, 64) ||
       !make_tmap(&mx, xperm, BF, 2, (uint64_t)j.l.rows_pad, D, BOXN, 64))
     return MOE_ERR_CUDA;
   tc::Params p = tc_params(j);
@@ -886,13 +1010,15 @@ moe_status tc_up(const Job &j) {
   p.tile_base = t1.tile_base;
   p.KB = D / tc::BK;
   p.out = h;
+  p.sA0 = j.w->s1;
+  p.sA1 = j.w->s3;
   prof(1, j.s);
-  st = launch_tc<1, CG, BN_MAX, BOXN, STAGES>(mw1, mw3, mx, p, j.s);
+  st = launch_tc<1, CG, BN_MAX, BOXN, STAGES, F8>(mw1, mw3, mx, p, j.s);
   prof(2, j.s);
   return st;
 }
 
-template <int CG, int BN_MAX, int BOXN, int STAGES>
+template <int CG, int BN_MAX, int BOXN, int STAGES, bool F8>
 moe_status tc_down(const Job &j) {
   const int G = j.G(), D = j.c->dim, I = j.c->inter;
   int32_t *tab = j.tab();
@@ -904,7 +1030,7 @@ moe_status tc_down(const Job &j) {
   bf16 *h = reinterpret_cast<bf16 *>(j.ws + j.l.h);
   CUtensorMap mw2, mh;
   const CUtensorMapDataType BF = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
-  if (!make_tmap(&mw2, j.w->w2, BF, 2, (uint64_t)G * D, I, tc::BM, 64) ||
+  if (!weight_tmap(&mw2, j.w->w2, F8, (uint64_t)G * D, I, tc::BM) ||
       !make_tmap(&mh, h, BF, 2, (uint64_t)j.l.rows_pad, I, BOXN, 64))
     return MOE_ERR_CUDA;
   tc::Params p = tc_params(j);
@@ -912,11 +1038,13 @@ moe_status tc_down(const Job &j) {
   p.tile_base = t2.tile_base;
   p.KB = I / tc::BK;
   p.out = j.out_perm;
+  p.sA0 = j.w->s2;
+  p.sA1 = j.w->s2;
   prof(3, j.s);
   if (j.y)
-    st = launch_tc<3, CG, BN_MAX, BOXN, STAGES>(mw2, mw2, mh, p, j.s);
+    st = launch_tc<3, CG, BN_MAX, BOXN, STAGES, F8>(mw2, mw2, mh, p, j.s);
   else
-    st = launch_tc<2, CG, BN_MAX, BOXN, STAGES>(mw2, mw2, mh, p, j.s);
+    st = launch_tc<2, CG, BN_MAX, BOXN, STAGES, F8>(mw2, mw2, mh, p, j.s);
   prof(4, j.s);
   return st;
 }
@@ -1034,19 +1162,32 @@ bool pair_ok(const Job &j) {
   return MOE_TC_PREFILL_CG == 2 && j.c->inter % 128 == 0 && j.c->dim % 256 == 0;
 }
 
+// e4m3 weights add an 8 KB code tile per stage (stage = 16 KB bf16 weights +
+// tokens + 8 KB codes); the ring depths shrink to fit shared memory, and half
+// as many weight bytes need to be in flight.
+template <bool F8>
+moe_status run_up_t(const Job &j) {
+  if (decode_variant(j)) return tc_up<1, DC_BN, 32, F8 ? 7 : DC_ST, F8>(j);
+  if (pair_ok(j)) return tc_up<2, PF_BN, 32, F8 ? 5 : PF_ST, F8>(j);
+  return tc_up<1, 256, 32, F8 ? 3 : 4, F8>(j);
+}
+
+template <bool F8>
+moe_status run_down_t(const Job &j) {
+  if (decode_variant(j)) return tc_down<1, DC_BN, 32, F8 ? 7 : DC_ST, F8>(j);
+  if (pair_ok(j)) return tc_down<2, PF_BN, 32, F8 ? 5 : PF_ST, F8>(j);
+  return tc_down<1, 256, 32, F8 ? 3 : 4, F8>(j);
+}
+
 moe_status run_up(const Job &j) {
   if (tc_path(j.c, j.x_dt, j.w->w_dt))
-    return decode_variant(j) ? tc_up<1, DC_BN, 32, DC_ST>(j)
-           : pair_ok(j)      ? tc_up<2, PF_BN, 32, PF_ST>(j)
-                             : tc_up<1, 256, 32, 4>(j);
+    return j.w->w_dt == MOE_E4M3 ? run_up_t<true>(j) : run_up_t<false>(j);
   return j.x_dt == MOE_BF16 ? simt_up_x<bf16>(j) : simt_up_x<float>(j);
 }
 
 moe_status run_down(const Job &j) {
   if (tc_path(j.c, j.x_dt, j.w->w_dt))
-    return decode_variant(j) ? tc_down<1, DC_BN, 32, DC_ST>(j)
-           : pair_ok(j)      ? tc_down<2, PF_BN, 32, PF_ST>(j)
-                             : tc_down<1, 256, 32, 4>(j);
+    return j.w->w_dt == MOE_E4M3 ? run_down_t<true>(j) : run_down_t<false>(j);
   return simt_down_w(j);
 }
 

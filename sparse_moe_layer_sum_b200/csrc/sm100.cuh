@@ -62,18 +62,40 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
   return ok != 0;
 }
 
+// try_wait with acquire at cluster scope: for phases completed by arrivals
+// from the other CTA of a pair that publish its shared-memory writes.
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t *bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred P1;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 P1, [%1], %2;\n\t"
+      "selp.b32 %0, 1, 0, P1;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Makes this thread's generic-proxy shared-memory writes visible to the async
+// proxy (TMA, tensor cores) before it signals their consumer.
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 // Waits for the phase with the given parity to complete, for at most
 // limit_ns.  Returns false (after raising *abort and recording
 // MOE_ERR_TIMEOUT) when the limit expires, or false at once when another
 // role has already raised *abort.  Every pipeline wait goes through here, so
 // a stalled pipeline ends with an error status instead of a hung GPU.
+template <bool CLUSTER = false>
 __device__ __forceinline__ bool wait_bounded(uint64_t *bar, uint32_t parity,
                                              volatile int *abort, int64_t limit_ns,
                                              int32_t *status) {
-  if (mbar_try_wait(bar, parity)) return true;
+  auto test = [&]() { return CLUSTER ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity); };
+  if (test()) return true;
   const uint64_t t0 = globaltimer_ns();
   for (uint32_t it = 1;; ++it) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (test()) return true;
     if ((it & 31u) == 0) {
       if (*abort) return false;
       if ((int64_t)(globaltimer_ns() - t0) > limit_ns) {

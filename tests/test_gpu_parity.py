@@ -42,6 +42,10 @@ CG1_PREFILL = custom("cg1_prefill", 230, dim=384, n_routed=16, n_groups=4, topk_
                      inter=128, seed=22)
 FP8_SMALL = custom("fp8_small", 260, w_format="e4m3", dim=512, n_routed=16, n_groups=4,
                    topk_groups=2, topk=4, inter=256, seed=17)
+FP8_DECODE = custom("fp8_decode", 40, w_format="e4m3", dim=1024, n_routed=64, n_groups=8,
+                    topk_groups=4, topk=8, inter=256, seed=23)
+FP8_CG1 = custom("fp8_cg1", 230, w_format="e4m3", dim=384, n_routed=16, n_groups=4,
+                 topk_groups=2, topk=4, inter=128, seed=24)
 
 TOL = {"f32": 1e-4, "bf16": 2e-2, "e4m3": 5e-2}
 MEAN_TOL = {"f32": 1e-6, "bf16": 2e-4, "e4m3": 2e-3}
@@ -116,7 +120,8 @@ def test_dispatch_reports_out_of_range():
 
 
 @pytest.mark.parametrize("w", [WORKLOADS["tiny_f32"], TINY_BF16, MID, MID_F32, DECODE_SMALL,
-                               ONE_TOKEN, CG1_PREFILL, FP8_SMALL], ids=lambda w: w.name)
+                               ONE_TOKEN, CG1_PREFILL, FP8_SMALL, FP8_DECODE, FP8_CG1],
+                         ids=lambda w: w.name)
 def test_experts_rows_match_oracle(w):
     """Expert outputs row by row, on a seeded index set (routing held fixed)."""
     x, p = make_block(w)
@@ -156,7 +161,8 @@ def test_experts_rows_match_oracle(w):
 
 @pytest.mark.parametrize("combine", ["scatter", "ordered"])
 @pytest.mark.parametrize("w", [WORKLOADS["tiny_f32"], TINY_BF16, MID, MID_F32, SOFTMAX_NOBIAS,
-                               ONE_GROUP, DECODE_SMALL, ONE_TOKEN, CG1_PREFILL, FP8_SMALL],
+                               ONE_GROUP, DECODE_SMALL, ONE_TOKEN, CG1_PREFILL, FP8_SMALL,
+                               FP8_DECODE, FP8_CG1],
                          ids=lambda w: w.name)
 def test_block_matches_oracle(w, combine):
     x, p = make_block(w)

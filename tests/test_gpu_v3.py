@@ -19,7 +19,8 @@ from sparse_moe_layer_sum_b200.inputs import WORKLOADS, make_block, sample_token
 pytestmark = pytest.mark.gpu
 
 TOL = {"bf16": 2e-2, "e4m3": 5e-2}
-CASES = [("v3_decode_t64", 64), ("v3_prefill_t4096", 12), ("v3_skew_t16384", 12)]
+CASES = [("v3_decode_t64", 64), ("v3_prefill_t4096", 12), ("v3_skew_t16384", 12),
+         ("v3_fp8_t8192", 6)]
 
 
 @pytest.fixture(scope="module", autouse=True)
