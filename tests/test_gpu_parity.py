@@ -48,7 +48,11 @@ FP8_CG1 = custom("fp8_cg1", 230, w_format="e4m3", dim=384, n_routed=16, n_groups
                  topk_groups=2, topk=4, inter=128, seed=24)
 
 TOL = {"f32": 1e-4, "bf16": 2e-2, "e4m3": 5e-2}
-MEAN_TOL = {"f32": 1e-6, "bf16": 2e-4, "e4m3": 2e-3}
+# mean |error| / rms per expert output.  e4m3: the tensor-core path rounds each
+# dequantised weight q*scale to bf16 (relative rms 2^-8/sqrt(12) ~ 1.1e-3 per
+# matmul, twice, plus the h roundings this moves) -- a few 1e-3; a wrong scale
+# block would show errors of tens of percent
+MEAN_TOL = {"f32": 1e-6, "bf16": 2e-4, "e4m3": 1e-2}
 
 
 @pytest.fixture(scope="module", autouse=True)
