@@ -28,6 +28,7 @@
 // CUDA-core path: any other dtype combination (the fp32 configuration) runs
 // on simt_gemm1 / simt_gemm2 in fp32.
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_fp8.h>
 #include <cudaTypedefs.h>
 #include <math.h>
@@ -155,6 +156,21 @@ __global__ void __launch_bounds__(256) gather_rows(const uint4 *__restrict__ x,
   for (int v = lane; v < vec_per_row; v += 32) d[v] = __ldg(s + v);
 }
 
+// The same rows converted to fp16 (the e4m3 path computes in fp16; bf16 values
+// in the fp16 normal range convert exactly).
+__global__ void __launch_bounds__(256) gather_rows_f16(const __nv_bfloat162 *__restrict__ x,
+                                                       const int32_t *__restrict__ sorted_token,
+                                                       __half2 *__restrict__ xp, int rows_routed,
+                                                       int rows_total, int T, int pairs_per_row) {
+  const int row = (int)((blockIdx.x * (size_t)blockDim.x + threadIdx.x) / 32);
+  const int lane = threadIdx.x % 32;
+  if (row >= rows_total) return;
+  const int src = row < rows_routed ? sorted_token[row] : (row - rows_routed) % T;
+  const __nv_bfloat162 *s = x + (size_t)src * pairs_per_row;
+  __half2 *d = xp + (size_t)row * pairs_per_row;
+  for (int v = lane; v < pairs_per_row; v += 32) d[v] = __float22half2_rn(__bfloat1622float2(s[v]));
+}
+
 // ------------------------------------------------------- tensor-core GEMMs
 
 namespace tc {
@@ -162,10 +178,14 @@ namespace tc {
 constexpr int BK = 64;                 // K elements per ring stage (128 bytes bf16)
 constexpr int BM = 128;                // MMA M: weight rows per tile
 constexpr int A_BYTES = BM * BK * 2;   // 16 KB
-// warp 0 issues TMA loads, warp 1 MMAs, warps 2-5 run the epilogue, warps 6-7
-// convert e4m3 weight tiles to bf16 (idle with bf16 weights)
-constexpr int THREADS = 256;
-constexpr int CONV_WARPS = 2;
+// warp 0 issues TMA loads, warp 1 MMAs, warps 2-5 run the epilogue, warps 6-9
+// expand e4m3 weight tiles (idle with bf16 weights)
+constexpr int THREADS = 320;
+constexpr int CONV_WARPS = 4;
+// e4m3 path: the block scales are taken times 2^8 when the codes are expanded
+// (keeping scale and products in the fp16 normal range) and the accumulator is
+// multiplied by 2^-8 in the epilogue -- both exact powers of two
+constexpr float F8_SCALE_UP = 256.0f, F8_SCALE_DOWN = 1.0f / 256.0f;
 constexpr int EPI_WARPS = 4;
 constexpr int XB_STRIDE = 17;          // exchange buffer row stride (floats)
 
@@ -406,7 +426,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN_MAX);
         const int nmma = (t.nvalid + 15) & ~15;
-        const uint32_t idesc = idesc_bf16_f32(BM * CG, nmma);
+        const uint32_t idesc = F8 ? idesc_f16_f32(BM * CG, nmma) : idesc_bf16_f32(BM * CG, nmma);
         for (int kb = 0; kb < p.KB; ++kb) {
           if (!wait_bounded(full + stage, phase, abort_flag, p.timeout_ns, p.status) ||
               (F8 && !wait_bounded<CG == 2>(conv + stage, phase, abort_flag, p.timeout_ns,
@@ -455,12 +475,13 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
   } else if (warp >= 2 + EPI_WARPS) {
     if (F8) {
-      // ----------------------------------------------- e4m3 -> bf16 converter
-      // A8 row r (64 codes) becomes A row r (64 bf16) in the 128-byte swizzled
-      // layout: 16-byte chunk c of row r lands at chunk c ^ (r % 8).  Each code
-      // is multiplied by the fp32 scale of its 128 x 128 block and rounded
-      // once to bf16.
-      const int ct = threadIdx.x - 32 * (2 + EPI_WARPS);  // 0 .. 63
+      // ------------------------------------------------ e4m3 -> f16 converter
+      // A8 row r (64 codes) becomes A row r (64 fp16) in the 128-byte swizzled
+      // layout: 16-byte chunk c of row r lands at chunk c ^ (r % 8).  A code
+      // converts to fp16 exactly; it is then multiplied by 2^8 times the fp32
+      // scale of its 128 x 128 block (rounded once to fp16).  On this path
+      // the token rows and h are fp16 as well.
+      const int ct = threadIdx.x - 32 * (2 + EPI_WARPS);  // 0 .. 32 * CONV_WARPS - 1
       const int rows_w = MODE == 1 ? p.I : p.D;            // rows of one expert's matrix
       const int cols_w = MODE == 1 ? p.D : p.I;
       int stage = 0;
@@ -478,29 +499,22 @@ __global__ void __launch_bounds__(THREADS, 1)
             break;
           }
           pend8[stage] = -1;
-          const float sc0 = p.sA0[srow + kb / 2];
-          const float sc1 = MODE == 1 ? p.sA1[srow + kb / 2] : sc0;
+          const uint32_t s0 = f16x2_splat(p.sA0[srow + kb / 2] * F8_SCALE_UP);
+          const uint32_t s1 = MODE == 1 ? f16x2_splat(p.sA1[srow + kb / 2] * F8_SCALE_UP) : s0;
           const uint8_t *a8 = sm + stage * L::STAGE_BYTES + L::A8_OFF;
           uint8_t *a16 = sm + stage * L::STAGE_BYTES;
 #pragma unroll 4
           for (int it = 0; it < BM * 8 / (32 * CONV_WARPS); ++it) {
             const int idx = ct + it * 32 * CONV_WARPS;
             const int r = idx >> 3, c = idx & 7;
-            const float sc = (MODE == 1 && r >= 64) ? sc1 : sc0;
+            const uint32_t sc = (MODE == 1 && r >= 64) ? s1 : s0;
             const uint2 q = *reinterpret_cast<const uint2 *>(a8 + r * 64 + c * 8);
-            uint32_t w[4];
-            const uint32_t qq[2] = {q.x, q.y};
-#pragma unroll
-            for (int h = 0; h < 4; ++h) {
-              const __nv_fp8x2_storage_t pair =
-                  static_cast<__nv_fp8x2_storage_t>((qq[h >> 1] >> ((h & 1) * 16)) & 0xffffu);
-              const __half2_raw hr = __nv_cvt_fp8x2_to_halfraw2(pair, __NV_E4M3);
-              const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&hr));
-              const __nv_bfloat162 b = __floats2bfloat162_rn(f.x * sc, f.y * sc);
-              w[h] = *reinterpret_cast<const uint32_t *>(&b);
-            }
-            *reinterpret_cast<uint4 *>(a16 + r * 128 + ((c ^ (r & 7)) << 4)) =
-                make_uint4(w[0], w[1], w[2], w[3]);
+            uint4 o;
+            o.x = f16x2_mul(e4m3x2_to_f16x2((uint16_t)(q.x & 0xffffu)), sc);
+            o.y = f16x2_mul(e4m3x2_to_f16x2((uint16_t)(q.x >> 16)), sc);
+            o.z = f16x2_mul(e4m3x2_to_f16x2((uint16_t)(q.y & 0xffffu)), sc);
+            o.w = f16x2_mul(e4m3x2_to_f16x2((uint16_t)(q.y >> 16)), sc);
+            *reinterpret_cast<uint4 *>(a16 + r * 128 + ((c ^ (r & 7)) << 4)) = o;
           }
           fence_proxy_async_smem();
           __syncwarp();
@@ -520,6 +534,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   } else {
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;  // TMEM lane quarter this warp may access
+    const float acc_scale = F8 ? F8_SCALE_DOWN : 1.0f;
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int tile = unit; tile < total; tile += nunits) {
@@ -556,7 +571,8 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
           for (int j = 0; j < 32; ++j)
             if (c0 + j < t.nvalid)
-              atomicAdd(p.y + (size_t)s_tok[c0 + j] * p.D + d, s_gate[c0 + j] * __uint_as_float(v[j]));
+              atomicAdd(p.y + (size_t)s_tok[c0 + j] * p.D + d,
+                        s_gate[c0 + j] * (__uint_as_float(v[j]) * acc_scale));
         }
       } else if (MODE == 2) {
         // lanes are output features d, columns are tokens
@@ -576,7 +592,7 @@ __global__ void __launch_bounds__(THREADS, 1)
           tmem_wait_ld();
 #pragma unroll
           for (int j = 0; j < 32; ++j)
-            if (c0 + j < t.nvalid) out[(row0 + c0 + j) * p.D + d] = __uint_as_float(v[j]);
+            if (c0 + j < t.nvalid) out[(row0 + c0 + j) * p.D + d] = __uint_as_float(v[j]) * acc_scale;
         }
       } else {
         // lanes 0-63 hold w1.x (a), lanes 64-127 hold w3.x (u) for the same
@@ -602,10 +618,15 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
             const int col = is_a ? j : 16 + j;
-            const float a = is_a ? __uint_as_float(v[j]) : other[lane * XB_STRIDE + j];
-            const float u = is_a ? other[lane * XB_STRIDE + j] : __uint_as_float(v[16 + j]);
+            const float a = (is_a ? __uint_as_float(v[j]) : other[lane * XB_STRIDE + j]) * acc_scale;
+            const float u = (is_a ? other[lane * XB_STRIDE + j] : __uint_as_float(v[16 + j])) * acc_scale;
             const float h = a / (1.0f + expf(-a)) * u;
-            if (c0 + col < t.nvalid) out[(row0 + c0 + col) * p.I + f] = __float2bfloat16_rn(h);
+            if (c0 + col < t.nvalid) {
+              if (F8)  // fp16 h: the second matmul's operand on the e4m3 path
+                reinterpret_cast<__half *>(out)[(row0 + c0 + col) * p.I + f] = __float2half_rn(h);
+              else
+                out[(row0 + c0 + col) * p.I + f] = __float2bfloat16_rn(h);
+            }
           }
           named_bar_sync(1 + pr, 64);
         }
@@ -995,12 +1016,17 @@ moe_status tc_up(const Job &j) {
   bf16 *h = reinterpret_cast<bf16 *>(j.ws + j.l.h);
   prof(0, j.s);
   const int64_t threads = (int64_t)j.rows_total() * 32;
-  gather_rows<<<(unsigned)((threads + 255) / 256), 256, 0, j.s>>>(
-      static_cast<const uint4 *>(j.x), j.sorted_token, reinterpret_cast<uint4 *>(xperm),
-      j.rows_routed(), j.rows_total(), (int)j.T, D * 2 / 16);
+  if (F8)
+    gather_rows_f16<<<(unsigned)((threads + 255) / 256), 256, 0, j.s>>>(
+        static_cast<const __nv_bfloat162 *>(j.x), j.sorted_token,
+        reinterpret_cast<__half2 *>(xperm), j.rows_routed(), j.rows_total(), (int)j.T, D / 2);
+  else
+    gather_rows<<<(unsigned)((threads + 255) / 256), 256, 0, j.s>>>(
+        static_cast<const uint4 *>(j.x), j.sorted_token, reinterpret_cast<uint4 *>(xperm),
+        j.rows_routed(), j.rows_total(), (int)j.T, D * 2 / 16);
   if ((st = launch_status()) != MOE_OK) return st;
   CUtensorMap mw1, mw3, mx;
-  const CUtensorMapDataType BF = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  const CUtensorMapDataType BF = F8 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   if (!weight_tmap(&mw1, j.w->w1, F8, (uint64_t)G * I, D, 64) ||
       !weight_tmap(&mw3, j.w->w3, F8, (uint64_t)G * I, D, 64) ||
       !make_tmap(&mx, xperm, BF, 2, (uint64_t)j.l.rows_pad, D, BOXN, 64))
@@ -1029,7 +1055,7 @@ moe_status tc_down(const Job &j) {
   if (st != MOE_OK) return st;
   bf16 *h = reinterpret_cast<bf16 *>(j.ws + j.l.h);
   CUtensorMap mw2, mh;
-  const CUtensorMapDataType BF = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  const CUtensorMapDataType BF = F8 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   if (!weight_tmap(&mw2, j.w->w2, F8, (uint64_t)G * D, I, tc::BM) ||
       !make_tmap(&mh, h, BF, 2, (uint64_t)j.l.rows_pad, I, BOXN, 64))
     return MOE_ERR_CUDA;
