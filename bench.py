@@ -56,6 +56,22 @@ def dist_env():
             int(os.environ.get("WORLD_SIZE", 1)))
 
 
+def max_over_ranks(v: float, world: int, device) -> float:
+    """The largest value of v over all ranks (the job is as slow as its
+    slowest replica); v itself when there is one rank."""
+    if world == 1:
+        return v
+    t = torch.tensor([v], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tokens_per_s(world: int, T: int, steps: int, ms_total: float) -> float:
+    """Whole-job throughput of `world` replicas, each pushing `steps` batches of
+    T tokens, when the slowest one took ms_total."""
+    return world * T * steps / (ms_total / 1e3)
+
+
 # ---------------------------------------------------------------- clocks
 
 
@@ -222,15 +238,11 @@ def run_ours(args, rank, local_rank, world):
     clk = clocks.stop()
     if world > 1:
         torch.distributed.barrier()
-    ms_total = start.elapsed_time(end)
-    if world > 1:
-        t = torch.tensor([ms_total], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms_total = float(t.item())
+    ms_total = max_over_ranks(start.elapsed_time(end), world, dev)
     if blk.device_status() != 0:
         raise RuntimeError(f"device status {blk.device_status()} in the timed region")
     ms_step = ms_total / K
-    value = world * w.T * K / (ms_total / 1e3)
+    value = job_tokens_per_s(world, w.T, K, ms_total)
 
     # per-kernel durations inside the timed region
     spans = {"router": (0, 1), "dispatch": (1, 2), "gather": (3, 4), "gemm1": (4, 5),
@@ -294,12 +306,8 @@ def run_ours(args, rank, local_rank, world):
         blk.forward_host(x_host[i % N_X_BATCHES], y_host, x_dev)
     e1.record()
     torch.cuda.synchronize()
-    ms_e2e = e0.elapsed_time(e1)
-    if world > 1:
-        t = torch.tensor([ms_e2e], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms_e2e = float(t.item())
-    e2e = {"value": world * w.T * Ke / (ms_e2e / 1e3), "unit": "tokens/s",
+    ms_e2e = max_over_ranks(e0.elapsed_time(e1), world, dev)
+    e2e = {"value": job_tokens_per_s(world, w.T, Ke, ms_e2e), "unit": "tokens/s",
            "h2d_bytes_per_step": w.T * sh.dim * x_bytes, "d2h_bytes_per_step": w.T * sh.dim * 4,
            "steps": Ke}
 
