@@ -429,8 +429,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         const uint32_t idesc = F8 ? idesc_f16_f32(BM * CG, nmma) : idesc_bf16_f32(BM * CG, nmma);
         for (int kb = 0; kb < p.KB; ++kb) {
           if (!wait_bounded(full + stage, phase, abort_flag, p.timeout_ns, p.status) ||
-              (F8 && !wait_bounded<CG == 2>(conv + stage, phase, abort_flag, p.timeout_ns,
-                                            p.status))) {
+              (F8 && !wait_bounded(conv + stage, phase, abort_flag, p.timeout_ns, p.status))) {
             ok = false;
             break;
           }

@@ -290,10 +290,13 @@ __device__ __forceinline__ uint32_t mapa_shared(uint32_t saddr, uint32_t rank) {
   return r;
 }
 
-// Arrive on an mbarrier given by a shared::cluster address (any CTA of the cluster).
+// Arrive on an mbarrier given by a shared::cluster address (any CTA of the
+// cluster), with the default (CTA-scope release) semantics.  Data a CTA of a
+// pair writes for the tensor cores is published by its own
+// fence.proxy.async before it arrives; each SM's tensor core reads its own
+// CTA's share of the operands.
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
-               : "memory");
+  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
 
 // All threads of both CTAs of the cluster.
