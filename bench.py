@@ -330,7 +330,8 @@ def run_ours(args, rank, local_rank, world):
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None,
-        "dtype": "bf16" if w.w_format != "f32" else "f32",
+        # arithmetic type of the matmuls: e4m3 weights are expanded to f16
+        "dtype": {"bf16": "bf16", "f32": "f32", "e4m3": "f16"}[w.w_format],
         "data": "synthetic (seeded N(0,1) activations, N(0,1/fan_in) weights, U(-0.1,0.1) bias)",
         "config": {"workload": w.name, "T": w.T, "dim": sh.dim, "n_routed": sh.n_routed,
                    "combine": blk.combine_mode,

@@ -178,15 +178,18 @@ namespace tc {
 constexpr int BK = 64;                 // K elements per ring stage (128 bytes bf16)
 constexpr int BM = 128;                // MMA M: weight rows per tile
 constexpr int A_BYTES = BM * BK * 2;   // 16 KB
-// warp 0 issues TMA loads, warp 1 MMAs, warps 2-5 run the epilogue, warps 6-9
-// expand e4m3 weight tiles (idle with bf16 weights)
-constexpr int THREADS = 320;
-constexpr int CONV_WARPS = 4;
+// warp 0 issues TMA loads, warp 1 MMAs, warps 2-5 run the epilogue; with e4m3
+// weights, warps 6 .. 6 + CONV_WARPS - 1 expand the weight tiles
+#ifndef MOE_TC_CONV_WARPS
+#define MOE_TC_CONV_WARPS 8
+#endif
+constexpr int CONV_WARPS = MOE_TC_CONV_WARPS;
 // e4m3 path: the block scales are taken times 2^8 when the codes are expanded
 // (keeping scale and products in the fp16 normal range) and the accumulator is
 // multiplied by 2^-8 in the epilogue -- both exact powers of two
 constexpr float F8_SCALE_UP = 256.0f, F8_SCALE_DOWN = 1.0f / 256.0f;
 constexpr int EPI_WARPS = 4;
+__host__ __device__ constexpr int threads_of(bool f8) { return 32 * (2 + EPI_WARPS + (f8 ? CONV_WARPS : 0)); }
 constexpr int XB_STRIDE = 17;          // exchange buffer row stride (floats)
 
 struct Params {
@@ -261,7 +264,7 @@ __device__ __forceinline__ void sleep_ns(int64_t ns) {
 }
 
 template <int MODE, int CG, int BN_MAX, int BOXN, int STAGES, bool F8>
-__global__ void __launch_bounds__(THREADS, 1)
+__global__ void __launch_bounds__(threads_of(F8), 1)
     tc_expert_gemm(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA1,
                    const __grid_constant__ CUtensorMap tmB, const Params p) {
   using L = Layout<MODE, CG, BN_MAX, BOXN, STAGES, F8>;
@@ -314,9 +317,10 @@ __global__ void __launch_bounds__(THREADS, 1)
     if (MODE == 1) tma_prefetch_desc(&tmA1);
     tma_prefetch_desc(&tmB);
   }
-  for (int i = threadIdx.x; i <= p.G; i += THREADS) s_tstart[i] = p.tile_start[i];
-  for (int i = threadIdx.x; i < p.G; i += THREADS) s_tbase[i] = p.tile_base[i];
-  for (int i = threadIdx.x; i <= p.E; i += THREADS) s_off[i] = p.offsets[i];
+  constexpr int NT = threads_of(F8);
+  for (int i = threadIdx.x; i <= p.G; i += NT) s_tstart[i] = p.tile_start[i];
+  for (int i = threadIdx.x; i < p.G; i += NT) s_tbase[i] = p.tile_base[i];
+  for (int i = threadIdx.x; i <= p.E; i += NT) s_off[i] = p.offsets[i];
   if (warp == 1) {
     if (CG == 2) {
       tmem_alloc_pair(tmem_slot, L::TMEM_COLS);
@@ -491,15 +495,23 @@ __global__ void __launch_bounds__(THREADS, 1)
         const int r0 = MODE == 1 ? t.ft * L::FEAT + (int)rank * 64 : t.ft * L::FEAT + (int)rank * BM;
         const size_t srow = ((size_t)t.g * (rows_w / 128) + r0 / 128) * (cols_w / 128);
         const int k0 = k_rotation(t, p.KB);
+        // the block scales of the next k-block are loaded while this one's
+        // codes are awaited and expanded, keeping their latency off the path
+        float n0 = p.sA0[srow + k0 / 2], n1 = MODE == 1 ? p.sA1[srow + k0 / 2] : 0.0f;
         for (int i = 0; i < p.KB; ++i) {
-          const int kb = k0 + i < p.KB ? k0 + i : k0 + i - p.KB;
+          const int kn = k0 + i + 1 < p.KB ? k0 + i + 1 : k0 + i + 1 - p.KB;
+          const float c0 = n0, c1 = n1;
+          if (i + 1 < p.KB) {
+            n0 = p.sA0[srow + kn / 2];
+            if (MODE == 1) n1 = p.sA1[srow + kn / 2];
+          }
           if (!wait_bounded(a8full + stage, phase, abort_flag, p.timeout_ns, p.status)) {
             ok = false;
             break;
           }
           pend8[stage] = -1;
-          const uint32_t s0 = f16x2_splat(p.sA0[srow + kb / 2] * F8_SCALE_UP);
-          const uint32_t s1 = MODE == 1 ? f16x2_splat(p.sA1[srow + kb / 2] * F8_SCALE_UP) : s0;
+          const uint32_t s0 = f16x2_splat(c0 * F8_SCALE_UP);
+          const uint32_t s1 = MODE == 1 ? f16x2_splat(c1 * F8_SCALE_UP) : s0;
           const uint8_t *a8 = sm + stage * L::STAGE_BYTES + L::A8_OFF;
           uint8_t *a16 = sm + stage * L::STAGE_BYTES;
 #pragma unroll 4
@@ -912,7 +924,7 @@ moe_status launch_tc(const CUtensorMap &a0, const CUtensorMap &a1, const CUtenso
   if (nsm < 2) return MOE_ERR_CUDA;
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[1];
-  cfg.blockDim = dim3(tc::THREADS);
+  cfg.blockDim = dim3(tc::threads_of(F8));
   cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
   cfg.gridDim = dim3(nsm);
@@ -1165,6 +1177,9 @@ moe_status simt_down_w(const Job &j) {
 #ifndef MOE_TC_PREFILL_STAGES
 #define MOE_TC_PREFILL_STAGES 6
 #endif
+#ifndef MOE_TC_PREFILL_F8_STAGES
+#define MOE_TC_PREFILL_F8_STAGES 5
+#endif
 #ifndef MOE_TC_PREFILL_CG
 #define MOE_TC_PREFILL_CG 2
 #endif
@@ -1175,6 +1190,7 @@ moe_status simt_down_w(const Job &j) {
 #define MOE_TC_DECODE_STAGES 10
 #endif
 constexpr int PF_BN = MOE_TC_PREFILL_BN, PF_ST = MOE_TC_PREFILL_STAGES;
+constexpr int PF_ST8 = MOE_TC_PREFILL_F8_STAGES;
 constexpr int DC_BN = MOE_TC_DECODE_BN, DC_ST = MOE_TC_DECODE_STAGES;
 
 // few rows per expert (decode): one SM per tile, narrow token tiles and a deep
@@ -1193,14 +1209,14 @@ bool pair_ok(const Job &j) {
 template <bool F8>
 moe_status run_up_t(const Job &j) {
   if (decode_variant(j)) return tc_up<1, DC_BN, 32, F8 ? 7 : DC_ST, F8>(j);
-  if (pair_ok(j)) return tc_up<2, PF_BN, 32, F8 ? 5 : PF_ST, F8>(j);
+  if (pair_ok(j)) return tc_up<2, PF_BN, 32, F8 ? PF_ST8 : PF_ST, F8>(j);
   return tc_up<1, 256, 32, F8 ? 3 : 4, F8>(j);
 }
 
 template <bool F8>
 moe_status run_down_t(const Job &j) {
   if (decode_variant(j)) return tc_down<1, DC_BN, 32, F8 ? 7 : DC_ST, F8>(j);
-  if (pair_ok(j)) return tc_down<2, PF_BN, 32, F8 ? 5 : PF_ST, F8>(j);
+  if (pair_ok(j)) return tc_down<2, PF_BN, 32, F8 ? PF_ST8 : PF_ST, F8>(j);
   return tc_down<1, 256, 32, F8 ? 3 : 4, F8>(j);
 }
 

@@ -58,6 +58,16 @@ WORKLOADS = {
                                       BlockShape(dim=7168, n_routed=32, n_groups=8, topk_groups=4,
                                                  topk=8, inter=2048), 512, torch.bfloat16,
                                       "bf16", 1006, note="V3 dims, 32 experts, T=512"),
+    # the same for the T=64 decode batch: ~2 rows per expert, 32 experts
+    "prof_decode_e32_t8": Workload("prof_decode_e32_t8",
+                                   BlockShape(dim=7168, n_routed=32, n_groups=8, topk_groups=4,
+                                              topk=8, inter=2048), 8, torch.bfloat16,
+                                   "bf16", 1007, note="V3 dims, 32 experts, T=8"),
+    # and for the e4m3 T=8192 batch: ~256 rows per expert, 32 experts
+    "prof_fp8_e32_t1024": Workload("prof_fp8_e32_t1024",
+                                   BlockShape(dim=7168, n_routed=32, n_groups=8, topk_groups=4,
+                                              topk=8, inter=2048), 1024, torch.bfloat16,
+                                   "e4m3", 1008, note="V3 dims, 32 experts, T=1024, e4m3 weights"),
 }
 
 
