@@ -188,8 +188,12 @@ constexpr int CONV_WARPS = MOE_TC_CONV_WARPS;
 // (keeping scale and products in the fp16 normal range) and the accumulator is
 // multiplied by 2^-8 in the epilogue -- both exact powers of two
 constexpr float F8_SCALE_UP = 256.0f, F8_SCALE_DOWN = 1.0f / 256.0f;
-constexpr int EPI_WARPS = 4;
-__host__ __device__ constexpr int threads_of(bool f8) { return 32 * (2 + EPI_WARPS + (f8 ? CONV_WARPS : 0)); }
+// epilogue warps: four (one per TMEM lane quarter), or eight when a CTA holds
+// two weight tiles (two warps per lane quarter, alternating column chunks)
+__host__ __device__ constexpr int epi_warps(int at) { return at == 2 ? 8 : 4; }
+__host__ __device__ constexpr int threads_of(bool f8, int at) {
+  return 32 * (2 + epi_warps(at) + (f8 ? CONV_WARPS : 0));
+}
 constexpr int XB_STRIDE = 17;          // exchange buffer row stride (floats)
 
 struct Params {
@@ -216,34 +220,53 @@ struct Params {
 
 // CG = CTA group: 1 = one SM per tile; 2 = an SM pair per tile (cta_group::2),
 // where each CTA holds 128 weight rows and half of the token tile.
+// AT = weight tiles of 128 rows per CTA and stage.  AT = 1: one tile (GEMM1:
+// 64 rows of w1 over the same 64 rows of w3, so the SwiGLU halves meet in
+// different TMEM lanes).  AT = 2: two tiles, each with its own accumulator and
+// the same token rows (GEMM1: 128 rows of w1 and the same 128 rows of w3, so a
+// thread holds both halves of its features; GEMM2: two blocks of 128 rows of
+// w2), which halves the token bytes each weight byte is paired with.
 // F8: the weights arrive as e4m3 tiles (A8, 64 bytes per row) that the
 // converter warps expand into the bf16 tile the MMA reads.
-template <int MODE, int CG, int BN_MAX, int BOXN, int STAGES, bool F8>
+template <int MODE, int CG, int AT, int BN_MAX, int BOXN, int STAGES, bool F8>
 struct Layout {
+  static constexpr int EPI = epi_warps(AT);
+  static constexpr int NT = threads_of(F8, AT);
   static constexpr int B_ROWS = BN_MAX / CG;  // token rows one CTA holds per stage
   static constexpr int B_BYTES = B_ROWS * BK * 2;
-  static constexpr int A8_BYTES = F8 ? BM * BK : 0;
-  static constexpr int A8_OFF = A_BYTES + B_BYTES;  // within a stage
-  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + A8_BYTES;
+  static constexpr int A_ALL = AT * A_BYTES;  // all weight tiles of a stage
+  static constexpr int A8_BYTES = F8 ? AT * BM * BK : 0;
+  static constexpr int A8_OFF = A_ALL + B_BYTES;  // within a stage
+  static constexpr int STAGE_BYTES = A_ALL + B_BYTES + A8_BYTES;
+  // TMA parts of a stage's weights: GEMM1 always loads w1 and w3; rows per part
+  static constexpr int NPARTS = MODE == 1 ? 2 : AT;
+  static constexpr int PART_ROWS = MODE == 1 && AT == 1 ? 64 : BM;
   static constexpr int BAR_OFF = STAGES * STAGE_BYTES;
   // full, empty, [a8_full, converted], acc_full x2, acc_empty x2, drain
   static constexpr int NBARS = (F8 ? 4 : 2) * STAGES + 5;
   static constexpr int MISC_OFF = BAR_OFF + NBARS * 8;
   static constexpr int MISC_BYTES = 16 + 8 * STAGES;
   static constexpr int XBUF_OFF = (MISC_OFF + MISC_BYTES + 127) / 128 * 128;
-  // GEMM1: SwiGLU exchange buffers; MODE 3: the tile's (token, gate) list
-  static constexpr int XBUF_BYTES = MODE == 1 ? 2 * 2 * 32 * XB_STRIDE * 4 : MODE == 3 ? BN_MAX * 8 : 0;
+  // GEMM1 with AT = 1: SwiGLU exchange buffers; MODE 3: the tile's (token, gate) list
+  static constexpr int XBUF_BYTES =
+      MODE == 1 ? (AT == 1 ? 2 * 2 * 32 * XB_STRIDE * 4 : 0) : MODE == 3 ? BN_MAX * 8 : 0;
   static constexpr int TAB_OFF = XBUF_OFF + XBUF_BYTES;
+  // TMEM: AT accumulators of BN_MAX columns per tile, double-buffered when
+  // two tiles' worth fits in the 512 columns
+  static constexpr int ACC_COLS = AT * BN_MAX;
+  static constexpr int NBUF = 2 * ACC_COLS <= 512 ? 2 : 1;
   static constexpr uint32_t TMEM_COLS =
-      2 * BN_MAX <= 32 ? 32 : 2 * BN_MAX <= 64 ? 64 : 2 * BN_MAX <= 128 ? 128
-                                                : 2 * BN_MAX <= 256 ? 256 : 512;
-  // weight rows one tile covers: GEMM1 pairs 64 rows of w1 with the same 64
-  // rows of w3 per CTA; GEMM2 takes 128 rows of w2 per CTA
-  static constexpr int FEAT = (MODE == 1 ? 64 : BM) * CG;  // MODE 2 and 3: rows of w2
+      NBUF * ACC_COLS <= 32 ? 32 : NBUF * ACC_COLS <= 64 ? 64 : NBUF * ACC_COLS <= 128 ? 128
+                                 : NBUF * ACC_COLS <= 256 ? 256 : 512;
+  // weight rows one tile covers (per pair): GEMM1 features (each with a row
+  // of w1 and of w3), GEMM2 rows of w2
+  static constexpr int FEAT = (MODE == 1 ? (AT == 1 ? 64 : BM) : AT * BM) * CG;
   static size_t smem_bytes(int G, int E) {
     return 1024 + TAB_OFF + sizeof(int32_t) * (size_t)((G + 1) + G + (E + 1));
   }
   static_assert(CG == 1 || CG == 2, "CTA group");
+  static_assert(AT == 1 || AT == 2, "weight tiles per CTA");
+  static_assert(NBUF * ACC_COLS <= 512, "TMEM columns");
   static_assert(BN_MAX % 16 == 0 && BN_MAX >= 16 && BN_MAX <= 256, "MMA N range");
   static_assert(BOXN % 16 == 0 && B_ROWS % BOXN == 0, "B box rows");
 };
@@ -263,11 +286,11 @@ __device__ __forceinline__ void sleep_ns(int64_t ns) {
   }
 }
 
-template <int MODE, int CG, int BN_MAX, int BOXN, int STAGES, bool F8>
-__global__ void __launch_bounds__(threads_of(F8), 1)
+template <int MODE, int CG, int AT, int BN_MAX, int BOXN, int STAGES, bool F8>
+__global__ void __launch_bounds__(threads_of(F8, AT), 1)
     tc_expert_gemm(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA1,
                    const __grid_constant__ CUtensorMap tmB, const Params p) {
-  using L = Layout<MODE, CG, BN_MAX, BOXN, STAGES, F8>;
+  using L = Layout<MODE, CG, AT, BN_MAX, BOXN, STAGES, F8>;
   using namespace sm100;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -308,8 +331,8 @@ __global__ void __launch_bounds__(threads_of(F8), 1)
     }
     mbar_init(accf + 0, 1);
     mbar_init(accf + 1, 1);
-    mbar_init(acce + 0, EPI_WARPS * CG);
-    mbar_init(acce + 1, EPI_WARPS * CG);
+    mbar_init(acce + 0, L::EPI * CG);
+    mbar_init(acce + 1, L::EPI * CG);
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -317,7 +340,7 @@ __global__ void __launch_bounds__(threads_of(F8), 1)
     if (MODE == 1) tma_prefetch_desc(&tmA1);
     tma_prefetch_desc(&tmB);
   }
-  constexpr int NT = threads_of(F8);
+  constexpr int NT = L::NT;
   for (int i = threadIdx.x; i <= p.G; i += NT) s_tstart[i] = p.tile_start[i];
   for (int i = threadIdx.x; i < p.G; i += NT) s_tbase[i] = p.tile_base[i];
   for (int i = threadIdx.x; i <= p.E; i += NT) s_off[i] = p.offsets[i];
@@ -340,7 +363,11 @@ __global__ void __launch_bounds__(threads_of(F8), 1)
   if (warp == 0) {
     if (lane == 0) {
       // ---------------------------------------------------- TMA producer
-      const uint64_t pol_w = policy_evict_first();  // weights: streamed once
+      // weights: the first matmul keeps them at normal priority so that the
+      // token tiles of one expert that run at about the same time share them
+      // in L2; the second keeps them evict-first, because the fp32 sums it
+      // scatters into y need L2 more
+      const uint64_t pol_w = MODE == 1 ? policy_evict_normal() : policy_evict_first();
       const uint64_t pol_x = policy_evict_last();   // activations: re-read per feature tile
       int stage = 0;
       uint32_t phase = 0;
@@ -350,12 +377,14 @@ __global__ void __launch_bounds__(threads_of(F8), 1)
         const int nmma = (t.nvalid + 15) & ~15;
         const int brows = nmma / CG;  // this CTA's share of the token rows
         const int b0 = t.rowbase + t.n0 + (int)rank * brows;
-        const int arow = MODE == 1 ? t.g * p.I + t.ft * L::FEAT + (int)rank * 64
+        // first weight row of this CTA's part 0; part i of GEMM2 lies
+        // i * 128 * CG rows further, GEMM1's part 1 is w3 at the same rows
+        const int arow = MODE == 1 ? t.g * p.I + t.ft * L::FEAT + (int)rank * L::PART_ROWS
                                    : t.g * p.D + t.ft * L::FEAT + (int)rank * BM;
         const int nbox = (brows + BOXN - 1) / BOXN;
         // with e4m3 weights the full barrier counts only the token rows; the
         // weight tile arrives on this CTA's own a8_full barrier
-        const uint32_t bytes = (uint32_t)((F8 ? 0 : A_BYTES) + nbox * BOXN * BK * 2);
+        const uint32_t bytes = (uint32_t)((F8 ? 0 : L::A_ALL) + nbox * BOXN * BK * 2);
         const int k0 = k_rotation(t, p.KB);
         for (int i = 0; i < p.KB; ++i) {
           const int kb = k0 + i < p.KB ? k0 + i : k0 + i - p.KB;
@@ -367,17 +396,16 @@ __global__ void __launch_bounds__(threads_of(F8), 1)
           if (leader) mbar_arrive_expect_tx(full + stage, bytes * CG);
           pending[stage] = (int)phase;
           uint8_t *a_dst = sm + stage * L::STAGE_BYTES;
-          uint8_t *b_dst = a_dst + A_BYTES;
+          uint8_t *b_dst = a_dst + L::A_ALL;
           if (F8) {
             uint8_t *a8 = a_dst + L::A8_OFF;
             mbar_arrive_expect_tx(a8full + stage, L::A8_BYTES);
             pend8[stage] = (int)phase;
-            if (MODE == 1) {
-              tma_load_2d_hint(&tmA0, a8, a8full + stage, kb * BK, arow, pol_w);
-              tma_load_2d_hint(&tmA1, a8 + L::A8_BYTES / 2, a8full + stage, kb * BK, arow, pol_w);
-            } else {
-              tma_load_2d_hint(&tmA0, a8, a8full + stage, kb * BK, arow, pol_w);
-            }
+#pragma unroll
+            for (int i = 0; i < L::NPARTS; ++i)
+              tma_load_2d_hint(MODE == 1 && i == 1 ? &tmA1 : &tmA0,
+                               a8 + i * (L::A8_BYTES / L::NPARTS), a8full + stage, kb * BK,
+                               arow + (MODE == 1 ? 0 : i * BM * CG), pol_w);
             if (CG == 2) {
               const uint32_t fb = mapa_shared(smem_u32(full + stage), 0);
               for (int i = 0; i < nbox; ++i)
@@ -389,21 +417,19 @@ __global__ void __launch_bounds__(threads_of(F8), 1)
             }
           } else if (CG == 2) {
             const uint32_t fb = mapa_shared(smem_u32(full + stage), 0);
-            if (MODE == 1) {
-              tma_load_2d_pair(&tmA0, a_dst, fb, kb * BK, arow, pol_w);
-              tma_load_2d_pair(&tmA1, a_dst + A_BYTES / 2, fb, kb * BK, arow, pol_w);
-            } else {
-              tma_load_2d_pair(&tmA0, a_dst, fb, kb * BK, arow, pol_w);
-            }
+#pragma unroll
+            for (int i = 0; i < L::NPARTS; ++i)
+              tma_load_2d_pair(MODE == 1 && i == 1 ? &tmA1 : &tmA0,
+                               a_dst + i * (L::A_ALL / L::NPARTS), fb, kb * BK,
+                               arow + (MODE == 1 ? 0 : i * BM * CG), pol_w);
             for (int i = 0; i < nbox; ++i)
               tma_load_2d_pair(&tmB, b_dst + i * BOXN * BK * 2, fb, kb * BK, b0 + i * BOXN, pol_x);
           } else {
-            if (MODE == 1) {
-              tma_load_2d_hint(&tmA0, a_dst, full + stage, kb * BK, arow, pol_w);
-              tma_load_2d_hint(&tmA1, a_dst + A_BYTES / 2, full + stage, kb * BK, arow, pol_w);
-            } else {
-              tma_load_2d_hint(&tmA0, a_dst, full + stage, kb * BK, arow, pol_w);
-            }
+#pragma unroll
+            for (int i = 0; i < L::NPARTS; ++i)
+              tma_load_2d_hint(MODE == 1 && i == 1 ? &tmA1 : &tmA0,
+                               a_dst + i * (L::A_ALL / L::NPARTS), full + stage, kb * BK,
+                               arow + (MODE == 1 ? 0 : i * BM * CG), pol_w);
             for (int i = 0; i < nbox; ++i)
               tma_load_2d_hint(&tmB, b_dst + i * BOXN * BK * 2, full + stage, kb * BK,
                                b0 + i * BOXN, pol_x);
@@ -428,7 +454,7 @@ __global__ void __launch_bounds__(threads_of(F8), 1)
           break;
         }
         tc_fence_after();
-        const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN_MAX);
+        const uint32_t d_tmem = tmem_base + (uint32_t)(acc * L::ACC_COLS);
         const int nmma = (t.nvalid + 15) & ~15;
         const uint32_t idesc = F8 ? idesc_f16_f32(BM * CG, nmma) : idesc_bf16_f32(BM * CG, nmma);
         for (int kb = 0; kb < p.KB; ++kb) {
@@ -440,15 +466,19 @@ __global__ void __launch_bounds__(threads_of(F8), 1)
           pending[stage] = -1;
           tc_fence_after();
           const uint32_t a_addr = smem_u32(sm + stage * L::STAGE_BYTES);
-          const uint32_t b_addr = a_addr + A_BYTES;
+          const uint32_t b_addr = a_addr + L::A_ALL;
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk) {
-            const uint64_t ad = sdesc_sw128(a_addr + kk * 32), bd = sdesc_sw128(b_addr + kk * 32);
+            const uint64_t bd = sdesc_sw128(b_addr + kk * 32);
             const uint32_t accum = (kb | kk) != 0 ? 1u : 0u;
-            if (CG == 2)
-              mma_bf16_pair(d_tmem, ad, bd, idesc, accum);
-            else
-              mma_bf16(d_tmem, ad, bd, idesc, accum);
+#pragma unroll
+            for (int a = 0; a < AT; ++a) {
+              const uint64_t ad = sdesc_sw128(a_addr + a * A_BYTES + kk * 32);
+              if (CG == 2)
+                mma_bf16_pair(d_tmem + a * BN_MAX, ad, bd, idesc, accum);
+              else
+                mma_bf16(d_tmem + a * BN_MAX, ad, bd, idesc, accum);
+            }
           }
           if (CG == 2)
             mma_commit_pair_mc(empty + stage, 0x3);
@@ -464,8 +494,10 @@ __global__ void __launch_bounds__(threads_of(F8), 1)
           mma_commit_pair_mc(accf + acc, 0x3);
         else
           mma_commit(accf + acc);
-        acc ^= 1;
-        if (acc == 0) acc_phase ^= 1u;
+        if (++acc == L::NBUF) {
+          acc = 0;
+          acc_phase ^= 1u;
+        }
       }
       if (!ok) {
         // make sure no MMA is still writing TMEM before it is freed
@@ -476,7 +508,7 @@ __global__ void __launch_bounds__(threads_of(F8), 1)
         drain_wait(drain, 0, p.timeout_ns);
       }
     }
-  } else if (warp >= 2 + EPI_WARPS) {
+  } else if (warp >= 2 + L::EPI) {
     if (F8) {
       // ------------------------------------------------ e4m3 -> f16 converter
       // A8 row r (64 codes) becomes A row r (64 fp16) in the 128-byte swizzled
@@ -484,7 +516,7 @@ __global__ void __launch_bounds__(threads_of(F8), 1)
       // converts to fp16 exactly; it is then multiplied by 2^8 times the fp32
       // scale of its 128 x 128 block (rounded once to fp16).  On this path
       // the token rows and h are fp16 as well.
-      const int ct = threadIdx.x - 32 * (2 + EPI_WARPS);  // 0 .. 32 * CONV_WARPS - 1
+      const int ct = threadIdx.x - 32 * (2 + L::EPI);  // 0 .. 32 * CONV_WARPS - 1
       const int rows_w = MODE == 1 ? p.I : p.D;            // rows of one expert's matrix
       const int cols_w = MODE == 1 ? p.D : p.I;
       int stage = 0;
@@ -492,18 +524,23 @@ __global__ void __launch_bounds__(threads_of(F8), 1)
       bool ok = true;
       for (int tile = unit; ok && tile < total; tile += nunits) {
         const Tile t = decode_tile(tile, s_tstart, s_tbase, s_off, p.G, p.E, p.T, p.rows_routed);
-        const int r0 = MODE == 1 ? t.ft * L::FEAT + (int)rank * 64 : t.ft * L::FEAT + (int)rank * BM;
+        // scale rows of part 0 and part 1 (GEMM1: w1 and w3 at the same
+        // rows; GEMM2 with two parts: 128 * CG rows apart)
+        const int r0 = t.ft * L::FEAT + (int)rank * L::PART_ROWS;
         const size_t srow = ((size_t)t.g * (rows_w / 128) + r0 / 128) * (cols_w / 128);
+        const size_t srow1 =
+            MODE != 1 && AT == 2 ? srow + (size_t)CG * (cols_w / 128) : srow;
+        const float *sc1 = MODE == 1 ? p.sA1 : p.sA0;
         const int k0 = k_rotation(t, p.KB);
         // the block scales of the next k-block are loaded while this one's
         // codes are awaited and expanded, keeping their latency off the path
-        float n0 = p.sA0[srow + k0 / 2], n1 = MODE == 1 ? p.sA1[srow + k0 / 2] : 0.0f;
+        float n0 = p.sA0[srow + k0 / 2], n1 = L::NPARTS == 2 ? sc1[srow1 + k0 / 2] : 0.0f;
         for (int i = 0; i < p.KB; ++i) {
           const int kn = k0 + i + 1 < p.KB ? k0 + i + 1 : k0 + i + 1 - p.KB;
           const float c0 = n0, c1 = n1;
           if (i + 1 < p.KB) {
             n0 = p.sA0[srow + kn / 2];
-            if (MODE == 1) n1 = p.sA1[srow + kn / 2];
+            if (L::NPARTS == 2) n1 = sc1[srow1 + kn / 2];
           }
           if (!wait_bounded(a8full + stage, phase, abort_flag, p.timeout_ns, p.status)) {
             ok = false;
@@ -511,14 +548,14 @@ __global__ void __launch_bounds__(threads_of(F8), 1)
           }
           pend8[stage] = -1;
           const uint32_t s0 = f16x2_splat(c0 * F8_SCALE_UP);
-          const uint32_t s1 = MODE == 1 ? f16x2_splat(c1 * F8_SCALE_UP) : s0;
+          const uint32_t s1 = L::NPARTS == 2 ? f16x2_splat(c1 * F8_SCALE_UP) : s0;
           const uint8_t *a8 = sm + stage * L::STAGE_BYTES + L::A8_OFF;
           uint8_t *a16 = sm + stage * L::STAGE_BYTES;
 #pragma unroll 4
-          for (int it = 0; it < BM * 8 / (32 * CONV_WARPS); ++it) {
+          for (int it = 0; it < AT * BM * 8 / (32 * CONV_WARPS); ++it) {
             const int idx = ct + it * 32 * CONV_WARPS;
-            const int r = idx >> 3, c = idx & 7;
-            const uint32_t sc = (MODE == 1 && r >= 64) ? s1 : s0;
+            const int r = idx >> 3, c = idx & 7;  // rows of all parts lie back to back
+            const uint32_t sc = r >= L::PART_ROWS ? s1 : s0;
             const uint2 q = *reinterpret_cast<const uint2 *>(a8 + r * 64 + c * 8);
             uint4 o;
             o.x = f16x2_mul(e4m3x2_to_f16x2((uint16_t)(q.x & 0xffffu)), sc);
@@ -545,6 +582,10 @@ __global__ void __launch_bounds__(threads_of(F8), 1)
   } else {
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;  // TMEM lane quarter this warp may access
+    // with eight epilogue warps, the two warps of a lane quarter take
+    // alternate 32-column chunks
+    const int half = (warp - 2) >> 2;
+    constexpr int CSTEP = 32 * (L::EPI / 4);
     const float acc_scale = F8 ? F8_SCALE_DOWN : 1.0f;
     int acc = 0;
     uint32_t acc_phase = 0;
@@ -552,15 +593,15 @@ __global__ void __launch_bounds__(threads_of(F8), 1)
       const Tile t = decode_tile(tile, s_tstart, s_tbase, s_off, p.G, p.E, p.T, p.rows_routed);
       if (!wait_bounded(accf + acc, acc_phase, abort_flag, p.timeout_ns, p.status)) break;
       tc_fence_after();
-      const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN_MAX);
+      const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * L::ACC_COLS);
       if (MODE == 3) {
         // weighted scatter into y: y[t, d] += gate(t) * o[t, d] (gate 1 for the
         // shared expert), with fp32 reductions; first the tile's token list
         int32_t *s_tok = reinterpret_cast<int32_t *>(xbuf);
         float *s_gate = reinterpret_cast<float *>(s_tok + BN_MAX);
-        const int et = threadIdx.x - 64;  // 0..127 over the four epilogue warps
-        named_bar_sync(3, 128);            // the previous tile's readers are done
-        for (int c = et; c < t.nvalid; c += 128) {
+        const int et = threadIdx.x - 64;  // over all epilogue warps
+        named_bar_sync(3, 32 * L::EPI);    // the previous tile's readers are done
+        for (int c = et; c < t.nvalid; c += 32 * L::EPI) {
           int tok;
           float gate = 1.0f;
           if (t.g < p.E) {
@@ -573,17 +614,20 @@ __global__ void __launch_bounds__(threads_of(F8), 1)
           s_tok[c] = tok;
           s_gate[c] = gate;
         }
-        named_bar_sync(3, 128);
-        const int d = t.ft * L::FEAT + (int)rank * BM + q * 32 + lane;
-        for (int c0 = 0; c0 < t.nvalid; c0 += 32) {
-          uint32_t v[32];
-          tmem_ld_32x32b_x32(tb + (uint32_t)c0, v);
-          tmem_wait_ld();
+        named_bar_sync(3, 32 * L::EPI);
 #pragma unroll
-          for (int j = 0; j < 32; ++j)
-            if (c0 + j < t.nvalid)
-              atomicAdd(p.y + (size_t)s_tok[c0 + j] * p.D + d,
-                        s_gate[c0 + j] * (__uint_as_float(v[j]) * acc_scale));
+        for (int a = 0; a < AT; ++a) {
+          const int d = t.ft * L::FEAT + a * BM * CG + (int)rank * BM + q * 32 + lane;
+          for (int c0 = half * 32; c0 < t.nvalid; c0 += CSTEP) {
+            uint32_t v[32];
+            tmem_ld_32x32b_x32(tb + (uint32_t)(a * BN_MAX + c0), v);
+            tmem_wait_ld();
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              if (c0 + j < t.nvalid)
+                atomicAdd(p.y + (size_t)s_tok[c0 + j] * p.D + d,
+                          s_gate[c0 + j] * (__uint_as_float(v[j]) * acc_scale));
+          }
         }
       } else if (MODE == 2) {
         // lanes are output features d, columns are tokens
@@ -596,14 +640,41 @@ __global__ void __launch_bounds__(threads_of(F8), 1)
           out = p.out_shared;
           row0 = (size_t)(t.g - p.E) * p.T + t.n0;
         }
-        const int d = t.ft * L::FEAT + (int)rank * BM + q * 32 + lane;
-        for (int c0 = 0; c0 < t.nvalid; c0 += 32) {
-          uint32_t v[32];
-          tmem_ld_32x32b_x32(tb + (uint32_t)c0, v);
+#pragma unroll
+        for (int a = 0; a < AT; ++a) {
+          const int d = t.ft * L::FEAT + a * BM * CG + (int)rank * BM + q * 32 + lane;
+          for (int c0 = half * 32; c0 < t.nvalid; c0 += CSTEP) {
+            uint32_t v[32];
+            tmem_ld_32x32b_x32(tb + (uint32_t)(a * BN_MAX + c0), v);
+            tmem_wait_ld();
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              if (c0 + j < t.nvalid)
+                out[(row0 + c0 + j) * p.D + d] = __uint_as_float(v[j]) * acc_scale;
+          }
+        }
+      } else if (AT == 2) {
+        // lanes are features; the w1.x accumulator (a) and the w3.x one (u)
+        // sit BN_MAX columns apart in the same lanes
+        const int f = t.ft * L::FEAT + (int)rank * BM + q * 32 + lane;
+        const size_t row0 = (size_t)t.rowbase + t.n0;
+        for (int c0 = half * 32; c0 < t.nvalid; c0 += CSTEP) {
+          uint32_t va[32], vu[32];
+          tmem_ld_32x32b_x32(tb + (uint32_t)c0, va);
+          tmem_ld_32x32b_x32(tb + (uint32_t)(BN_MAX + c0), vu);
           tmem_wait_ld();
 #pragma unroll
-          for (int j = 0; j < 32; ++j)
-            if (c0 + j < t.nvalid) out[(row0 + c0 + j) * p.D + d] = __uint_as_float(v[j]) * acc_scale;
+          for (int j = 0; j < 32; ++j) {
+            const float a = __uint_as_float(va[j]) * acc_scale;
+            const float u = __uint_as_float(vu[j]) * acc_scale;
+            const float h = a / (1.0f + expf(-a)) * u;
+            if (c0 + j < t.nvalid) {
+              if (F8)  // fp16 h: the second matmul's operand on the e4m3 path
+                reinterpret_cast<__half *>(p.out)[(row0 + c0 + j) * p.I + f] = __float2half_rn(h);
+              else
+                static_cast<bf16 *>(p.out)[(row0 + c0 + j) * p.I + f] = __float2bfloat16_rn(h);
+            }
+          }
         }
       } else {
         // lanes 0-63 hold w1.x (a), lanes 64-127 hold w3.x (u) for the same
@@ -650,8 +721,10 @@ __global__ void __launch_bounds__(threads_of(F8), 1)
         else
           mbar_arrive(acce + acc);
       }
-      acc ^= 1;
-      if (acc == 0) acc_phase ^= 1u;
+      if (++acc == L::NBUF) {
+        acc = 0;
+        acc_phase ^= 1u;
+      }
     }
   }
 
@@ -909,11 +982,11 @@ WsLayout ws_layout(const moe_cfg *c, int64_t T, moe_dtype x_dt, moe_dtype w_dt) 
   return l;
 }
 
-template <int MODE, int CG, int BN_MAX, int BOXN, int STAGES, bool F8>
+template <int MODE, int CG, int AT, int BN_MAX, int BOXN, int STAGES, bool F8>
 moe_status launch_tc(const CUtensorMap &a0, const CUtensorMap &a1, const CUtensorMap &b,
                      const tc::Params &p, cudaStream_t s) {
-  using L = tc::Layout<MODE, CG, BN_MAX, BOXN, STAGES, F8>;
-  auto kern = tc::tc_expert_gemm<MODE, CG, BN_MAX, BOXN, STAGES, F8>;
+  using L = tc::Layout<MODE, CG, AT, BN_MAX, BOXN, STAGES, F8>;
+  auto kern = tc::tc_expert_gemm<MODE, CG, AT, BN_MAX, BOXN, STAGES, F8>;
   const size_t smem_max = 232448;
   if (L::smem_bytes(p.G, p.E) > smem_max) return MOE_ERR_UNSUPPORTED;
   const size_t smem = L::smem_bytes(p.G, p.E);
@@ -924,7 +997,7 @@ moe_status launch_tc(const CUtensorMap &a0, const CUtensorMap &a1, const CUtenso
   if (nsm < 2) return MOE_ERR_CUDA;
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[1];
-  cfg.blockDim = dim3(tc::threads_of(F8));
+  cfg.blockDim = dim3(L::NT);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
   cfg.gridDim = dim3(nsm);
@@ -1014,11 +1087,12 @@ bool weight_tmap(CUtensorMap *m, const void *w, bool f8, uint64_t rows, uint64_t
   return make_tmap(m, w, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, rows, cols, box_rows, 64);
 }
 
-template <int CG, int BN_MAX, int BOXN, int STAGES, bool F8>
+template <int CG, int AT, int BN_MAX, int BOXN, int STAGES, bool F8>
 moe_status tc_up(const Job &j) {
+  using L = tc::Layout<1, CG, AT, BN_MAX, BOXN, STAGES, F8>;
   const int G = j.G(), D = j.c->dim, I = j.c->inter;
   int32_t *tab = j.tab();
-  Tiling t1{BN_MAX, I / (64 * CG), tab, tab + (G + 1)};
+  Tiling t1{BN_MAX, I / L::FEAT, tab, tab + (G + 1)};
   Tiling none{0, 0, nullptr, nullptr};
   prep_tiles<<<1, 32, 0, j.s>>>(j.offsets, j.E(), G, (int)j.T, t1, none);
   moe_status st = launch_status();
@@ -1038,8 +1112,8 @@ moe_status tc_up(const Job &j) {
   if ((st = launch_status()) != MOE_OK) return st;
   CUtensorMap mw1, mw3, mx;
   const CUtensorMapDataType BF = F8 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
-  if (!weight_tmap(&mw1, j.w->w1, F8, (uint64_t)G * I, D, 64) ||
-      !weight_tmap(&mw3, j.w->w3, F8, (uint64_t)G * I, D, 64) ||
+  if (!weight_tmap(&mw1, j.w->w1, F8, (uint64_t)G * I, D, L::PART_ROWS) ||
+      !weight_tmap(&mw3, j.w->w3, F8, (uint64_t)G * I, D, L::PART_ROWS) ||
       !make_tmap(&mx, xperm, BF, 2, (uint64_t)j.l.rows_pad, D, BOXN, 64))
     return MOE_ERR_CUDA;
   tc::Params p = tc_params(j);
@@ -1050,16 +1124,17 @@ moe_status tc_up(const Job &j) {
   p.sA0 = j.w->s1;
   p.sA1 = j.w->s3;
   prof(1, j.s);
-  st = launch_tc<1, CG, BN_MAX, BOXN, STAGES, F8>(mw1, mw3, mx, p, j.s);
+  st = launch_tc<1, CG, AT, BN_MAX, BOXN, STAGES, F8>(mw1, mw3, mx, p, j.s);
   prof(2, j.s);
   return st;
 }
 
-template <int CG, int BN_MAX, int BOXN, int STAGES, bool F8>
+template <int CG, int AT, int BN_MAX, int BOXN, int STAGES, bool F8>
 moe_status tc_down(const Job &j) {
+  using L = tc::Layout<3, CG, AT, BN_MAX, BOXN, STAGES, F8>;
   const int G = j.G(), D = j.c->dim, I = j.c->inter;
   int32_t *tab = j.tab();
-  Tiling t2{BN_MAX, D / (tc::BM * CG), tab + (2 * G + 1), tab + (3 * G + 2)};
+  Tiling t2{BN_MAX, D / L::FEAT, tab + (2 * G + 1), tab + (3 * G + 2)};
   Tiling none{0, 0, nullptr, nullptr};
   prep_tiles<<<1, 32, 0, j.s>>>(j.offsets, j.E(), G, (int)j.T, t2, none);
   moe_status st = launch_status();
@@ -1079,9 +1154,9 @@ moe_status tc_down(const Job &j) {
   p.sA1 = j.w->s2;
   prof(3, j.s);
   if (j.y)
-    st = launch_tc<3, CG, BN_MAX, BOXN, STAGES, F8>(mw2, mw2, mh, p, j.s);
+    st = launch_tc<3, CG, AT, BN_MAX, BOXN, STAGES, F8>(mw2, mw2, mh, p, j.s);
   else
-    st = launch_tc<2, CG, BN_MAX, BOXN, STAGES, F8>(mw2, mw2, mh, p, j.s);
+    st = launch_tc<2, CG, AT, BN_MAX, BOXN, STAGES, F8>(mw2, mw2, mh, p, j.s);
   prof(4, j.s);
   return st;
 }
@@ -1174,11 +1249,14 @@ moe_status simt_down_w(const Job &j) {
 #ifndef MOE_TC_PREFILL_BN
 #define MOE_TC_PREFILL_BN 256
 #endif
-#ifndef MOE_TC_PREFILL_STAGES
-#define MOE_TC_PREFILL_STAGES 6
+// weight tiles per SM in the first matmul (two: w1 and w3 in accumulators of
+// their own, half the token bytes per weight byte) and in the second (one:
+// its K loop is short, and double-buffered accumulators hide the epilogue)
+#ifndef MOE_TC_PREFILL_AT_UP
+#define MOE_TC_PREFILL_AT_UP 2
 #endif
-#ifndef MOE_TC_PREFILL_F8_STAGES
-#define MOE_TC_PREFILL_F8_STAGES 5
+#ifndef MOE_TC_PREFILL_AT_DOWN
+#define MOE_TC_PREFILL_AT_DOWN 1
 #endif
 #ifndef MOE_TC_PREFILL_CG
 #define MOE_TC_PREFILL_CG 2
@@ -1189,8 +1267,12 @@ moe_status simt_down_w(const Job &j) {
 #ifndef MOE_TC_DECODE_STAGES
 #define MOE_TC_DECODE_STAGES 10
 #endif
-constexpr int PF_BN = MOE_TC_PREFILL_BN, PF_ST = MOE_TC_PREFILL_STAGES;
-constexpr int PF_ST8 = MOE_TC_PREFILL_F8_STAGES;
+constexpr int PF_BN = MOE_TC_PREFILL_BN;
+constexpr int PF_AT_UP = MOE_TC_PREFILL_AT_UP, PF_AT_DOWN = MOE_TC_PREFILL_AT_DOWN;
+// ring depth filling about 200 KB of shared memory: a stage holds AT 16 KB
+// weight tiles, PF_BN / 2 token rows of 128 bytes and, with e4m3 weights, AT
+// 8 KB code tiles
+constexpr int pf_stages(int at, bool f8) { return 200 * 1024 / (at * (f8 ? 24576 : 16384) + PF_BN * 64); }
 constexpr int DC_BN = MOE_TC_DECODE_BN, DC_ST = MOE_TC_DECODE_STAGES;
 
 // few rows per expert (decode): one SM per tile, narrow token tiles and a deep
@@ -1198,26 +1280,28 @@ constexpr int DC_BN = MOE_TC_DECODE_BN, DC_ST = MOE_TC_DECODE_STAGES;
 // token tiles of up to PF_BN rows, each SM holding half of them
 bool decode_variant(const Job &j) { return j.T * j.c->topk <= (int64_t)16 * j.c->n_routed; }
 
-// an SM pair per tile (cta_group::2) covers 128 features of w1/w3 and 256 rows of w2
+// an SM pair per tile (cta_group::2) covers 64 * 2 * PF_AT_UP features of
+// w1/w3 and 256 * PF_AT_DOWN rows of w2
 bool pair_ok(const Job &j) {
-  return MOE_TC_PREFILL_CG == 2 && j.c->inter % 128 == 0 && j.c->dim % 256 == 0;
+  return MOE_TC_PREFILL_CG == 2 && j.c->inter % (128 * PF_AT_UP) == 0 &&
+         j.c->dim % (256 * PF_AT_DOWN) == 0;
 }
 
-// e4m3 weights add an 8 KB code tile per stage (stage = 16 KB bf16 weights +
-// tokens + 8 KB codes); the ring depths shrink to fit shared memory, and half
-// as many weight bytes need to be in flight.
+// e4m3 weights add 8 KB of codes per weight tile and stage; the ring depths
+// shrink to fit shared memory, and half as many weight bytes need to be in
+// flight.
 template <bool F8>
 moe_status run_up_t(const Job &j) {
-  if (decode_variant(j)) return tc_up<1, DC_BN, 32, F8 ? 7 : DC_ST, F8>(j);
-  if (pair_ok(j)) return tc_up<2, PF_BN, 32, F8 ? PF_ST8 : PF_ST, F8>(j);
-  return tc_up<1, 256, 32, F8 ? 3 : 4, F8>(j);
+  if (decode_variant(j)) return tc_up<1, 1, DC_BN, 32, F8 ? 7 : DC_ST, F8>(j);
+  if (pair_ok(j)) return tc_up<2, PF_AT_UP, PF_BN, 32, pf_stages(PF_AT_UP, F8), F8>(j);
+  return tc_up<1, 1, 256, 32, F8 ? 3 : 4, F8>(j);
 }
 
 template <bool F8>
 moe_status run_down_t(const Job &j) {
-  if (decode_variant(j)) return tc_down<1, DC_BN, 32, F8 ? 7 : DC_ST, F8>(j);
-  if (pair_ok(j)) return tc_down<2, PF_BN, 32, F8 ? PF_ST8 : PF_ST, F8>(j);
-  return tc_down<1, 256, 32, F8 ? 3 : 4, F8>(j);
+  if (decode_variant(j)) return tc_down<1, 1, DC_BN, 32, F8 ? 7 : DC_ST, F8>(j);
+  if (pair_ok(j)) return tc_down<2, PF_AT_DOWN, PF_BN, 32, pf_stages(PF_AT_DOWN, F8), F8>(j);
+  return tc_down<1, 1, 256, 32, F8 ? 3 : 4, F8>(j);
 }
 
 moe_status run_up(const Job &j) {
