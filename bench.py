@@ -45,6 +45,8 @@ def parse():
     ap.add_argument("--cpu-sample", type=int, default=8,
                     help="tokens the oracle pushes through the block for cpu_baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-graph", action="store_true",
+                    help="skip the CUDA-graph replay timing of the same forward")
     ap.add_argument("--combine", choices=["scatter", "ordered"], default="scatter",
                     help="weighted sum into y inside the second matmul, or ordered and "
                          "bit-reproducible in a separate pass")
@@ -311,6 +313,42 @@ def run_ours(args, rank, local_rank, world):
            "h2d_bytes_per_step": w.T * sh.dim * x_bytes, "d2h_bytes_per_step": w.T * sh.dim * 4,
            "steps": Ke}
 
+    # the same forward captured once as a CUDA graph and replayed: what the
+    # launch gaps between the kernels cost (each step copies its batch into
+    # the graph's input buffer first, inside the timed region)
+    graph = None
+    if not args.no_graph:
+        x_g = xs[0].clone()
+        side = torch.cuda.Stream(device=dev)
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            blk.forward(x_g)
+        torch.cuda.current_stream().wait_stream(side)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            blk.forward(x_g)
+        Kg = max(1, min(K, 50))
+        for i in range(3):
+            x_g.copy_(xs[i % N_X_BATCHES])
+            g.replay()
+        torch.cuda.synchronize()
+        if world > 1:
+            torch.distributed.barrier()
+        g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        g0.record()
+        for i in range(Kg):
+            x_g.copy_(xs[i % N_X_BATCHES])
+            g.replay()
+        g1.record()
+        torch.cuda.synchronize()
+        ms_g = max_over_ranks(g0.elapsed_time(g1), world, dev)
+        if blk.device_status() != 0:
+            raise RuntimeError(f"device status {blk.device_status()} in the graph replays")
+        graph = {"value": job_tokens_per_s(world, w.T, Kg, ms_g), "unit": "tokens/s",
+                 "ms_per_step": ms_g / Kg, "steps": Kg,
+                 "gpu_launches_per_step": blk.launches_per_forward}
+        del g
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         try:
@@ -341,7 +379,7 @@ def run_ours(args, rank, local_rank, world):
                          f"{(sh.n_routed + 1) * 3 * sh.dim * sh.inter * w_bytes / 1e9:.1f} GB "
                          "of expert weights per step"},
         "roofline": roof, "step_roofline": step_roof,
-        "kernels_ms": dur, "cpu_baseline": cpu, "e2e": e2e,
+        "kernels_ms": dur, "cpu_baseline": cpu, "e2e": e2e, "graph": graph,
         "gpu_launches": K * blk.launches_per_forward,
         "clocks": clk, "touched_experts": touched, "hot_share": hot,
     }

@@ -63,6 +63,12 @@ WORKLOADS = {
                                    BlockShape(dim=7168, n_routed=32, n_groups=8, topk_groups=4,
                                               topk=8, inter=2048), 8, torch.bfloat16,
                                    "bf16", 1007, note="V3 dims, 32 experts, T=8"),
+    # the V3 router (dim 7168, 256 experts, T=4096) with narrow experts, so
+    # that a capture of the router kernels holds little else on the device
+    "prof_router_t4096": Workload("prof_router_t4096",
+                                  BlockShape(dim=7168, n_routed=256, n_groups=8, topk_groups=4,
+                                             topk=8, inter=128), 4096, torch.bfloat16,
+                                  "bf16", 1009, note="V3 router shapes, inter 128, T=4096"),
     # and for the e4m3 T=8192 batch: ~256 rows per expert, 32 experts
     "prof_fp8_e32_t1024": Workload("prof_fp8_e32_t1024",
                                    BlockShape(dim=7168, n_routed=32, n_groups=8, topk_groups=4,
