@@ -271,6 +271,14 @@ struct Layout {
   static_assert(BOXN % 16 == 0 && B_ROWS % BOXN == 0, "B box rows");
 };
 
+// silu(a) * u for the tensor-core epilogues, whose h is rounded to bf16 (or
+// fp16) right after: the hardware exp2 and reciprocal used here are within a
+// few parts in 1e6 of the exact value for the |a| that occur, far inside that
+// rounding, at a third of the instructions of the IEEE-exact forms
+__device__ __forceinline__ float swiglu_h(float a, float u) {
+  return __fdividef(a, 1.0f + __expf(-a)) * u;
+}
+
 // Waits for a barrier phase with a time limit but ignores the abort flag;
 // used only to drain copies already in flight before the CTA exits.
 __device__ __forceinline__ void drain_wait(uint64_t *bar, uint32_t parity, int64_t limit_ns) {
@@ -594,6 +602,19 @@ __global__ void __launch_bounds__(threads_of(F8, AT), 1)
       if (!wait_bounded(accf + acc, acc_phase, abort_flag, p.timeout_ns, p.status)) break;
       tc_fence_after();
       const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * L::ACC_COLS);
+      // hands the accumulator back to the MMA once this warp has read it
+      bool released = false;
+      auto release = [&]() {
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          if (CG == 2)
+            mbar_arrive_cluster(mapa_shared(smem_u32(acce + acc), 0));  // the leader's barrier
+          else
+            mbar_arrive(acce + acc);
+        }
+        released = true;
+      };
       if (MODE == 3) {
         // weighted scatter into y: y[t, d] += gate(t) * o[t, d] (gate 1 for the
         // shared expert), with fp32 reductions; first the tile's token list
@@ -656,6 +677,8 @@ __global__ void __launch_bounds__(threads_of(F8, AT), 1)
       } else if (AT == 2) {
         // lanes are features; the w1.x accumulator (a) and the w3.x one (u)
         // sit BN_MAX columns apart in the same lanes
+        // the accumulator is single-buffered here, so each warp releases it
+        // right after its last TMEM read, before that chunk's arithmetic
         const int f = t.ft * L::FEAT + (int)rank * BM + q * 32 + lane;
         const size_t row0 = (size_t)t.rowbase + t.n0;
         for (int c0 = half * 32; c0 < t.nvalid; c0 += CSTEP) {
@@ -663,11 +686,11 @@ __global__ void __launch_bounds__(threads_of(F8, AT), 1)
           tmem_ld_32x32b_x32(tb + (uint32_t)c0, va);
           tmem_ld_32x32b_x32(tb + (uint32_t)(BN_MAX + c0), vu);
           tmem_wait_ld();
+          if (c0 + CSTEP >= t.nvalid) release();
 #pragma unroll
           for (int j = 0; j < 32; ++j) {
-            const float a = __uint_as_float(va[j]) * acc_scale;
-            const float u = __uint_as_float(vu[j]) * acc_scale;
-            const float h = a / (1.0f + expf(-a)) * u;
+            const float h = swiglu_h(__uint_as_float(va[j]) * acc_scale,
+                                     __uint_as_float(vu[j]) * acc_scale);
             if (c0 + j < t.nvalid) {
               if (F8)  // fp16 h: the second matmul's operand on the e4m3 path
                 reinterpret_cast<__half *>(p.out)[(row0 + c0 + j) * p.I + f] = __float2half_rn(h);
@@ -702,7 +725,7 @@ __global__ void __launch_bounds__(threads_of(F8, AT), 1)
             const int col = is_a ? j : 16 + j;
             const float a = (is_a ? __uint_as_float(v[j]) : other[lane * XB_STRIDE + j]) * acc_scale;
             const float u = (is_a ? other[lane * XB_STRIDE + j] : __uint_as_float(v[16 + j])) * acc_scale;
-            const float h = a / (1.0f + expf(-a)) * u;
+            const float h = swiglu_h(a, u);
             if (c0 + col < t.nvalid) {
               if (F8)  // fp16 h: the second matmul's operand on the e4m3 path
                 reinterpret_cast<__half *>(out)[(row0 + c0 + col) * p.I + f] = __float2half_rn(h);
@@ -713,14 +736,7 @@ __global__ void __launch_bounds__(threads_of(F8, AT), 1)
           named_bar_sync(1 + pr, 64);
         }
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) {
-        if (CG == 2)
-          mbar_arrive_cluster(mapa_shared(smem_u32(acce + acc), 0));  // the leader's barrier
-        else
-          mbar_arrive(acce + acc);
-      }
+      if (!released) release();
       if (++acc == L::NBUF) {
         acc = 0;
         acc_phase ^= 1u;

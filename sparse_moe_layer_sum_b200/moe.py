@@ -274,12 +274,12 @@ class MoEBlock:
             self.ws_dispatch.data_ptr(), self.ws_dispatch.numel(), self.status.data_ptr(), s),
             "moe_dispatch_build")
 
-    def _experts(self, x, cfgp, s):
+    def _experts(self, x, cfgp, s, y):
         if self.combine_mode == "scatter":
             check(fn("moe_experts", "moe_experts_forward_combine")(
                 cfgp, self.T, x.data_ptr(), _dt(x), ctypes.byref(self.wstruct),
                 self.offsets.data_ptr(), self.sorted_token.data_ptr(), self.indices.data_ptr(),
-                self.weights.data_ptr(), self.y.data_ptr(), self.ws_experts.data_ptr(),
+                self.weights.data_ptr(), y.data_ptr(), self.ws_experts.data_ptr(),
                 self.ws_experts.numel(), self.status.data_ptr(), s),
                 "moe_experts_forward_combine")
             return
@@ -289,23 +289,27 @@ class MoEBlock:
             _ptr(self.out_shared), self.ws_experts.data_ptr(), self.ws_experts.numel(),
             self.status.data_ptr(), s), "moe_experts_forward")
 
-    def _combine(self, cfgp, s):
+    def _combine(self, cfgp, s, y):
         if self.combine_mode == "scatter":
             return  # done inside the experts' second matmul
         check(fn("moe_combine", "moe_combine")(
             cfgp, self.T, self.weights.data_ptr(), self.slot_of.data_ptr(),
-            self.out_perm.data_ptr(), _ptr(self.out_shared), self.y.data_ptr(),
+            self.out_perm.data_ptr(), _ptr(self.out_shared), y.data_ptr(),
             self.status.data_ptr(), s), "moe_combine")
 
-    def forward(self, x: torch.Tensor) -> torch.Tensor:
-        """Enqueue the four libraries for x [T, dim]; returns self.y (fp32)."""
+    def forward(self, x: torch.Tensor, y: Optional[torch.Tensor] = None) -> torch.Tensor:
+        """Enqueue the four libraries for x [T, dim]; returns y (fp32 [T, dim],
+        self.y unless another device buffer is given)."""
         assert x.shape == (self.T, self.shape.dim) and x.is_cuda and x.is_contiguous()
+        if y is None:
+            y = self.y
+        assert y.shape == (self.T, self.shape.dim) and y.dtype == torch.float32 and y.is_contiguous()
         cfgp, s = ctypes.byref(self.cfg), _stream()
         self._router(x, cfgp, s)
         self._dispatch(cfgp, s)
-        self._experts(x, cfgp, s)
-        self._combine(cfgp, s)
-        return self.y
+        self._experts(x, cfgp, s, y)
+        self._combine(cfgp, s, y)
+        return y
 
     def forward_profiled(self, x: torch.Tensor, ev) -> torch.Tensor:
         """forward() with 10 CUDA events recorded on the stream: around the
@@ -322,11 +326,11 @@ class MoEBlock:
         handles = (ctypes.c_void_p * 5)(*[e.cuda_event for e in ev[3:8]])
         check(fn("moe_experts", "moe_experts_set_profile_events")(handles, 5), "profile events")
         try:
-            self._experts(x, cfgp, s)
+            self._experts(x, cfgp, s, self.y)
         finally:
             fn("moe_experts", "moe_experts_set_profile_events")(None, 0)
         ev[8].record()
-        self._combine(cfgp, s)
+        self._combine(cfgp, s, self.y)
         ev[9].record()
         return self.y
 
@@ -339,6 +343,66 @@ class MoEBlock:
         y_host.copy_(self.y, non_blocking=True)
         return y_host
 
+    def host_pipeline(self) -> "HostPipeline":
+        """A HostPipeline over this block (see there)."""
+        return HostPipeline(self)
+
     def device_status(self) -> int:
         """The first device-side error of the forwards so far (0 = none); syncs."""
         return int(self.status.item())
+
+
+class HostPipeline:
+    """End-to-end forwards from pinned host memory with the copies overlapped.
+
+    submit(x_host, y_host) enqueues one batch: its input copy runs on a
+    host-to-device stream, the block on the caller's current stream, and the
+    copy of its y into y_host on a device-to-host stream.  Two device input
+    and output buffers alternate, so batch i's copies overlap the compute of
+    batches i-1 and i+1.  Ordering is kept with CUDA events only (no host
+    synchronisation); finish() makes the current stream wait for the last
+    output copy.  y_host must stay untouched until then.
+    """
+
+    def __init__(self, blk: "MoEBlock"):
+        self.blk = blk
+        dev = blk.y.device
+        T, D = blk.T, blk.shape.dim
+        self.x_dev = [torch.empty(T, D, dtype=blk.x_dtype, device=dev) for _ in range(2)]
+        self.y_dev = [torch.empty(T, D, dtype=torch.float32, device=dev) for _ in range(2)]
+        self.h2d = torch.cuda.Stream(device=dev)
+        self.d2h = torch.cuda.Stream(device=dev)
+        ev = lambda: [torch.cuda.Event() for _ in range(2)]  # noqa: E731
+        self.x_ready, self.x_free, self.y_ready, self.y_free = ev(), ev(), ev(), ev()
+        self.used = [False, False]
+        self.i = 0
+        self.last = None
+
+    def submit(self, x_host: torch.Tensor, y_host: torch.Tensor) -> None:
+        b = self.i % 2
+        comp = torch.cuda.current_stream(self.x_dev[b].device)
+        if self.i == 0:  # copies start after whatever the caller enqueued so far
+            self.h2d.wait_stream(comp)
+            self.d2h.wait_stream(comp)
+        with torch.cuda.stream(self.h2d):
+            if self.used[b]:
+                self.h2d.wait_event(self.x_free[b])     # the block two batches back read it
+            self.x_dev[b].copy_(x_host, non_blocking=True)
+            self.x_ready[b].record(self.h2d)
+        comp.wait_event(self.x_ready[b])
+        if self.used[b]:
+            comp.wait_event(self.y_free[b])             # its output copy has left
+        self.blk.forward(self.x_dev[b], self.y_dev[b])
+        self.x_free[b].record(comp)
+        self.y_ready[b].record(comp)
+        with torch.cuda.stream(self.d2h):
+            self.d2h.wait_event(self.y_ready[b])
+            y_host.copy_(self.y_dev[b], non_blocking=True)
+            self.y_free[b].record(self.d2h)
+        self.last = self.y_free[b]
+        self.used[b] = True
+        self.i += 1
+
+    def finish(self) -> None:
+        if self.last is not None:
+            torch.cuda.current_stream(self.x_dev[0].device).wait_event(self.last)
