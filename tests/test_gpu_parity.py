@@ -11,8 +11,9 @@ import torch
 from oracle import moe_oracle as O
 from parity import compare_routing, oracle_route, oracle_shape, oracle_y, y_close
 from sparse_moe_layer_sum_b200 import moe
-from sparse_moe_layer_sum_b200.inputs import (WORKLOADS, custom, make_block, random_topk_indices,
-                                              to_host_f32)
+from sparse_moe_layer_sum_b200.moe import BlockShape
+from sparse_moe_layer_sum_b200.inputs import (WORKLOADS, Workload, custom, make_block,
+                                              random_topk_indices, to_host_f32)
 
 pytestmark = pytest.mark.gpu
 
@@ -44,6 +45,15 @@ FP8_SMALL = custom("fp8_small", 260, w_format="e4m3", dim=512, n_routed=16, n_gr
                    topk_groups=2, topk=4, inter=256, seed=17)
 FP8_DECODE = custom("fp8_decode", 40, w_format="e4m3", dim=1024, n_routed=64, n_groups=8,
                     topk_groups=4, topk=8, inter=256, seed=23)
+# skewed routing on the SM-pair path: 8 hot experts get two thirds of the
+# 12,000 assignments, so they run as up to six token tiles each (every weight
+# tile streamed once per token tile)
+MID_SKEW = Workload("mid_skew", BlockShape(dim=1024, n_routed=64, n_groups=8, topk_groups=4,
+                                           topk=8, inter=256), 1500, torch.bfloat16, "bf16", 25,
+                    hot_experts=8, hot_bias=0.5)
+FP8_SKEW = Workload("fp8_skew", BlockShape(dim=1024, n_routed=64, n_groups=8, topk_groups=4,
+                                           topk=8, inter=256), 1500, torch.bfloat16, "e4m3", 26,
+                    hot_experts=8, hot_bias=0.5)
 FP8_CG1 = custom("fp8_cg1", 230, w_format="e4m3", dim=384, n_routed=16, n_groups=4,
                  topk_groups=2, topk=4, inter=128, seed=24)
 
@@ -166,7 +176,7 @@ def test_experts_rows_match_oracle(w):
 @pytest.mark.parametrize("combine", ["scatter", "ordered"])
 @pytest.mark.parametrize("w", [WORKLOADS["tiny_f32"], TINY_BF16, MID, MID_F32, SOFTMAX_NOBIAS,
                                ONE_GROUP, DECODE_SMALL, ONE_TOKEN, CG1_PREFILL, FP8_SMALL,
-                               FP8_DECODE, FP8_CG1],
+                               FP8_DECODE, FP8_CG1, MID_SKEW, FP8_SKEW],
                          ids=lambda w: w.name)
 def test_block_matches_oracle(w, combine):
     x, p = make_block(w)
@@ -178,6 +188,9 @@ def test_block_matches_oracle(w, combine):
     tokens = np.nonzero(rep.same_set)[0]
     y_orc = oracle_y(w, x, p, r, tokens=tokens)
     y_close(y.cpu().numpy()[tokens], y_orc, TOL[w.w_format])
+    if w.hot_experts:  # the skew did what it is for
+        c = blk.counts.cpu().numpy()
+        assert c.max() > 2 * 256
     # counts agree with the oracle's bincount unless a near-tie flipped
     if rep.set_flips == 0:
         d = O.dispatch(r.indices, w.shape.n_routed)
