@@ -7,23 +7,27 @@
 //
 // Tensor-core path (bf16 activations; bf16 or e4m3 weights), sm_100a:
 //   gather_rows   X_perm[p] = x[sorted_token[p]] (expert-contiguous rows),
-//                 followed by the T rows of x for the shared expert.
-//   GEMM1         h = silu(X W1^T) * (X W3^T), bf16 out
-//   GEMM2         o = h W2^T, fp32 out
+//                 followed by the T rows of x for the shared expert
+//                 (gather_rows_f16 converts them to fp16 for e4m3 weights).
+//   GEMM1         h = silu(X W1^T) * (X W3^T), bf16 out (fp16 with e4m3)
+//   GEMM2         o = h W2^T, fp32 out, or gate * o added into y
 // Both GEMMs are one persistent, warp-specialised kernel template
 // (tc_expert_gemm): warp 0 issues TMA loads into a shared-memory ring, one
-// thread of warp 1 issues tcgen05.mma into a double-buffered TMEM
-// accumulator, warps 2-5 drain the accumulator with tcgen05.ld and run the
-// epilogue while the next tile's MMAs proceed.
+// thread of warp 1 issues tcgen05.mma into TMEM, four or eight epilogue
+// warps drain TMEM with tcgen05.ld, and with e4m3 weights eight converter
+// warps expand each code tile into the fp16 tile the MMA reads.
 //
 // The operands are swapped relative to the usual token-major GEMM: the 128
-// rows of an MMA (M) are weight rows and the MMA's N is the expert's tokens.
-// N is a run-time field of the instruction descriptor, so a tile spends MMA
-// work only on the tokens its expert really has (rounded up to 16) -- from 1
-// token per expert at decode to 256 at prefill -- and each weight byte is
-// streamed from HBM once per token tile.  For GEMM1 a 128-row A tile holds 64
-// rows of W1 and the same 64 rows of W3, so one accumulator carries both
-// halves of the SwiGLU; the epilogue pairs the warps that hold them.
+// rows of an MMA (M) per SM are weight rows and the MMA's N is the expert's
+// tokens.  N is a run-time field of the instruction descriptor, so a tile
+// spends MMA work only on the tokens its expert really has (rounded up to
+// 16) -- from 1 token per expert at decode to 256 at prefill -- and each
+// weight byte is streamed from HBM once per token tile.  Prefill tiles run on
+// SM pairs (cta_group::2, M = 256).  In the first matmul each SM of a pair
+// holds 128 rows of W1 and the same 128 rows of W3 in two accumulators (AT =
+// 2), so a thread holds both SwiGLU halves of its feature; at decode a
+// 128-row tile holds 64 rows of each and the epilogue pairs the warps that
+// hold them (AT = 1).
 //
 // CUDA-core path: any other dtype combination (the fp32 configuration) runs
 // on simt_gemm1 / simt_gemm2 in fp32.
@@ -176,10 +180,11 @@ __global__ void __launch_bounds__(256) gather_rows_f16(const __nv_bfloat162 *__r
 namespace tc {
 
 constexpr int BK = 64;                 // K elements per ring stage (128 bytes bf16)
-constexpr int BM = 128;                // MMA M: weight rows per tile
+constexpr int BM = 128;                // MMA M per SM: weight rows of one weight tile
 constexpr int A_BYTES = BM * BK * 2;   // 16 KB
-// warp 0 issues TMA loads, warp 1 MMAs, warps 2-5 run the epilogue; with e4m3
-// weights, warps 6 .. 6 + CONV_WARPS - 1 expand the weight tiles
+// warp 0 issues TMA loads, warp 1 MMAs, warps 2 .. 1 + epi_warps(AT) run the
+// epilogue; with e4m3 weights the CONV_WARPS warps after them expand the
+// weight tiles
 #ifndef MOE_TC_CONV_WARPS
 #define MOE_TC_CONV_WARPS 8
 #endif
