@@ -247,15 +247,17 @@ class MoEBlock:
 
     # kernels one forward launches: router 3 (bf16 x on the tensor-core path:
     # weight split, scores, selection) or 2, dispatch 3, experts 5 on the
-    # tensor-core path (two tile tables, row gather, two GEMMs) or 4, then
-    # combine 1 (ordered) or nothing (scatter; y is zeroed by a memset node)
+    # tensor-core path, with bf16 or e4m3 weights (two tile tables, row
+    # gather, two GEMMs) or 4 on the CUDA-core path, then combine 1 (ordered)
+    # or nothing (scatter; y is zeroed by a memset node)
     @property
     def launches_per_forward(self) -> int:
         sh = self.shape
         tc_router = (self.x_dtype == torch.bfloat16 and sh.n_routed % 128 == 0
                      and sh.dim % 64 == 0 and self.T >= 32)
-        tc_experts = (self.x_dtype == torch.bfloat16 and self.p.w1.dtype == torch.bfloat16
-                      and sh.dim % 128 == 0 and sh.inter % 128 == 0)
+        tc_experts = (self.x_dtype == torch.bfloat16 and sh.dim % 128 == 0
+                      and sh.inter % 128 == 0
+                      and self.p.w1.dtype in (torch.bfloat16, torch.uint8, torch.float8_e4m3fn))
         return ((3 if tc_router else 2) + 3 + (5 if tc_experts else 4)
                 + (1 if self.combine_mode == "ordered" else 0))
 
