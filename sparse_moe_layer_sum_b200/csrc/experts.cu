@@ -564,18 +564,42 @@ __global__ void __launch_bounds__(threads_of(F8, AT), 1)
           const uint32_t s1 = L::NPARTS == 2 ? f16x2_splat(c1 * F8_SCALE_UP) : s0;
           const uint8_t *a8 = sm + stage * L::STAGE_BYTES + L::A8_OFF;
           uint8_t *a16 = sm + stage * L::STAGE_BYTES;
+          if (AT == 2) {
+            // two weight tiles per stage: each step turns 16 codes (one
+            // 16-byte load) into two 16-byte chunks (2c, 2c + 1) of the row
+#pragma unroll
+            for (int it = 0; it < AT * BM * 4 / (32 * CONV_WARPS); ++it) {
+              const int idx = ct + it * 32 * CONV_WARPS;
+              const int r = idx >> 2, c = idx & 3;  // rows of all parts lie back to back
+              const uint32_t sc = r >= L::PART_ROWS ? s1 : s0;
+              const uint4 q = *reinterpret_cast<const uint4 *>(a8 + r * 64 + c * 16);
+              uint4 o0, o1;
+              o0.x = f16x2_mul(e4m3x2_to_f16x2((uint16_t)(q.x & 0xffffu)), sc);
+              o0.y = f16x2_mul(e4m3x2_to_f16x2((uint16_t)(q.x >> 16)), sc);
+              o0.z = f16x2_mul(e4m3x2_to_f16x2((uint16_t)(q.y & 0xffffu)), sc);
+              o0.w = f16x2_mul(e4m3x2_to_f16x2((uint16_t)(q.y >> 16)), sc);
+              o1.x = f16x2_mul(e4m3x2_to_f16x2((uint16_t)(q.z & 0xffffu)), sc);
+              o1.y = f16x2_mul(e4m3x2_to_f16x2((uint16_t)(q.z >> 16)), sc);
+              o1.z = f16x2_mul(e4m3x2_to_f16x2((uint16_t)(q.w & 0xffffu)), sc);
+              o1.w = f16x2_mul(e4m3x2_to_f16x2((uint16_t)(q.w >> 16)), sc);
+              *reinterpret_cast<uint4 *>(a16 + r * 128 + (((2 * c) ^ (r & 7)) << 4)) = o0;
+              *reinterpret_cast<uint4 *>(a16 + r * 128 + (((2 * c + 1) ^ (r & 7)) << 4)) = o1;
+            }
+          } else {
+            // one tile: 8 codes (one 8-byte load) per 16-byte chunk c
 #pragma unroll 4
-          for (int it = 0; it < AT * BM * 8 / (32 * CONV_WARPS); ++it) {
-            const int idx = ct + it * 32 * CONV_WARPS;
-            const int r = idx >> 3, c = idx & 7;  // rows of all parts lie back to back
-            const uint32_t sc = r >= L::PART_ROWS ? s1 : s0;
-            const uint2 q = *reinterpret_cast<const uint2 *>(a8 + r * 64 + c * 8);
-            uint4 o;
-            o.x = f16x2_mul(e4m3x2_to_f16x2((uint16_t)(q.x & 0xffffu)), sc);
-            o.y = f16x2_mul(e4m3x2_to_f16x2((uint16_t)(q.x >> 16)), sc);
-            o.z = f16x2_mul(e4m3x2_to_f16x2((uint16_t)(q.y & 0xffffu)), sc);
-            o.w = f16x2_mul(e4m3x2_to_f16x2((uint16_t)(q.y >> 16)), sc);
-            *reinterpret_cast<uint4 *>(a16 + r * 128 + ((c ^ (r & 7)) << 4)) = o;
+            for (int it = 0; it < AT * BM * 8 / (32 * CONV_WARPS); ++it) {
+              const int idx = ct + it * 32 * CONV_WARPS;
+              const int r = idx >> 3, c = idx & 7;
+              const uint32_t sc = r >= L::PART_ROWS ? s1 : s0;
+              const uint2 q = *reinterpret_cast<const uint2 *>(a8 + r * 64 + c * 8);
+              uint4 o;
+              o.x = f16x2_mul(e4m3x2_to_f16x2((uint16_t)(q.x & 0xffffu)), sc);
+              o.y = f16x2_mul(e4m3x2_to_f16x2((uint16_t)(q.x >> 16)), sc);
+              o.z = f16x2_mul(e4m3x2_to_f16x2((uint16_t)(q.y & 0xffffu)), sc);
+              o.w = f16x2_mul(e4m3x2_to_f16x2((uint16_t)(q.y >> 16)), sc);
+              *reinterpret_cast<uint4 *>(a16 + r * 128 + ((c ^ (r & 7)) << 4)) = o;
+            }
           }
           fence_proxy_async_smem();
           __syncwarp();
