@@ -79,20 +79,6 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
   return ok != 0;
 }
 
-// try_wait with acquire at cluster scope: for phases completed by arrivals
-// from the other CTA of a pair that publish its shared-memory writes.
-__device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t *bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred P1;\n\t"
-      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 P1, [%1], %2;\n\t"
-      "selp.b32 %0, 1, 0, P1;\n\t}"
-      : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-
 // Makes this thread's generic-proxy shared-memory writes visible to the async
 // proxy (TMA, tensor cores) before it signals their consumer.
 __device__ __forceinline__ void fence_proxy_async_smem() {
@@ -104,11 +90,10 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
 // MOE_ERR_TIMEOUT) when the limit expires, or false at once when another
 // role has already raised *abort.  Every pipeline wait goes through here, so
 // a stalled pipeline ends with an error status instead of a hung GPU.
-template <bool CLUSTER = false>
 __device__ __forceinline__ bool wait_bounded(uint64_t *bar, uint32_t parity,
                                              volatile int *abort, int64_t limit_ns,
                                              int32_t *status) {
-  auto test = [&]() { return CLUSTER ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity); };
+  auto test = [&]() { return mbar_try_wait(bar, parity); };
   if (test()) return true;
   const uint64_t t0 = globaltimer_ns();
   for (uint32_t it = 1;; ++it) {
@@ -337,31 +322,6 @@ __device__ __forceinline__ void tma_load_2d_pair(const CUtensorMap *m, void *dst
       "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
       ".L2::cache_hint [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(smem_u32(dst)),
       "l"(reinterpret_cast<uint64_t>(m)), "r"(x), "r"(y), "r"(mbar_cluster_addr), "l"(policy)
-      : "memory");
-}
-
-// Four rows (row0..row3, each one 128-byte box) of a 2-D tensor into
-// consecutive 128-byte rows of shared memory: the rows are gathered by index.
-__device__ __forceinline__ void tma_gather4(const CUtensorMap *m, void *dst, uint64_t *bar,
-                                            int32_t x, int4 rows, uint64_t policy) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
-      ".L2::cache_hint [%0], [%1, {%2, %3, %4, %5, %6}], [%7], %8;" ::"r"(smem_u32(dst)),
-      "l"(reinterpret_cast<uint64_t>(m)), "r"(x), "r"(rows.x), "r"(rows.y), "r"(rows.z),
-      "r"(rows.w), "r"(smem_u32(bar)), "l"(policy)
-      : "memory");
-}
-
-// Same, counted on an mbarrier of either CTA of the pair.
-__device__ __forceinline__ void tma_gather4_pair(const CUtensorMap *m, void *dst,
-                                                 uint32_t mbar_cluster_addr, int32_t x, int4 rows,
-                                                 uint64_t policy) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.tile::gather4.mbarrier::"
-      "complete_tx::bytes.L2::cache_hint [%0], [%1, {%2, %3, %4, %5, %6}], [%7], %8;" ::"r"(
-          smem_u32(dst)),
-      "l"(reinterpret_cast<uint64_t>(m)), "r"(x), "r"(rows.x), "r"(rows.y), "r"(rows.z),
-      "r"(rows.w), "r"(mbar_cluster_addr), "l"(policy)
       : "memory");
 }
 
