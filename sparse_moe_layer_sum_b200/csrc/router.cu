@@ -6,10 +6,15 @@
 // sum_j s_j over the chosen experts -- the four equations under "All 4 steps"
 // and the gate-forward code excerpt under "Code".
 //
-// Two kernels:
-//  1. router_scores: z = x W_r^T in fp32 on the CUDA cores (tiled, with a
-//     deterministic split over dim when there are too few token tiles to
-//     fill the GPU).  fp32 inputs and fp32 FMA: the excerpt scores in fp32.
+// The scores z = x W_r^T are fp32-accurate either way:
+//  1a. bf16 x (T >= 32, experts a multiple of 128, dim of 64), on the tensor
+//      cores: split_w3 writes W_r as three bf16 terms whose sum is W_r
+//      exactly; router_scores_tc multiplies x by all three with tcgen05 MMAs
+//      (exact products) and adds each k-block's partial into fp32 registers,
+//      with a deterministic split over dim when there are too few tiles to
+//      fill the GPU.
+//  1b. otherwise router_scores, tiled fp32 FMA on the CUDA cores with the
+//      same kind of split.  The excerpt scores in fp32.
 //  2. router_select: one warp per token; sums the split partials in a fixed
 //     order, applies sigmoid/softmax and the bias, picks groups and experts
 //     with warp-shuffle arg-max rounds and writes gates, indices and the
