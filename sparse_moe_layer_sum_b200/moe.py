@@ -3,8 +3,13 @@
 Argument marshalling only: every step of the block runs in the CUDA kernels
 of the four C-ABI libraries; PyTorch provides device memory and the stream.
 
-    block = MoEBlock(shape, params)        # weights already on the GPU
-    y = block.forward(x)                   # x [T, dim] on the GPU -> y fp32
+    block = MoEBlock(shape, params, T, torch.bfloat16)   # weights already on the GPU
+    y = block.forward(x)                   # x [T, dim] on the GPU -> y [T, dim] fp32
+
+    pipe = block.host_pipeline()           # end to end from pinned host memory,
+    for xh, yh in batches:                 # copies overlapped with compute
+        pipe.submit(xh, yh)
+    pipe.finish()                          # then synchronise the stream
 """
 from __future__ import annotations
 
