@@ -125,6 +125,10 @@ def test_experts_validation():
               None) == INVALID
     assert fc(ctypes.byref(c), 8, P, 1, ctypes.byref(w), P, P, P, P, P, P, 8, None,
               None) == WORKSPACE
+    # empty batch: validated, then nothing to launch
+    assert f(ctypes.byref(c), 0, P, 1, ctypes.byref(w), P, P, P, P, P, 1 << 40, None, None) == 0
+    assert fc(ctypes.byref(c), 0, P, 1, ctypes.byref(w), P, P, P, P, P, P, 1 << 40, None,
+              None) == 0
 
 
 def test_combine_and_selftest_validation():
