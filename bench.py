@@ -29,10 +29,14 @@ sys.path.insert(0, ROOT)
 
 from sparse_moe_layer_sum_b200 import moe  # noqa: E402
 from sparse_moe_layer_sum_b200.inputs import WORKLOADS, make_block, sample_tokens  # noqa: E402
-from sparse_moe_layer_sum_b200.roofline import block_work, kernel_work, load_peaks  # noqa: E402
+from sparse_moe_layer_sum_b200.roofline import (block_work, kernel_work, load_peaks,  # noqa: E402
+                                                 method_bytes, tensor_peak)
 
 METRIC = "MoE block tokens/s (V3 shape, bf16, T=4096) and % of roofline on 1 B200"
 N_X_BATCHES = 4  # rotating input batches: with the 22.6 GB of weights, > L2 per step
+# the other configurations timed in short loops after the headline one:
+# (workload, FP8 x FP8 activations)
+OTHER_CONFIGS = [("v3_decode_t64", False), ("v3_skew_t16384", False), ("v3_fp8_t8192", False)]
 
 
 def parse():
@@ -47,6 +51,11 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-graph", action="store_true",
                     help="skip the CUDA-graph replay timing of the same forward")
+    ap.add_argument("--other-steps", type=int, default=20,
+                    help="timed steps for each other configuration (0: skip them)")
+    ap.add_argument("--fp8-act", action="store_true",
+                    help="e4m3-weight workloads: quantise the activations to e4m3 too "
+                         "(FP8 x FP8 matmuls)")
     ap.add_argument("--combine", choices=["scatter", "ordered"], default="scatter",
                     help="weighted sum into y inside the second matmul, or ordered and "
                          "bit-reproducible in a separate pass")
@@ -133,7 +142,7 @@ class ClockSampler:
 # ---------------------------------------------------------------- oracle leg
 
 
-def cpu_oracle_tokens_per_s(w, x, params, n_tokens: int, seed: int = 7):
+def cpu_oracle_tokens_per_s(w, x, params, n_tokens: int, seed: int = 7, fp8_act=False):
     """Time the oracle (as it stands) on a seeded sample of the workload's
     tokens: routing and the block output of each sampled token.  Host copies
     of the expert weights are fetched outside the timed part."""
@@ -163,7 +172,9 @@ def cpu_oracle_tokens_per_s(w, x, params, n_tokens: int, seed: int = 7):
         fetch_s += time.perf_counter() - t0
         return mats
 
-    act = "bf16" if w.x_dtype == torch.bfloat16 else "f32"
+    # h rounded as the CUDA path rounds it (the oracle's readings 3 and 6)
+    act = ("f32" if w.x_dtype == torch.float32 else
+           ("e4m3" if fp8_act else "f16") if w.w_format == "e4m3" else "bf16")
     t0 = time.perf_counter()
     route = O.router(xs, w_r, bias, shape)
     O.moe_forward(xs, route, fetch, lambda: fetch(shape.n_routed_experts),
@@ -198,35 +209,43 @@ def traffic_for(kernel_name: str):
     return entry.get("dram_bytes_per_launch")
 
 
-def run_ours(args, rank, local_rank, world):
-    torch.cuda.set_device(local_rank)
-    dev = torch.device("cuda", local_rank)
-    from sparse_moe_layer_sum_b200 import build
-    build.build_all()
-    w = WORKLOADS[args.workload]
-    sh = w.shape
+def make_inputs(w, dev, rank):
+    """The block's weights and N_X_BATCHES seeded input batches for this rank."""
     x0, params = make_block(w, dev, x_seed_offset=1 + rank * N_X_BATCHES)
     xs = [x0]
     gx = torch.Generator(device=dev)
     for i in range(1, N_X_BATCHES):
         gx.manual_seed(w.seed + 104729 * (1 + rank * N_X_BATCHES + i))
-        xs.append(torch.randn(w.T, sh.dim, generator=gx, device=dev).to(w.x_dtype))
-    blk = moe.MoEBlock(sh, params, w.T, w.x_dtype, device=dev, combine=args.combine)
+        xs.append(torch.randn(w.T, w.shape.dim, generator=gx, device=dev).to(w.x_dtype))
+    return xs, params
 
-    for i in range(max(args.warmup, 1)):
+
+def mma_type(w, fp8_act: bool) -> str:
+    """Operand type of the expert matmuls: e4m3 weights are expanded to fp16,
+    unless the FP8 x FP8 path quantises the activations too."""
+    if w.w_format == "e4m3":
+        return "e4m3" if fp8_act else "f16"
+    return "bf16" if w.x_dtype == torch.bfloat16 else "f32"
+
+
+def time_block(w, blk, xs, K, warmup, world, dev, local_rank):
+    """Warm up, then time K forwards (max over ranks) with per-kernel events;
+    also the routing of each input batch (counts, near-ties)."""
+    for i in range(max(warmup, 1)):
         blk.forward(xs[i % N_X_BATCHES])
     torch.cuda.synchronize()
     st = blk.device_status()
     if st != 0:
         raise RuntimeError(f"device status {st} after warm-up")
-
-    K = args.steps
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(10)] for _ in range(K)]
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    counts = []
+    counts, ties = [], []
     for i in range(N_X_BATCHES):   # routing of each input batch, for the byte counts
         blk.forward(xs[i])
         counts.append(blk.counts.cpu())
+        # tokens whose smallest routing decision gap (the router's own report)
+        # is below 1e-6: their choice may depend on rounding
+        ties.append(int((blk.sel_gap < 1e-6).sum()))
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()
@@ -243,61 +262,133 @@ def run_ours(args, rank, local_rank, world):
     ms_total = max_over_ranks(start.elapsed_time(end), world, dev)
     if blk.device_status() != 0:
         raise RuntimeError(f"device status {blk.device_status()} in the timed region")
-    ms_step = ms_total / K
-    value = job_tokens_per_s(world, w.T, K, ms_total)
-
-    # per-kernel durations inside the timed region
     spans = {"router": (0, 1), "dispatch": (1, 2), "gather": (3, 4), "gemm1": (4, 5),
              "gemm2": (6, 7), "combine": (8, 9)}
     dur = {k: statistics.mean(evs[i][a].elapsed_time(evs[i][b]) for i in range(K))
            for k, (a, b) in spans.items()}
+    return {"ms_total": ms_total, "ms_step": ms_total / K, "dur": dur, "counts": counts,
+            "near_ties": ties, "clocks": clk}
+
+
+def rooflines(w, blk, K, tm, fp8_act=False):
+    """Dominant-kernel and whole-step rooflines from the measured timings."""
+    sh = w.shape
     peaks, peak_src = load_peaks(ROOT)
     w_bytes = {"bf16": 2, "f32": 4, "e4m3": 1}[w.w_format]
     x_bytes = 2 if w.x_dtype == torch.bfloat16 else 4
     scale_b = (3 * (sh.dim // 128) * (sh.inter // 128) * 4) if w.w_format == "e4m3" else 0
-    touched = [int((c > 0).sum()) for c in counts]
-    kw = [kernel_work(sh.dim, sh.n_routed, sh.inter, sh.topk, sh.n_shared, w.T, n, w_bytes,
-                      x_bytes, scale_b, scatter=blk.combine_mode == "scatter") for n in touched]
-    bw = [block_work(sh.dim, sh.n_routed, sh.inter, sh.topk, sh.n_shared, w.T, n, w_bytes,
-                     x_bytes, scale_b, sh.has_bias) for n in touched]
+    touched = [int((c > 0).sum()) for c in tm["counts"]]
+    args = (sh.dim, sh.n_routed, sh.inter, sh.topk, sh.n_shared, w.T)
+    kw = [kernel_work(*args, n, w_bytes, x_bytes, scale_b, scatter=blk.combine_mode == "scatter")
+          for n in touched]
+    mb = [method_bytes(sh.dim, sh.inter, sh.topk, sh.n_shared, w.T, n, w_bytes, x_bytes, scale_b)
+          for n in touched]
+    bw = [block_work(*args, n, w_bytes, x_bytes, scale_b, sh.has_bias) for n in touched]
     steps_per_batch = [sum(1 for i in range(K) if i % N_X_BATCHES == b) for b in range(N_X_BATCHES)]
 
     def avg(f):
         return sum(f(b) * steps_per_batch[b] for b in range(N_X_BATCHES)) / K
 
+    dur = tm["dur"]
     dominant = max(("gemm1", "gemm2", "router", "combine", "gather", "dispatch"), key=dur.get)
     bytes_dom = avg(lambda b: kw[b][dominant].bytes)
+    bytes_meth = avg(lambda b: mb[b][dominant]) if dominant in ("gemm1", "gemm2") else bytes_dom
     flops_dom = avg(lambda b: kw[b][dominant].flops)
     # tensor peak: the sustained (power-capped) figure when the timed loop runs
     # long enough for the clocks to settle under the power cap, else the burst one
-    sustained = ms_total > 500.0 and "bf16_tflops_sustained" in peaks
+    sustained = tm["ms_total"] > 500.0 and "bf16_tflops_sustained" in peaks
+    mma = mma_type(w, fp8_act)
     hbm = peaks["hbm_gbs"]
-    tflops = peaks["bf16_tflops_sustained"] if sustained else peaks["bf16_tflops"]
-    t_hbm = bytes_dom / (hbm * 1e9)
-    t_tc = flops_dom / (tflops * 1e12)
+    tflops = tensor_peak(peaks, sustained, mma)
     dsec = dur[dominant] / 1e3
     kname = {"gemm1": "tc_expert_gemm<1>",
              "gemm2": "tc_expert_gemm<3>" if blk.combine_mode == "scatter" else "tc_expert_gemm<2>"
              }.get(dominant, dominant)
-    if t_hbm >= t_tc:
-        roof = {"bound": "hbm", "achieved": bytes_dom / dsec / 1e9, "peak": hbm, "unit": "GB/s"}
+    if bytes_meth / (hbm * 1e9) >= flops_dom / (tflops * 1e12):
+        roof = {"bound": "hbm", "achieved": bytes_meth / dsec / 1e9, "peak": hbm, "unit": "GB/s"}
+        roof["frac"] = roof["achieved"] / hbm
+        roof["frac_method"] = roof["frac"]
+        roof["frac_impl"] = bytes_dom / dsec / 1e9 / hbm
     else:
         roof = {"bound": "tensor", "achieved": flops_dom / dsec / 1e12, "peak": tflops,
                 "unit": "TFLOP/s"}
-    roof["frac"] = roof["achieved"] / roof["peak"]
+        roof["frac"] = roof["frac_method"] = roof["frac_impl"] = roof["achieved"] / tflops
     roof["traffic"] = traffic_for(kname)
     roof["kernel"] = kname
+    roof["scope"] = "dominant kernel (the whole step is step_roofline)"
+    roof["mma_type"] = mma
     roof["peak_source"] = (f"{peak_src} ({'MEASURED_PEAKS.json' if peak_src == 'measured' else 'recipe fallback'}"
-                           f"{', tensor peak sustained' if sustained else ', tensor peak burst'})")
-    roof["algorithmic_bytes_per_launch"] = bytes_dom
+                           f"{', tensor peak sustained' if sustained else ', tensor peak burst'}"
+                           f"{', e4m3 = 2 x bf16 (nominal ratio)' if mma == 'e4m3' else ''})")
+    roof["method_bytes_per_launch"] = bytes_meth
+    roof["impl_bytes_per_launch"] = bytes_dom
     roof["algorithmic_flops_per_launch"] = flops_dom
     b_alg = avg(lambda b: bw[b].bytes)
     f_alg = avg(lambda b: bw[b].flops)
+    ms_step = tm["ms_step"]
     t_roof = max(b_alg / (hbm * 1e9), f_alg / (tflops * 1e12))
     step_roof = {"bytes": b_alg, "flops": f_alg, "t_roof_ms": t_roof * 1e3,
                  "frac": t_roof * 1e3 / ms_step,
                  "bound": "hbm" if b_alg / (hbm * 1e9) >= f_alg / (tflops * 1e12) else "tensor",
+                 "tensor_peak_tflops": tflops,
+                 "hbm_frac": b_alg / (ms_step / 1e3) / (hbm * 1e9),
+                 "tensor_frac": f_alg / (ms_step / 1e3) / (tflops * 1e12),
                  "hbm_frac_vs_nominal_8TBs": b_alg / (ms_step / 1e3) / 8e12}
+    if w.w_format == "e4m3" and mma != "e4m3":
+        # the same step against the dense FP8 peak (2 x bf16), which an
+        # FP8 x FP8 matmul could reach
+        fp8 = tensor_peak(peaks, sustained, "e4m3")
+        step_roof["tensor_frac_vs_fp8_peak"] = f_alg / (ms_step / 1e3) / (fp8 * 1e12)
+        step_roof["frac_vs_fp8_peak"] = max(b_alg / (hbm * 1e9), f_alg / (fp8 * 1e12)) / (ms_step / 1e3)
+    return roof, step_roof, touched
+
+
+def near_tie_report(w, tm):
+    n = tm["near_ties"]
+    return {"threshold": 1e-6, "tokens_per_batch": n, "fraction": sum(n) / (len(n) * w.T)}
+
+
+def other_config(name, args, dev, local_rank, fp8_act=False):
+    """A short timed loop of another configuration, for the same JSON line."""
+    w = WORKLOADS[name]
+    xs, params = make_inputs(w, dev, 0)
+    blk = moe.MoEBlock(w.shape, params, w.T, w.x_dtype, device=dev, combine=args.combine,
+                       fp8_act=fp8_act)
+    K = args.other_steps
+    tm = time_block(w, blk, xs, K, 3, 1, dev, local_rank)
+    roof, step_roof, touched = rooflines(w, blk, K, tm, fp8_act)
+    out = {"value": job_tokens_per_s(1, w.T, K, tm["ms_total"]), "unit": "tokens/s",
+           "ms_per_step": tm["ms_step"], "steps": K, "warmup": 3, "T": w.T,
+           "weights": w.w_format, "mma_type": mma_type(w, fp8_act),
+           "step_roofline": step_roof, "roofline": roof, "kernels_ms": tm["dur"],
+           "near_ties": near_tie_report(w, tm), "clocks": tm["clocks"],
+           "touched_experts": touched}
+    if w.hot_experts:
+        hot_ids = torch.randperm(w.shape.n_routed, generator=torch.Generator().manual_seed(2024))[:16]
+        out["hot_share"] = float(tm["counts"][0][hot_ids].sum() / tm["counts"][0].sum())
+    del blk, xs, params
+    torch.cuda.empty_cache()
+    return out
+
+
+def run_ours(args, rank, local_rank, world):
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    from sparse_moe_layer_sum_b200 import build
+    build.build_all()
+    w = WORKLOADS[args.workload]
+    sh = w.shape
+    xs, params = make_inputs(w, dev, rank)
+    x0 = xs[0]
+    blk = moe.MoEBlock(sh, params, w.T, w.x_dtype, device=dev, combine=args.combine,
+                       fp8_act=args.fp8_act)
+    K = args.steps
+    tm = time_block(w, blk, xs, K, args.warmup, world, dev, local_rank)
+    ms_total, ms_step = tm["ms_total"], tm["ms_step"]
+    value = job_tokens_per_s(world, w.T, K, ms_total)
+    roof, step_roof, touched = rooflines(w, blk, K, tm, args.fp8_act)
+    x_bytes = 2 if w.x_dtype == torch.bfloat16 else 4
+    w_bytes = {"bf16": 2, "f32": 4, "e4m3": 1}[w.w_format]
 
     # end to end through the public API from pinned host memory: every step
     # copies its batch in and its y out, overlapped with the neighbouring
@@ -363,7 +454,8 @@ def run_ours(args, rank, local_rank, world):
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         try:
-            tps, cores, wall = cpu_oracle_tokens_per_s(w, x0, params, args.cpu_sample)
+            tps, cores, wall = cpu_oracle_tokens_per_s(w, x0, params, args.cpu_sample,
+                                                       fp8_act=args.fp8_act)
             cpu = {"value": tps, "unit": "tokens/s", "cores": cores, "kind": "oracle",
                    "sample": f"{args.cpu_sample} seeded tokens of the {w.name} batch: fp64 "
                              f"routing and block output ({wall:.1f} s of oracle time; weight "
@@ -374,25 +466,47 @@ def run_ours(args, rank, local_rank, world):
     hot = None
     if w.hot_experts:
         hot_ids = torch.randperm(sh.n_routed, generator=torch.Generator().manual_seed(2024))[:16]
-        hot = float(counts[0][hot_ids].sum() / counts[0].sum())
+        hot = float(tm["counts"][0][hot_ids].sum() / tm["counts"][0].sum())
+    launches = K * blk.launches_per_forward
+
+    # the other configurations, each in a short loop of its own (one GPU only)
+    others = None
+    if world == 1 and args.other_steps > 0:
+        del blk, xs, params, x_host, y_host, pipe
+        torch.cuda.empty_cache()
+        others = {}
+        for name, fp8 in OTHER_CONFIGS:
+            if name == w.name and fp8 == args.fp8_act:
+                continue
+            key = name + ("_fp8act" if fp8 else "")
+            try:
+                others[key] = other_config(name, args, dev, local_rank, fp8)
+            except Exception as exc:  # reported, never fatal to the headline
+                others[key] = {"error": repr(exc)[:300]}
+
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None,
         # arithmetic type of the matmuls: e4m3 weights are expanded to f16
-        "dtype": {"bf16": "bf16", "f32": "f32", "e4m3": "f16"}[w.w_format],
+        # unless the activations are quantised to e4m3 as well
+        "dtype": mma_type(w, args.fp8_act),
         "data": "synthetic (seeded N(0,1) activations, N(0,1/fan_in) weights, U(-0.1,0.1) bias)",
         "config": {"workload": w.name, "T": w.T, "dim": sh.dim, "n_routed": sh.n_routed,
-                   "combine": blk.combine_mode,
+                   "combine": args.combine,
                    "topk": sh.topk, "inter": sh.inter, "weights": w.w_format,
+                   "activations": "e4m3 (1x128 blocks)" if args.fp8_act else
+                   ("bf16" if w.x_dtype == torch.bfloat16 else "f32"),
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                    "l2": f"inputs larger than L2: {N_X_BATCHES} rotating x batches and "
                          f"{(sh.n_routed + 1) * 3 * sh.dim * sh.inter * w_bytes / 1e9:.1f} GB "
                          "of expert weights per step"},
         "roofline": roof, "step_roofline": step_roof,
-        "kernels_ms": dur, "cpu_baseline": cpu, "e2e": e2e, "graph": graph,
-        "gpu_launches": K * blk.launches_per_forward,
-        "clocks": clk, "touched_experts": touched, "hot_share": hot,
+        "kernels_ms": tm["dur"], "cpu_baseline": cpu, "e2e": e2e, "graph": graph,
+        "gpu_launches": launches,
+        "clocks": tm["clocks"], "touched_experts": touched, "hot_share": hot,
+        "near_ties": near_tie_report(w, tm),
+        "other_configs": others,
     }
     if rank == 0:
         print(json.dumps(line), flush=True)

@@ -52,8 +52,10 @@ moe_status moe_dispatch_build(const moe_cfg *cfg, int64_t T, const int32_t *indi
  * ceil(T / 64) * n_routed <= 262144 (for example T up to 65536 tokens with
  * 256 experts); larger calls return MOE_ERR_WORKSPACE and launch nothing.
  * The first call on a device looks up the array's device address with that
- * device current (and caches it), so make that first call before any stream
- * capture.  This entry point allocates and frees no memory.  All calls share
+ * device current (and caches it, together with the id of the context it
+ * belongs to; a later call in a new context of that device, for instance
+ * after cudaDeviceReset, looks it up again), so make the first call in each
+ * context before any stream capture.  This entry point allocates and frees no memory.  All calls share
  * the one array: calls that may overlap on the GPU (other streams, other
  * threads) race on it and must be serialised by the caller.  Outputs,
  * limits and errors are those of moe_dispatch_build.

@@ -35,14 +35,28 @@ extern "C" {
  *   s1, s3  [n_routed + n_shared, inter/128, dim/128] fp32 (MOE_E4M3 only)
  *   s2      [n_routed + n_shared, dim/128, inter/128] fp32 (MOE_E4M3 only)
  * For MOE_E4M3 the weight is value(q) * scale of its 128 x 128 block.
+ *   act_e4m3  0: the matmuls take bf16 activations (e4m3 weights are
+ *             expanded to fp16 on the fly, fp16 x fp16 MMAs).
+ *             1 (MOE_E4M3 weights only): FP8 x FP8 -- the expert rows of x
+ *             and the hidden h (after its bf16 rounding) are quantised to
+ *             e4m3 in 1 x 128 blocks along the reduction dimension, each
+ *             block with fp32 scale = block amax / 448 (the weights' rule;
+ *             an all-zero block has scale 0), and the matmuls run as
+ *             e4m3 x e4m3 tensor-core MMAs whose per-block partial sums are
+ *             scaled by weight scale x activation scale in fp32.  The pages
+ *             name FP8 experts but no activation format; this path trades
+ *             about 5% rms of extra error for twice the tensor throughput.
+ *             Needs dim % 256 == 0 and inter % 128 == 0.
  */
 typedef struct {
   const void *w1, *w3, *w2;
   moe_dtype w_dt;
   const float *s1, *s3, *s2;
+  int32_t act_e4m3;
 } moe_expert_weights;
 
-/* Bytes of device workspace moe_experts_forward needs. */
+/* Bytes of device workspace moe_experts_forward needs (for MOE_E4M3 weights,
+ * enough for either activation path). */
 size_t moe_experts_workspace_size(const moe_cfg *cfg, int64_t T, moe_dtype x_dt,
                                   moe_dtype w_dt);
 

@@ -49,6 +49,44 @@ moe_status moe_router_forward(const moe_cfg *cfg, int64_t T, const void *x, moe_
                               int32_t *indices, float *sel_gap, void *ws, size_t ws_bytes,
                               int32_t *dev_status, moe_stream_t stream);
 
+/*
+ * Preparation of the router weight, done once when the weights are loaded.
+ *
+ * On the tensor-core scoring path (bf16 x, T >= 32, n_routed a multiple of
+ * 128, dim a multiple of 64) z = x W_r^T is computed as x hi^T + x mid^T +
+ * x lo^T with three bf16 matrices whose sum is W_r exactly (each holds the
+ * next 8 significant bits of every element; the remainders are exact in
+ * fp32), so every product is exact and z carries only fp32 accumulation
+ * error, as the excerpt's fp32 linear would.  moe_router_forward writes
+ * that split into its workspace on every call; moe_router_prepare writes it
+ * once into a caller-owned buffer, and moe_router_forward_prepared reads it
+ * from there.
+ *
+ * moe_router_prepare_size: bytes of the split (3 * n_routed * dim * 2), or 0
+ * when the tensor-core path cannot apply to cfg (or cfg is invalid).
+ * moe_router_prepare: w_r [n_routed, dim] fp32 -> prep (device, caller-owned,
+ * prep_bytes >= moe_router_prepare_size(cfg)); enqueued on `stream`.
+ * Returns MOE_ERR_UNSUPPORTED when the size is 0, MOE_ERR_WORKSPACE when
+ * prep_bytes is too small, MOE_ERR_INVALID for NULL pointers.  prep must be
+ * prepared again whenever w_r changes.
+ */
+size_t moe_router_prepare_size(const moe_cfg *cfg);
+moe_status moe_router_prepare(const moe_cfg *cfg, const float *w_r, void *prep,
+                              size_t prep_bytes, moe_stream_t stream);
+
+/*
+ * moe_router_forward with the prepared split of w_r: identical results, one
+ * launch fewer.  `prep` (required, from moe_router_prepare on this w_r) is
+ * read when the tensor-core path applies; otherwise the call scores from
+ * w_r exactly as moe_router_forward does.  All other arguments, limits and
+ * errors are those of moe_router_forward (the same workspace size).
+ */
+moe_status moe_router_forward_prepared(const moe_cfg *cfg, int64_t T, const void *x,
+                                       moe_dtype x_dt, const float *w_r, const void *prep,
+                                       const float *bias, float *weights, int32_t *indices,
+                                       float *sel_gap, void *ws, size_t ws_bytes,
+                                       int32_t *dev_status, moe_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

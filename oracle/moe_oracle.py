@@ -41,6 +41,11 @@ Readings of points the pages leave open:
    into an fp64 y that stands in for the excerpt's fp32 accumulator.
 5. FP8 weights: e4m3 codes with one fp32 scale per 128 x 128 block of the
    [out, in] weight matrix; the dequantised weight is fp32(q) * scale.
+6. FP8 activations (the optional FP8 x FP8 path of the FP8-weight
+   configuration; the pages name FP8 experts but no activation format):
+   each row of x, and each row of h after its bf16 rounding, is quantised to
+   e4m3 in 1 x 128 blocks with the weights' rule, scale = block amax / 448,
+   in fp32 arithmetic.
 
 Parity pins for every function live in ``tests/test_oracle_*.py``.
 """
@@ -140,6 +145,86 @@ def e4m3_table() -> np.ndarray:
         else:
             out[code] = sign * (1.0 + man / 8.0) * 2.0 ** (ex - 7)
     return out
+
+
+def round_f32_to_f16(v: np.ndarray) -> np.ndarray:
+    """Round fp32 values to the nearest IEEE binary16 value (ties to even), as fp64.
+
+    binary16 has 10 fraction bits, exponent bias 15 and subnormals below
+    2^-14 with spacing 2^-24.  A finite value v with |v| in [2^e, 2^(e+1))
+    (e >= -14) is a multiple of 2^(e-10) once rounded; below 2^-14 the
+    spacing stays 2^-24.  Magnitudes that round above 65504 are out of range
+    (not used: the callers keep far below it).
+    """
+    v = np.asarray(v, dtype=np.float32).astype(np.float64)
+    mag = np.abs(v)
+    with np.errstate(divide="ignore"):
+        e = np.floor(np.log2(np.where(mag > 0, mag, 1.0)))
+    e = np.maximum(e, -14.0)
+    step = np.exp2(e - 10.0)
+    r = np.rint(v / step) * step          # np.rint rounds halves to even
+    if np.any(np.abs(r) > 65504.0):
+        raise OverflowError("value outside the binary16 range")
+    return r
+
+
+E4M3_MAX = 448.0
+
+
+def round_to_e4m3(v: np.ndarray) -> np.ndarray:
+    """Nearest float8 e4m3 value (ties to even), saturated to +-448, as fp64.
+
+    e4m3 keeps 3 fraction bits with exponent bias 7: a value with |v| in
+    [2^e, 2^(e+1)) (e >= -6) rounds to a multiple of 2^(e-3); below 2^-6 the
+    subnormal spacing is 2^-9.  Magnitudes beyond the largest finite value
+    448 are clamped to it (the "satfinite" conversion).  NaN is not handled.
+    """
+    v = np.asarray(v, dtype=np.float64)
+    mag = np.abs(v)
+    with np.errstate(divide="ignore"):
+        e = np.floor(np.log2(np.where(mag > 0, mag, 1.0)))
+    e = np.maximum(e, -6.0)
+    step = np.exp2(e - 3.0)
+    r = np.rint(v / step) * step
+    return np.clip(r, -E4M3_MAX, E4M3_MAX)
+
+
+def e4m3_code(values: np.ndarray) -> np.ndarray:
+    """The uint8 code of e4m3 values (exact e4m3 values in, e.g. from
+    round_to_e4m3); +0 for zero."""
+    t = e4m3_table()
+    finite = np.nonzero(np.isfinite(t))[0]
+    lut = {float(t[c]): c for c in finite if not (t[c] == 0 and c == 0x80)}
+    return np.vectorize(lambda x: lut[float(x)], otypes=[np.uint8])(np.asarray(values))
+
+
+def quantize_e4m3_rows(v: np.ndarray, block: int = 128):
+    """Per-row 1 x block e4m3 quantisation of activations, fp32 arithmetic.
+
+    For each row and each run of `block` columns: amax = max |v| (exact),
+    scale = fp32(amax / 448) (an IEEE fp32 division), code = the e4m3 value
+    nearest fp32(v / scale) (IEEE fp32 division, ties to even, saturated);
+    an all-zero block has scale 0 and codes 0.  This is the weights' rule
+    (scale = block amax / 448) applied to 1 x 128 blocks of a row.
+    Returns (values [rows, cols] fp64 of the codes, scales [rows, cols/block] fp32);
+    the dequantised activation is values * scale.
+    """
+    v = np.asarray(v, dtype=np.float32)
+    r, c = v.shape
+    vb = v.reshape(r, c // block, block)
+    amax = np.abs(vb).max(axis=-1)
+    scale = (amax / np.float32(E4M3_MAX)).astype(np.float32)
+    safe = np.where(scale > 0, scale, np.float32(1.0)).astype(np.float32)
+    q = (vb / safe[:, :, None]).astype(np.float32)        # fp32 division
+    vals = round_to_e4m3(q.astype(np.float64))
+    vals = np.where(scale[:, :, None] > 0, vals, 0.0)
+    return vals.reshape(r, c), scale
+
+
+def dequant_e4m3_rows(vals: np.ndarray, scales: np.ndarray, block: int = 128) -> np.ndarray:
+    """fp64 activation from the e4m3 values and per-row 1 x block scales."""
+    s = np.repeat(np.asarray(scales, dtype=np.float64), block, axis=-1)
+    return np.asarray(vals, dtype=np.float64) * s
 
 
 def dequant_e4m3_block(q_codes: np.ndarray, scales: np.ndarray, block: int = 128) -> np.ndarray:
@@ -289,18 +374,27 @@ def expert_ffn(x_rows: np.ndarray, w1: np.ndarray, w3: np.ndarray, w2: np.ndarra
     """One expert on a set of rows: w2(silu(w1 x) * w3 x) (reading 1).
 
     x_rows [n, D]; w1, w3 [I, D]; w2 [D, I] in the nn.Linear [out, in] layout.
-    The hidden activation h is rounded to ``act_dtype`` ("bf16" or "f32")
-    once, through fp32 (reading 3).  Returns fp64 [n, D].
+    The hidden activation h is rounded once, through fp32, to the type of
+    the second matmul's operand (reading 3): ``act_dtype`` "bf16", "f16" or
+    "f32".  "e4m3" (reading 6): the rows of x and the bf16-rounded h are
+    each quantised to e4m3 in 1 x 128 blocks (quantize_e4m3_rows) and the
+    matmuls take the dequantised values.  Returns fp64 [n, D].
     """
     x64 = np.asarray(x_rows, dtype=np.float64)
+    if act_dtype == "e4m3":
+        x64 = dequant_e4m3_rows(*quantize_e4m3_rows(x64.astype(np.float32)))
     a = x64 @ np.asarray(w1, dtype=np.float64).T
     u = x64 @ np.asarray(w3, dtype=np.float64).T
     h = (silu(a) * u).astype(np.float32)
     if act_dtype == "bf16":
         h = round_f32_to_bf16(h)
+    elif act_dtype == "f16":
+        h = round_f32_to_f16(h)
+    elif act_dtype == "e4m3":
+        h = dequant_e4m3_rows(*quantize_e4m3_rows(round_f32_to_bf16(h)))
     elif act_dtype != "f32":
         raise ValueError(act_dtype)
-    return h.astype(np.float64) @ np.asarray(w2, dtype=np.float64).T
+    return np.asarray(h, dtype=np.float64) @ np.asarray(w2, dtype=np.float64).T
 
 
 # expert weights are fetched lazily so that callers can keep large weight

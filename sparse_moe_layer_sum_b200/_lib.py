@@ -34,6 +34,7 @@ class MoEExpertWeights(ctypes.Structure):
         ("w1", ctypes.c_void_p), ("w3", ctypes.c_void_p), ("w2", ctypes.c_void_p),
         ("w_dt", ctypes.c_int32),
         ("s1", ctypes.c_void_p), ("s3", ctypes.c_void_p), ("s2", ctypes.c_void_p),
+        ("act_e4m3", ctypes.c_int32),
     ]
 
 
@@ -45,6 +46,10 @@ SIGNATURES = {
     ("moe_router", "moe_router_workspace_size"): (_sz, [_cfgp, _i64]),
     ("moe_router", "moe_router_forward"): (
         _i32, [_cfgp, _i64, _vp, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp, _vp]),
+    ("moe_router", "moe_router_prepare_size"): (_sz, [_cfgp]),
+    ("moe_router", "moe_router_prepare"): (_i32, [_cfgp, _vp, _vp, _sz, _vp]),
+    ("moe_router", "moe_router_forward_prepared"): (
+        _i32, [_cfgp, _i64, _vp, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp, _vp]),
     ("moe_dispatch", "moe_dispatch_workspace_size"): (_sz, [_cfgp, _i64]),
     ("moe_dispatch", "moe_dispatch_build"): (
         _i32, [_cfgp, _i64, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp, _vp]),

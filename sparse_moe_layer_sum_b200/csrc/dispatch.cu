@@ -14,6 +14,9 @@
 //                       time; lanes holding the same expert rank themselves
 //                       with __match_any_sync, so the order inside an expert
 //                       is the pair order (token ascending) -- deterministic.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
 #include <mutex>
 
 #include "common.cuh"
@@ -135,19 +138,51 @@ __device__ __align__(256) int32_t g_noalloc_scratch[NOALLOC_SCRATCH_INTS];
 
 constexpr int MAX_DEVICES = 64;
 std::mutex g_noalloc_mu;
+// per device: the scratch array's device address and the id of the context
+// it was looked up in (a context that is destroyed and created again, as
+// after cudaDeviceReset, loads the module anew, possibly elsewhere)
 int32_t *g_noalloc_ptr[MAX_DEVICES] = {};
+unsigned long long g_noalloc_ctx[MAX_DEVICES] = {};
+
+// Unique id of the current context (0 when the driver cannot tell).
+unsigned long long current_ctx_id() {
+  static PFN_cuCtxGetCurrent_v4000 get_ctx = nullptr;
+  static PFN_cuCtxGetId_v12000 get_id = nullptr;
+  static bool looked = false;
+  if (!looked) {
+    looked = true;
+    void *f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_ctx = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(f);
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<PFN_cuCtxGetId_v12000>(f);
+  }
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (!get_ctx || !get_id || get_ctx(&ctx) != CUDA_SUCCESS || !ctx ||
+      get_id(ctx, &id) != CUDA_SUCCESS)
+    return 0;
+  return id;
+}
 
 // Device address of the scratch array on the current device.  In host code the
 // array's name only stands for a host-side symbol, so the address is looked up
-// once per device (with that device current) and cached.
+// (with the device current) on the first call in each context and cached.
 moe_status noalloc_scratch(int32_t **out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= MAX_DEVICES) return MOE_ERR_CUDA;
   std::lock_guard<std::mutex> lock(g_noalloc_mu);
-  if (!g_noalloc_ptr[dev]) {
+  // no current context yet (id 0): the look-up below makes the runtime's
+  // primary context current, and the id is read again after it
+  const unsigned long long ctx = current_ctx_id();
+  if (!g_noalloc_ptr[dev] || ctx == 0 || ctx != g_noalloc_ctx[dev]) {
     void *ptr = nullptr;
     if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || !ptr) return MOE_ERR_CUDA;
     g_noalloc_ptr[dev] = static_cast<int32_t *>(ptr);
+    g_noalloc_ctx[dev] = current_ctx_id();
   }
   *out = g_noalloc_ptr[dev];
   return MOE_OK;

@@ -106,7 +106,7 @@ __global__ void __launch_bounds__(32) prep_tiles(const int32_t *__restrict__ off
 }
 
 struct Tile {
-  int g, ft, tt, n0, nvalid, rowbase;
+  int g, ft, tt, ntt, n0, nvalid, rowbase;
 };
 
 // First k-block of a tile.  Tiles that run at the same time share operands
@@ -137,6 +137,7 @@ __device__ __forceinline__ Tile decode_tile(int tile, const int32_t *tstart, con
   const int local = tile - tstart[lo];
   t.ft = local / ntt;
   t.tt = local - t.ft * ntt;
+  t.ntt = ntt;
   t.n0 = t.tt * base;
   t.nvalid = min(base, n - t.n0);
   t.rowbase = lo < E ? off[lo] : rows_routed + (lo - E) * T;
@@ -376,17 +377,20 @@ __global__ void __launch_bounds__(threads_of(F8, AT), 1)
   if (warp == 0) {
     if (lane == 0) {
       // ---------------------------------------------------- TMA producer
-      // weights: the first matmul keeps them at normal priority so that the
-      // token tiles of one expert that run at about the same time share them
-      // in L2; the second keeps them evict-first, because the fp32 sums it
-      // scatters into y need L2 more
-      const uint64_t pol_w = MODE == 1 ? policy_evict_normal() : policy_evict_first();
+      // weights: kept at normal L2 priority when the expert has more than one
+      // token tile, so that its token tiles, which run at about the same time
+      // on neighbouring units, share them in L2; in the second matmul an
+      // expert with a single token tile loads them evict-first, because the
+      // fp32 sums it scatters into y need L2 more
+      const uint64_t pol_normal = policy_evict_normal();
+      const uint64_t pol_first = MODE == 1 ? pol_normal : policy_evict_first();
       const uint64_t pol_x = policy_evict_last();   // activations: re-read per feature tile
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
       for (int tile = unit; ok && tile < total; tile += nunits) {
         const Tile t = decode_tile(tile, s_tstart, s_tbase, s_off, p.G, p.E, p.T, p.rows_routed);
+        const uint64_t pol_w = t.ntt > 1 ? pol_normal : pol_first;
         const int nmma = (t.nvalid + 15) & ~15;
         const int brows = nmma / CG;  // this CTA's share of the token rows
         const int b0 = t.rowbase + t.n0 + (int)rank * brows;
@@ -1381,6 +1385,7 @@ moe_status make_job(Job &j, const moe_cfg *cfg, int64_t T, const void *x, moe_dt
     if (!w->s1 || !w->s3 || !w->s2) return MOE_ERR_INVALID;
     if (cfg->dim % 128 != 0 || cfg->inter % 128 != 0) return MOE_ERR_UNSUPPORTED;
   }
+  if (w->act_e4m3) return MOE_ERR_UNSUPPORTED;
   j.l = ws_layout(cfg, T, x_dt, w->w_dt);
   if (ws_bytes < j.l.total) return MOE_ERR_WORKSPACE;
   j.c = cfg;

@@ -589,11 +589,29 @@ MOE_EXPORT size_t moe_router_workspace_size(const moe_cfg *cfg, int64_t T) {
   return simt > tc ? simt : tc;
 }
 
-MOE_EXPORT moe_status moe_router_forward(const moe_cfg *cfg, int64_t T, const void *x,
-                                         moe_dtype x_dt, const float *w_r, const float *bias,
-                                         float *weights, int32_t *indices, float *sel_gap,
-                                         void *ws, size_t ws_bytes, int32_t *dev_status,
-                                         moe_stream_t stream) {
+namespace moe {
+namespace {
+
+// bytes of the three-term bf16 split of W_r (0 when the tensor-core scores do
+// not apply to this configuration)
+size_t split_bytes(const moe_cfg *c) {
+  if (c->n_routed % tcr::BM != 0 || c->dim % tcr::BK != 0) return 0;
+  return (size_t)3 * c->n_routed * c->dim * 2;
+}
+
+moe_status enqueue_split(const moe_cfg *cfg, const float *w_r, __nv_bfloat16 *w3,
+                         cudaStream_t s) {
+  const int64_t nw = (int64_t)cfg->n_routed * cfg->dim;
+  split_w3<<<(unsigned)((nw + 255) / 256), 256, 0, s>>>(w_r, w3, nw);
+  return launch_status();
+}
+
+// The forward behind both entry points; w_split is the prepared split of W_r
+// or NULL (then it is written into the workspace first).
+moe_status router_forward(const moe_cfg *cfg, int64_t T, const void *x, moe_dtype x_dt,
+                          const float *w_r, const void *w_split, const float *bias,
+                          float *weights, int32_t *indices, float *sel_gap, void *ws,
+                          size_t ws_bytes, int32_t *dev_status, cudaStream_t s) {
   moe_status st = check_cfg(cfg);
   if (st != MOE_OK) return st;
   if (T < 0 || T > (int64_t)1 << 30) return MOE_ERR_INVALID;
@@ -605,17 +623,18 @@ MOE_EXPORT moe_status moe_router_forward(const moe_cfg *cfg, int64_t T, const vo
     return MOE_ERR_UNSUPPORTED;
   if (ws_bytes < moe_router_workspace_size(cfg, T)) return MOE_ERR_WORKSPACE;
 
-  cudaStream_t s = as_stream(stream);
   float *z_part = static_cast<float *>(ws);
   int nsplit;
   if (tc_router(cfg, x_dt) && T >= 32) {
     const TcPlan tp = plan_tc(cfg, T);
-    const int64_t nw = (int64_t)cfg->n_routed * cfg->dim;
-    __nv_bfloat16 *w3 = static_cast<__nv_bfloat16 *>(ws);
+    const __nv_bfloat16 *w3 = static_cast<const __nv_bfloat16 *>(w_split);
     z_part = reinterpret_cast<float *>(static_cast<uint8_t *>(ws) +
-                                       align_up((size_t)3 * nw * 2, 1024));
-    split_w3<<<(unsigned)((nw + 255) / 256), 256, 0, s>>>(w_r, w3, nw);
-    if ((st = launch_status()) != MOE_OK) return st;
+                                       align_up(split_bytes(cfg), 1024));
+    if (!w3) {
+      __nv_bfloat16 *w3ws = static_cast<__nv_bfloat16 *>(ws);
+      if ((st = enqueue_split(cfg, w_r, w3ws, s)) != MOE_OK) return st;
+      w3 = w3ws;
+    }
     CUtensorMap mw, mx;
     if (!make_tmap_bf16(&mw, w3, (uint64_t)3 * cfg->n_routed, cfg->dim, tcr::BM) ||
         !make_tmap_bf16(&mx, x, (uint64_t)T, cfg->dim, 32))
@@ -643,19 +662,19 @@ MOE_EXPORT moe_status moe_router_forward(const moe_cfg *cfg, int64_t T, const vo
     if ((st = launch_status()) != MOE_OK) return st;
     nsplit = tp.nsplit;
   } else {
-  const Plan p = plan_scores(cfg, T);
-  nsplit = p.nsplit;
-  dim3 grid((unsigned)((T + SC_BM - 1) / SC_BM), (unsigned)((cfg->n_routed + SC_BN - 1) / SC_BN),
-            (unsigned)p.nsplit);
-  if (x_dt == MOE_BF16)
-    router_scores<__nv_bfloat16><<<grid, SC_THREADS, 0, s>>>(
-        static_cast<const __nv_bfloat16 *>(x), w_r, z_part, (int)T, cfg->n_routed, cfg->dim,
-        p.cols_per_split);
-  else
-    router_scores<float><<<grid, SC_THREADS, 0, s>>>(static_cast<const float *>(x), w_r, z_part,
-                                                     (int)T, cfg->n_routed, cfg->dim,
-                                                     p.cols_per_split);
-  if ((st = launch_status()) != MOE_OK) return st;
+    const Plan p = plan_scores(cfg, T);
+    nsplit = p.nsplit;
+    dim3 grid((unsigned)((T + SC_BM - 1) / SC_BM),
+              (unsigned)((cfg->n_routed + SC_BN - 1) / SC_BN), (unsigned)p.nsplit);
+    if (x_dt == MOE_BF16)
+      router_scores<__nv_bfloat16><<<grid, SC_THREADS, 0, s>>>(
+          static_cast<const __nv_bfloat16 *>(x), w_r, z_part, (int)T, cfg->n_routed, cfg->dim,
+          p.cols_per_split);
+    else
+      router_scores<float><<<grid, SC_THREADS, 0, s>>>(static_cast<const float *>(x), w_r,
+                                                       z_part, (int)T, cfg->n_routed, cfg->dim,
+                                                       p.cols_per_split);
+    if ((st = launch_status()) != MOE_OK) return st;
   }
 
   SelectArgs a;
@@ -679,6 +698,44 @@ MOE_EXPORT moe_status moe_router_forward(const moe_cfg *cfg, int64_t T, const vo
       return MOE_ERR_CUDA;
   }
   router_select<<<(unsigned)((T + SEL_WARPS - 1) / SEL_WARPS), SEL_WARPS * 32, smem, s>>>(a);
-  (void)dev_status;
   return launch_status();
+}
+
+}  // namespace
+}  // namespace moe
+
+MOE_EXPORT size_t moe_router_prepare_size(const moe_cfg *cfg) {
+  if (check_cfg(cfg) != MOE_OK) return 0;
+  return split_bytes(cfg);
+}
+
+MOE_EXPORT moe_status moe_router_prepare(const moe_cfg *cfg, const float *w_r, void *prep,
+                                         size_t prep_bytes, moe_stream_t stream) {
+  moe_status st = check_cfg(cfg);
+  if (st != MOE_OK) return st;
+  if (!w_r || !prep) return MOE_ERR_INVALID;
+  const size_t need = split_bytes(cfg);
+  if (need == 0) return MOE_ERR_UNSUPPORTED;
+  if (prep_bytes < need) return MOE_ERR_WORKSPACE;
+  return enqueue_split(cfg, w_r, static_cast<__nv_bfloat16 *>(prep), as_stream(stream));
+}
+
+MOE_EXPORT moe_status moe_router_forward(const moe_cfg *cfg, int64_t T, const void *x,
+                                         moe_dtype x_dt, const float *w_r, const float *bias,
+                                         float *weights, int32_t *indices, float *sel_gap,
+                                         void *ws, size_t ws_bytes, int32_t *dev_status,
+                                         moe_stream_t stream) {
+  return router_forward(cfg, T, x, x_dt, w_r, nullptr, bias, weights, indices, sel_gap, ws,
+                        ws_bytes, dev_status, as_stream(stream));
+}
+
+MOE_EXPORT moe_status moe_router_forward_prepared(const moe_cfg *cfg, int64_t T, const void *x,
+                                                  moe_dtype x_dt, const float *w_r,
+                                                  const void *prep, const float *bias,
+                                                  float *weights, int32_t *indices,
+                                                  float *sel_gap, void *ws, size_t ws_bytes,
+                                                  int32_t *dev_status, moe_stream_t stream) {
+  if (!prep) return MOE_ERR_INVALID;
+  return router_forward(cfg, T, x, x_dt, w_r, prep, bias, weights, indices, sel_gap, ws,
+                        ws_bytes, dev_status, as_stream(stream));
 }

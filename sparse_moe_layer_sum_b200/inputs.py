@@ -7,8 +7,10 @@ one fp32 scale per 128 x 128 weight block for the FP8-weight workload).
 
 Distributions: x ~ N(0, 1); router weight W_r ~ N(0, 1/dim) in fp32; bias ~
 U(-0.1, 0.1) in fp32; expert weights ~ N(0, 1/fan_in) (fan_in = dim for
-w1/w3 and inter for w2).  Draw order: x, W_r, bias, then for every group
-0..E (E = the shared expert) w1, w3, w2.
+w1/w3 and inter for w2).  Draw order: x, W_r, bias, then for each chunk of
+consecutive groups 0..E (E = the shared expert; a chunk holds as many groups
+as fit 2^30 elements of one matrix) one draw of w1, one of w3 and one of w2
+for all groups of the chunk.
 """
 from __future__ import annotations
 
@@ -127,16 +129,21 @@ def make_block(w: Workload, device="cuda", x_seed_offset: int = 0):
         w3 = torch.empty(G, I, D, dtype=wdt, device=dev)
         w2 = torch.empty(G, D, I, dtype=wdt, device=dev)
         s1 = s3 = s2 = None
-    for e in range(G):
-        a = torch.randn(I, D, generator=g, device=dev, dtype=torch.float32) / math.sqrt(D)
-        b = torch.randn(I, D, generator=g, device=dev, dtype=torch.float32) / math.sqrt(D)
-        c = torch.randn(D, I, generator=g, device=dev, dtype=torch.float32) / math.sqrt(I)
-        if w.w_format == "e4m3":
-            w1[e], s1[e] = quantize_e4m3_blocks(a)
-            w3[e], s3[e] = quantize_e4m3_blocks(b)
-            w2[e], s2[e] = quantize_e4m3_blocks(c)
-        else:
-            w1[e], w3[e], w2[e] = a, b, c
+    # one draw per matrix kind and chunk of groups (a handful of launches in
+    # all), chunks bounded so that the fp32 temporaries stay a few GB
+    chunk = max(1, min(G, (1 << 30) // (I * D)))
+    for e0 in range(0, G, chunk):
+        n = min(chunk, G - e0)
+        for wt, sc, (r, c), fan in ((w1, s1, (I, D), D), (w3, s3, (I, D), D), (w2, s2, (D, I), I)):
+            m = torch.randn(n, r, c, generator=g, device=dev, dtype=torch.float32)
+            m.mul_(1.0 / math.sqrt(fan))
+            if w.w_format == "e4m3":
+                q, s = quantize_e4m3_blocks(m.reshape(n * r, c))
+                wt[e0:e0 + n] = q.reshape(n, r, c)
+                sc[e0:e0 + n] = s.reshape(n, r // 128, c // 128)
+            else:
+                wt[e0:e0 + n] = m
+            del m
     return x, BlockParams(w_r, bias, w1, w3, w2, s1, s3, s2)
 
 

@@ -73,10 +73,28 @@ def _ws(nbytes: int, device) -> torch.Tensor:
 # ---------------------------------------------------------------- the four
 
 
+def router_prepare(shape: BlockShape, w_r: torch.Tensor) -> Optional[torch.Tensor]:
+    """moe_router_prepare: the three-term bf16 split of w_r (uint8 device
+    buffer), or None when the tensor-core scoring cannot apply to the shape."""
+    _check_cuda(w_r)
+    cfg = shape.cfg()
+    n = fn("moe_router", "moe_router_prepare_size")(ctypes.byref(cfg))
+    if not n:
+        return None
+    prep = torch.empty(n, dtype=torch.uint8, device=w_r.device)
+    check(fn("moe_router", "moe_router_prepare")(ctypes.byref(cfg), w_r.data_ptr(),
+                                                 prep.data_ptr(), n, _stream()),
+          "moe_router_prepare")
+    return prep
+
+
 def router_forward(shape: BlockShape, x: torch.Tensor, w_r: torch.Tensor,
-                   bias: Optional[torch.Tensor], *, gap: bool = False, ws=None, status=None):
-    """moe_router_forward: (weights [T,k] fp32, indices [T,k] int32, gap [T] or None)."""
-    _check_cuda(x, w_r, bias)
+                   bias: Optional[torch.Tensor], *, gap: bool = False, ws=None, status=None,
+                   prep: Optional[torch.Tensor] = None):
+    """moe_router_forward (moe_router_forward_prepared when `prep` from
+    router_prepare is given): (weights [T,k] fp32, indices [T,k] int32, gap
+    [T] or None)."""
+    _check_cuda(x, w_r, bias, prep)
     cfg = shape.cfg()
     T = x.shape[0]
     weights = torch.empty(T, shape.topk, dtype=torch.float32, device=x.device)
@@ -85,6 +103,13 @@ def router_forward(shape: BlockShape, x: torch.Tensor, w_r: torch.Tensor,
     need = fn("moe_router", "moe_router_workspace_size")(ctypes.byref(cfg), T)
     if ws is None or ws.numel() < need:
         ws = _ws(need, x.device)
+    if prep is not None:
+        st = fn("moe_router", "moe_router_forward_prepared")(
+            ctypes.byref(cfg), T, x.data_ptr(), _dt(x), w_r.data_ptr(), prep.data_ptr(),
+            _ptr(bias), weights.data_ptr(), indices.data_ptr(), _ptr(sel_gap), ws.data_ptr(),
+            ws.numel(), _ptr(status), _stream())
+        check(st, "moe_router_forward_prepared")
+        return weights, indices, sel_gap
     st = fn("moe_router", "moe_router_forward")(
         ctypes.byref(cfg), T, x.data_ptr(), _dt(x), w_r.data_ptr(), _ptr(bias),
         weights.data_ptr(), indices.data_ptr(), _ptr(sel_gap), ws.data_ptr(), ws.numel(),
@@ -114,10 +139,12 @@ def dispatch_build(shape: BlockShape, indices: torch.Tensor, *, ws=None, status=
     return counts, offsets, sorted_token, slot_of
 
 
-def expert_weights_struct(w1, w3, w2, s1=None, s3=None, s2=None) -> MoEExpertWeights:
+def expert_weights_struct(w1, w3, w2, s1=None, s3=None, s2=None,
+                          fp8_act: bool = False) -> MoEExpertWeights:
+    """moe_expert_weights; fp8_act selects the FP8 x FP8 path (e4m3 weights)."""
     _check_cuda(w1, w3, w2, s1, s3, s2)
     return MoEExpertWeights(w1.data_ptr(), w3.data_ptr(), w2.data_ptr(), _dt(w1), _ptr(s1),
-                            _ptr(s3), _ptr(s2))
+                            _ptr(s3), _ptr(s2), int(fp8_act))
 
 
 def experts_forward(shape: BlockShape, x: torch.Tensor, wstruct: MoEExpertWeights,
@@ -218,9 +245,12 @@ class MoEBlock:
     """
 
     def __init__(self, shape: BlockShape, params: BlockParams, T: int, x_dtype: torch.dtype,
-                 device=None, combine: str = "scatter"):
+                 device=None, combine: str = "scatter", fp8_act: bool = False):
         if combine not in ("scatter", "ordered"):
             raise ValueError(combine)
+        if fp8_act and params.s1 is None:
+            raise ValueError("fp8_act needs e4m3 expert weights")
+        self.fp8_act = fp8_act
         self.combine_mode = combine
         self.x_dtype = x_dtype
         self.shape, self.p, self.T = shape, params, T
@@ -228,10 +258,19 @@ class MoEBlock:
         self.cfg = shape.cfg()
         k, D = shape.topk, shape.dim
         self.wstruct = expert_weights_struct(params.w1, params.w3, params.w2, params.s1,
-                                             params.s3, params.s2)
+                                             params.s3, params.s2, fp8_act)
         cfgp = ctypes.byref(self.cfg)
         x_dt = _lib.DTYPES[_TORCH_DT[x_dtype]]
         self.ws_router = _ws(fn("moe_router", "moe_router_workspace_size")(cfgp, T), dev)
+        # the router weight's three-term bf16 split, written once here and
+        # read by every forward (tensor-core scoring path only)
+        self.router_prep = None
+        nprep = fn("moe_router", "moe_router_prepare_size")(cfgp)
+        if nprep and x_dtype == torch.bfloat16:
+            self.router_prep = torch.empty(nprep, dtype=torch.uint8, device=dev)
+            check(fn("moe_router", "moe_router_prepare")(
+                cfgp, params.w_r.data_ptr(), self.router_prep.data_ptr(), nprep, _stream()),
+                "moe_router_prepare")
         self.ws_dispatch = _ws(fn("moe_dispatch", "moe_dispatch_workspace_size")(cfgp, T), dev)
         self.ws_experts = _ws(fn("moe_experts", "moe_experts_workspace_size")(
             cfgp, T, x_dt, self.wstruct.w_dt), dev)
@@ -250,8 +289,8 @@ class MoEBlock:
         self.y = torch.empty(T, D, dtype=f32, device=dev)
         self.status = torch.zeros(1, dtype=i32, device=dev)
 
-    # kernels one forward launches: router 3 (bf16 x on the tensor-core path:
-    # weight split, scores, selection) or 2, dispatch 3, experts 5 on the
+    # kernels one forward launches: router 2 (scores, selection; the weight
+    # split is prepared once), dispatch 3, experts 5 on the
     # tensor-core path, with bf16 or e4m3 weights (two tile tables, row
     # gather, two GEMMs) or 4 on the CUDA-core path, then combine 1 (ordered)
     # or nothing (scatter; y is zeroed by a memset node)
@@ -263,11 +302,19 @@ class MoEBlock:
         tc_experts = (self.x_dtype == torch.bfloat16 and sh.dim % 128 == 0
                       and sh.inter % 128 == 0
                       and self.p.w1.dtype in (torch.bfloat16, torch.uint8, torch.float8_e4m3fn))
-        return ((3 if tc_router else 2) + 3 + (5 if tc_experts else 4)
+        return ((2 if tc_router and self.router_prep is not None else 3 if tc_router else 2)
+                + 3 + (5 if tc_experts else 4)
                 + (1 if self.combine_mode == "ordered" else 0))
 
     def _router(self, x, cfgp, s):
         p = self.p
+        if self.router_prep is not None:
+            check(fn("moe_router", "moe_router_forward_prepared")(
+                cfgp, self.T, x.data_ptr(), _dt(x), p.w_r.data_ptr(), self.router_prep.data_ptr(),
+                _ptr(p.bias), self.weights.data_ptr(), self.indices.data_ptr(),
+                self.sel_gap.data_ptr(), self.ws_router.data_ptr(), self.ws_router.numel(),
+                self.status.data_ptr(), s), "moe_router_forward_prepared")
+            return
         check(fn("moe_router", "moe_router_forward")(
             cfgp, self.T, x.data_ptr(), _dt(x), p.w_r.data_ptr(), _ptr(p.bias),
             self.weights.data_ptr(), self.indices.data_ptr(), self.sel_gap.data_ptr(),

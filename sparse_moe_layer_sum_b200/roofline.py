@@ -43,6 +43,25 @@ def block_work(D, E, I, k, S, T, n_touched, w_bytes, x_bytes, scale_bytes_per_ex
     return Work(weights + router + io, flops)
 
 
+def tensor_peak(peaks: dict, sustained: bool, mma: str) -> float:
+    """Dense tensor peak (TFLOP/s) for the MMA operand type: the measured bf16
+    figure (burst or sustained); fp16 equals it; e4m3 is twice it, the
+    nominal fp8 : bf16 ratio of the part (4.5 : 2.25 PFLOP/s dense)."""
+    bf16 = peaks["bf16_tflops_sustained"] if sustained else peaks["bf16_tflops"]
+    return {"bf16": 1.0, "f16": 1.0, "e4m3": 2.0, "f32": 1.0}[mma] * bf16
+
+
+def method_bytes(D, I, k, S, T, n_touched, w_bytes, x_bytes, scale_bytes_per_expert=0.0):
+    """Bytes of each matmul that the method itself fixes, with no
+    implementation buffers: the weights of the touched experts and the
+    shared one, plus x read by the first and y (fp32) written by the second.
+    The expert-ordered copies of the rows and h are left out."""
+    n_w = n_touched + S
+    sc = scale_bytes_per_expert / 3.0
+    return {"gemm1": n_w * (2 * D * I * w_bytes + 2 * sc) + T * D * x_bytes,
+            "gemm2": n_w * (D * I * w_bytes + sc) + T * D * 4}
+
+
 def kernel_work(D, E, I, k, S, T, n_touched, w_bytes, x_bytes, scale_bytes_per_expert=0.0,
                 scatter=False):
     """Per kernel of one forward: the bytes it must move and flops it must do.

@@ -44,11 +44,25 @@ def _expert_getter(params, w_format: str):
     return get
 
 
-def oracle_y(w: Workload, x: torch.Tensor, params, route: O.RouterResult, tokens=None):
+def oracle_act(w: Workload, fp8_act: bool = False) -> str:
+    """How the oracle rounds the expert activations for a workload's CUDA path
+    (the oracle's readings 3 and 6): fp32 activations stay fp32; bf16 ones
+    round h to bf16, except on the e4m3-weight tensor-core path, whose
+    second-matmul operand h is fp16; the FP8 x FP8 path quantises x and h
+    to e4m3 in 1 x 128 blocks."""
+    if w.x_dtype == torch.float32:
+        return "f32"
+    if w.w_format == "e4m3":
+        return "e4m3" if fp8_act else "f16"
+    return "bf16"
+
+
+def oracle_y(w: Workload, x: torch.Tensor, params, route: O.RouterResult, tokens=None,
+             fp8_act: bool = False):
     """Oracle block output (fp64) for the rows `tokens` (all when None)."""
     get = _expert_getter(params, w.w_format)
     E = w.shape.n_routed
-    act = "bf16" if w.x_dtype == torch.bfloat16 else "f32"
+    act = oracle_act(w, fp8_act)
     xs = to_host_f32(x)
     shared = (lambda: get(E)) if w.shape.n_shared else None
     return O.moe_forward(xs, route, get, shared, E, act, tokens=tokens)

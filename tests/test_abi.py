@@ -78,6 +78,26 @@ def test_router_validation():
     assert router(v3_cfg(), T=0) == 0                          # empty batch: nothing to do
 
 
+def test_router_prepare_validation():
+    size = fn("moe_router", "moe_router_prepare_size")
+    prep = fn("moe_router", "moe_router_prepare")
+    fwd = fn("moe_router", "moe_router_forward_prepared")
+    c = v3_cfg()
+    assert size(ctypes.byref(c)) == 3 * 256 * 7168 * 2          # three bf16 terms of W_r
+    small = v3_cfg(dim=256, n_routed=16, n_groups=4, topk_groups=2, topk=4, inter=128)
+    assert size(ctypes.byref(small)) == 0                      # no tensor-core tiling
+    assert size(ctypes.byref(v3_cfg(topk=200))) == 0           # invalid config
+    assert size(None) == 0
+    assert prep(ctypes.byref(c), None, P, 1 << 30, None) == INVALID
+    assert prep(ctypes.byref(c), P, None, 1 << 30, None) == INVALID
+    assert prep(ctypes.byref(c), P, P, 1024, None) == WORKSPACE
+    assert prep(ctypes.byref(small), P, P, 1 << 30, None) == UNSUPPORTED
+    args = lambda pr: (ctypes.byref(c), 4, P, 1, P, pr, P, P, P, None, P, 1 << 30, None, None)
+    assert fwd(*args(None)) == INVALID                         # the split is required
+    assert fwd(ctypes.byref(c), 0, P, 1, P, P, P, P, P, None, P, 1 << 30, None, None) == 0
+    assert fwd(ctypes.byref(c), 4, P, 1, P, P, P, P, P, None, P, 16, None, None) == WORKSPACE
+
+
 def test_workspace_sizes_grow_with_tokens():
     c = v3_cfg()
     f = fn("moe_router", "moe_router_workspace_size")

@@ -2,25 +2,36 @@
 benchmark times (MoEBlock.forward on the current stream).
 
 Routing is checked on every token (indices bit-exact away from near-ties,
-per-expert counts); the block output on a seeded sample of tokens, which the
-oracle computes one by one.
+per-expert counts); the block output on a seeded sample of 64 tokens, which
+the oracle computes one by one; and expert outputs row by row, through the
+ordered path (moe_experts_forward), for the experts whose tiles differ most:
+the hottest expert, the smallest non-empty one, one whose rows straddle a
+token-tile boundary, and the shared expert's first and last token tiles.
+
+Set MOE_PARITY_REPORT=<file> to append one JSON line per configuration with
+the near-tie counts and errors.
 """
 import gc
+import json
+import os
 
 import numpy as np
 import pytest
 import torch
 
 from oracle import moe_oracle as O
-from parity import compare_routing, oracle_route, oracle_y, y_close
+from parity import (_expert_getter, compare_routing, oracle_act, oracle_route, oracle_y,
+                    y_close)
 from sparse_moe_layer_sum_b200 import moe
-from sparse_moe_layer_sum_b200.inputs import WORKLOADS, make_block, sample_tokens
+from sparse_moe_layer_sum_b200.inputs import WORKLOADS, make_block, sample_tokens, to_host_f32
 
 pytestmark = pytest.mark.gpu
 
 TOL = {"bf16": 2e-2, "e4m3": 5e-2}
-CASES = [("v3_decode_t64", 64), ("v3_prefill_t4096", 12), ("v3_skew_t16384", 12),
-         ("v3_fp8_t8192", 6)]
+# per-expert rows: max |d| / rms(expert output) (the same bounds) and mean
+MEAN_TOL = {"bf16": 2e-4, "e4m3": 1e-3}
+CASES = ["v3_decode_t64", "v3_prefill_t4096", "v3_skew_t16384", "v3_fp8_t8192"]
+N_Y = 64
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -29,8 +40,37 @@ def built():
     build.build_all()
 
 
-@pytest.mark.parametrize("name,n_sample", CASES, ids=[c[0] for c in CASES])
-def test_v3_block(name, n_sample):
+def token_tiles(n: int, rows_max: int):
+    """First row of each token tile of an expert with n rows (the kernels'
+    split: the fewest tiles of at most rows_max rows, equal sizes rounded up
+    to 16)."""
+    if n <= 0:
+        return []
+    ntt0 = -(-n // rows_max)
+    base = (-(-n // ntt0) + 15) // 16 * 16
+    return list(range(0, n, base))
+
+
+def rows_to_check(n: int, rows_max: int, rng) -> np.ndarray:
+    """Rows of an n-row expert within 8 of every token-tile start and of its
+    end, plus 16 at random."""
+    pick = set()
+    for s in token_tiles(n, rows_max):
+        pick.update(range(max(0, s - 8), min(n, s + 8)))
+    pick.update(range(max(0, n - 8), n))
+    pick.update(rng.choice(n, size=min(n, 16), replace=False).tolist())
+    return np.array(sorted(pick))
+
+
+def report(line: dict):
+    path = os.environ.get("MOE_PARITY_REPORT")
+    if path:
+        with open(path, "a") as f:
+            f.write(json.dumps(line) + "\n")
+
+
+@pytest.mark.parametrize("name", CASES)
+def test_v3_block(name):
     w = WORKLOADS[name]
     x, p = make_block(w)
     blk = moe.MoEBlock(w.shape, p, w.T, x.dtype)
@@ -46,16 +86,77 @@ def test_v3_block(name, n_sample):
         assert np.array_equal(counts, O.dispatch(r.indices, w.shape.n_routed).counts)
     # offsets are the exclusive scan of the counts
     assert np.array_equal(blk.offsets.cpu().numpy()[1:], np.cumsum(counts))
-    tokens = sample_tokens(w.T, n_sample).numpy()
+    # the GPU's own near-tie report (sel_gap) flags the oracle's near-ties
+    gap = blk.sel_gap.cpu().numpy()
+    gpu_flagged = int((gap < 1e-6).sum())
+    tokens = sample_tokens(w.T, N_Y).numpy()
     tokens = tokens[rep.same_set[tokens]]
     y_orc = oracle_y(w, x, p, r, tokens=tokens)
     err = y_close(y[torch.from_numpy(tokens).cuda()].cpu().numpy(), y_orc, TOL[w.w_format])
-    print(f"{name}: near-ties {rep.flagged} set flips {rep.set_flips} order flips "
-          f"{rep.order_flips} max gate rel err {rep.max_w_rel:.2e} y err {err:.2e} rms "
-          f"touched {(counts > 0).sum()} zero-count {(counts == 0).sum()}")
+    line = {"workload": name, "T": w.T, "near_ties_oracle": rep.flagged,
+            "near_ties_gpu": gpu_flagged, "set_flips": rep.set_flips,
+            "order_flips": rep.order_flips, "max_gate_rel_err": rep.max_w_rel,
+            "y_tokens": int(tokens.size), "y_max_err_rms": err,
+            "touched": int((counts > 0).sum()), "zero_count": int((counts == 0).sum())}
     if w.hot_experts:
         hot = torch.randperm(256, generator=torch.Generator().manual_seed(2024))[:16].numpy()
-        print(f"{name}: hot-expert share {counts[hot].sum() / counts.sum():.3f}")
+        line["hot_share"] = float(counts[hot].sum() / counts.sum())
+    print(line)
+    report(line)
     del blk, y, x, p
+    gc.collect()
+    torch.cuda.empty_cache()
+
+
+@pytest.mark.parametrize("name", CASES)
+def test_v3_expert_rows(name):
+    """Expert outputs of the full-size launch, row by row, against the oracle."""
+    w = WORKLOADS[name]
+    sh = w.shape
+    x, p = make_block(w)
+    blk = moe.MoEBlock(sh, p, w.T, x.dtype, combine="ordered")
+    blk.forward(x)
+    torch.cuda.synchronize()
+    assert blk.device_status() == 0
+    counts = blk.counts.cpu().numpy()
+    offsets = blk.offsets.cpu().numpy()
+    st = blk.sorted_token.cpu().numpy()
+    # the tile height the experts' kernels use for this batch (decode: 32-row
+    # tiles on one SM; otherwise 256-row tiles on an SM pair)
+    rows_max = 32 if w.T * sh.topk <= 16 * sh.n_routed else 256
+    nz = np.nonzero(counts)[0]
+    chosen = {"hottest": int(nz[np.argmax(counts[nz])]), "smallest": int(nz[np.argmin(counts[nz])])}
+    multi = [e for e in nz if len(token_tiles(counts[e], rows_max)) > 1]
+    if multi:
+        chosen["straddles_tile"] = int(min(multi, key=lambda e: counts[e]))
+    rng = np.random.default_rng(3)
+    xs = to_host_f32(x)
+    act = oracle_act(w)
+    get = _expert_getter(p, w.w_format)
+    out_perm = blk.out_perm
+    line = {"workload": name}
+    for tag, e in chosen.items():
+        rows = rows_to_check(int(counts[e]), rows_max, rng)
+        ref = O.expert_ffn(xs[st[offsets[e] + rows]], *get(e), act)
+        got = out_perm[torch.from_numpy(offsets[e] + rows).cuda()].cpu().numpy()
+        rms = np.sqrt(np.mean(ref ** 2))
+        mx = float(np.max(np.abs(got - ref)) / rms)
+        mean = float(np.mean(np.abs(got - ref)) / rms)
+        line[tag] = {"expert": e, "rows": int(counts[e]), "checked": int(rows.size),
+                     "max": mx, "mean": mean}
+        assert mx <= TOL[w.w_format], (tag, e, mx)
+        assert mean <= MEAN_TOL[w.w_format], (tag, e, mean)
+    # shared expert: rows of its first and last token tiles (all T tokens)
+    rows = rows_to_check(w.T, rows_max, rng)
+    ref = O.expert_ffn(xs[rows], *get(sh.n_routed), act)
+    got = blk.out_shared[torch.from_numpy(rows).cuda()].cpu().numpy()
+    rms = np.sqrt(np.mean(ref ** 2))
+    mx = float(np.max(np.abs(got - ref)) / rms)
+    mean = float(np.mean(np.abs(got - ref)) / rms)
+    line["shared"] = {"rows": w.T, "checked": int(rows.size), "max": mx, "mean": mean}
+    assert mx <= TOL[w.w_format] and mean <= MEAN_TOL[w.w_format], line["shared"]
+    print(line)
+    report(line)
+    del blk, x, p, out_perm
     gc.collect()
     torch.cuda.empty_cache()

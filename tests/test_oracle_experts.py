@@ -109,3 +109,60 @@ def test_weighted_sum_definition_per_token():
         for j in range(4):
             acc += r.weights[t, j] * expert_ffn(x[t:t + 1], *experts[r.indices[t, j]], "f32")[0]
         assert np.allclose(y[t], acc, rtol=1e-12, atol=1e-12)
+
+
+def _two_unit_expert():
+    # D = I = 128 (one quantisation block each).  x = 3.5 at column 0, so its
+    # block scale is 3.5 / 448 = 2^-7 and x survives the quantisation
+    # exactly.  a_0 = ln 3, u_0 = 2 -> h_0 = 1.5 ln 3 = 1.64792 -> bf16
+    # 1.6484375; a_1 = ln 3, u_1 = 0.6 -> h_1 = 0.49438 -> bf16 0.494140625.
+    # Output row 0 sums h_0 + h_1 (w2 row 0 = 1 at columns 0 and 1).
+    D = I = 128
+    x = np.zeros((1, D), np.float32)
+    x[0, 0] = 3.5
+    w1 = np.zeros((I, D))
+    w3 = np.zeros((I, D))
+    w2 = np.zeros((D, I))
+    w1[0, 0] = w1[1, 0] = math.log(3) / 3.5
+    w3[0, 0] = 2.0 / 3.5
+    w3[1, 0] = 0.6 / 3.5
+    w2[0, 0] = w2[0, 1] = 1.0
+    return x, w1, w3, w2
+
+
+def test_two_unit_chain_bf16_and_e4m3():
+    x, w1, w3, w2 = _two_unit_expert()
+    assert expert_ffn(x, w1, w3, w2, "bf16")[0, 0] == 1.6484375 + 0.494140625
+    # e4m3: h's block amax 1.6484375 sets scale = fp32(1.6484375 / 448); h_0
+    # becomes 448 steps of it, h_1 = 0.494140625 / scale = 134.29 -> the
+    # e4m3 binade [128, 256) has step 16 -> 128 steps
+    scale = float(np.float32(1.6484375) / np.float32(448.0))
+    assert expert_ffn(x, w1, w3, w2, "e4m3")[0, 0] == (448 + 128) * scale
+    assert np.all(expert_ffn(x, w1, w3, w2, "e4m3")[0, 1:] == 0)
+
+
+def test_two_unit_chain_f16():
+    # fp16 keeps 10 fraction bits: h_0 = 1.5 ln 3 in [1, 2) rounds to a
+    # multiple of 2^-10, h_1 = 0.45 ln 3 in [0.25, 0.5) to a multiple of 2^-12
+    x, w1, w3, w2 = _two_unit_expert()
+    h0 = float(np.float32(0.75 * math.log(3) * 2.0))
+    h1 = float(np.float32(0.75 * math.log(3) * 0.6))
+    want = round(h0 / 2.0 ** -10) * 2.0 ** -10 + round(h1 / 2.0 ** -12) * 2.0 ** -12
+    assert want == 1.6474609375 + 0.494384765625
+    assert expert_ffn(x, w1, w3, w2, "f16")[0, 0] == want
+
+
+def test_e4m3_activation_error_is_a_few_percent():
+    # the quantisation error of x and h (3 fraction bits, half-step 2^-4
+    # relative) shows as a few percent rms on random data; zero or tens of
+    # percent would mean a skipped or mis-scaled step
+    rng = np.random.default_rng(9)
+    x = rng.standard_normal((32, 256)).astype(np.float32)
+    w1, w3, w2 = _tiny_weights(rng, 256, 256)
+    ref = expert_ffn(x, w1, w3, w2, "f32")
+    got = expert_ffn(x, w1, w3, w2, "e4m3")
+    rel = np.sqrt(np.mean((got - ref) ** 2) / np.mean(ref ** 2))
+    assert 0.01 < rel < 0.1, rel
+    f16 = expert_ffn(x, w1, w3, w2, "f16")
+    rel16 = np.sqrt(np.mean((f16 - ref) ** 2) / np.mean(ref ** 2))
+    assert 1e-5 < rel16 < 1e-3, rel16

@@ -67,3 +67,96 @@ def test_dequant_block_scale_layout():
     w = dequant_e4m3_block(q, s)
     assert w[0, 0] == 1 and w[127, 127] == 1 and w[0, 128] == 2 and w[0, 383] == 3
     assert w[128, 0] == 4 and w[255, 255] == 5 and w[255, 256] == 6
+
+
+# ------------------------------------------------------------ fp16, e4m3 encode
+
+from conftest import read_golden  # noqa: E402
+from oracle.moe_oracle import (dequant_e4m3_rows, e4m3_code, quantize_e4m3_rows,  # noqa: E402
+                               round_f32_to_f16, round_to_e4m3)
+
+
+def test_f16_round_special_values():
+    cases = {
+        1.0 + 2.0 ** -11: 1.0,                     # halfway, even neighbour 1
+        1.0 + 3 * 2.0 ** -11: 1.0 + 2.0 ** -9,     # halfway, even neighbour 1 + 2^-9
+        65504.0: 65504.0,                          # largest finite
+        2.0 ** -24: 2.0 ** -24,                    # smallest subnormal
+        2.0 ** -25: 0.0,                           # half of it: ties to even (0)
+        3 * 2.0 ** -25: 2.0 ** -23,                # 1.5 subnormal steps -> 2
+        -(2.0 ** -14 + 2.0 ** -25): -(2.0 ** -14),  # below the normal spacing, rounds down
+        0.1: 0.0999755859375,
+    }
+    for v, want in cases.items():
+        got = float(round_f32_to_f16(np.array([v], dtype=np.float32))[0])
+        assert got == want, (v, got, want)
+
+
+def test_f16_round_matches_torch():
+    g = torch.Generator().manual_seed(6)
+    v = torch.randn(100000, generator=g) * torch.exp(torch.randn(100000, generator=g) * 3)
+    v = v.clamp(-60000, 60000)
+    assert np.array_equal(round_f32_to_f16(v.numpy()), v.to(torch.float16).double().numpy())
+
+
+def test_e4m3_round_midpoints_go_to_even_codes():
+    # brute force over every pair of neighbouring positive finite codes: the
+    # midpoint rounds to the code whose lowest bit is 0, a hair off it to
+    # the nearer one
+    t = e4m3_table()
+    for c in range(0x00, 0x7E):
+        lo, hi = t[c], t[c + 1]
+        mid = 0.5 * (lo + hi)
+        want = lo if c % 2 == 0 else hi
+        assert round_to_e4m3(np.array([mid]))[0] == want, (c, mid)
+        assert round_to_e4m3(np.array([-mid]))[0] == -want
+        assert round_to_e4m3(np.array([mid - 1e-9 * hi]))[0] == lo
+        assert round_to_e4m3(np.array([mid + 1e-9 * hi]))[0] == hi
+
+
+def test_e4m3_round_saturates_and_matches_torch():
+    assert round_to_e4m3(np.array([464.0, 1000.0, -1e9]))[0] == 448.0
+    assert list(round_to_e4m3(np.array([464.0, 1000.0, -1e9]))) == [448.0, 448.0, -448.0]
+    g = torch.Generator().manual_seed(7)
+    v = (torch.randn(100000, generator=g) * torch.exp(torch.randn(100000, generator=g) * 3))
+    v = v.clamp(-448, 448)
+    ref = v.to(torch.float8_e4m3fn).double().numpy()
+    assert np.array_equal(round_to_e4m3(v.double().numpy()), ref)
+
+
+def test_e4m3_code_inverts_the_table():
+    t = e4m3_table()
+    codes = np.array([c for c in range(256) if np.isfinite(t[c]) and c != 0x80], dtype=np.uint8)
+    assert np.array_equal(e4m3_code(t[codes]), codes)
+
+
+def test_activation_quantisation_worked_example():
+    g = read_golden("e4m3_act_quant.txt")
+    v = np.zeros((2, 256), dtype=np.float32)
+    v[0, [int(c) for c in g["row0_cols"]]] = [float(x) for x in g["row0_vals"]]
+    v[1, [int(c) for c in g["row1_cols"]]] = [float(x) for x in g["row1_vals"]]
+    vals, scales = quantize_e4m3_rows(v)
+    assert scales.dtype == np.float32
+    assert list(scales[0]) == [float(x) for x in g["row0_scales"]]
+    assert list(scales[1]) == [float(x) for x in g["row1_scales"]]
+    deq = dequant_e4m3_rows(vals, scales)
+    want0 = [float(x) for x in g["row0_codes_times_scale"]]
+    assert list(deq[0, [int(c) for c in g["row0_cols"]]]) == want0
+    assert list(deq[1, [int(c) for c in g["row1_cols"]]]) == [float(x) for x in g["row1_deq"]]
+    assert np.count_nonzero(deq) == 7                    # zeros stay zero, block 1 empty
+
+
+def test_activation_quantisation_error_bound():
+    # every dequantised value is within half an e4m3 step of the value: 2^-4
+    # relative above 2^-6 * scale, 2^-10 * scale absolute below
+    rng = np.random.default_rng(8)
+    v = (rng.standard_normal((64, 512)) * np.exp(rng.standard_normal((64, 1)))).astype(np.float32)
+    vals, scales = quantize_e4m3_rows(v)
+    deq = dequant_e4m3_rows(vals, scales)
+    s = np.repeat(scales.astype(np.float64), 128, axis=1)
+    bound = np.maximum(np.abs(v) * 2.0 ** -4, s * 2.0 ** -10) * (1 + 1e-6)
+    assert np.all(np.abs(deq - v) <= bound)
+    # the block maximum itself is kept to fp32 rounding of the scale
+    amax = np.abs(v.reshape(64, 4, 128)).max(-1)
+    deq_max = np.abs(deq.reshape(64, 4, 128)).max(-1)
+    assert np.allclose(deq_max, amax, rtol=2e-7)

@@ -8,7 +8,8 @@ bias), so a dropped term or a wrong factor shows up against these sums.
 """
 import pytest
 
-from sparse_moe_layer_sum_b200.roofline import block_work, kernel_work, load_peaks
+from sparse_moe_layer_sum_b200.roofline import (block_work, kernel_work, load_peaks,
+                                                 method_bytes, tensor_peak)
 
 D, E, I, K, S = 7168, 256, 2048, 8, 1
 PER_EXPERT = 44_040_192  # parameters of one expert, as the page counts them
@@ -67,3 +68,24 @@ def test_load_peaks_falls_back_without_a_measurement(tmp_path):
     peaks, src = load_peaks(str(tmp_path))
     assert src == "fallback"
     assert peaks["hbm_gbs"] == 6650.0 and peaks["bf16_tflops"] == 1590.0
+
+
+def test_method_bytes_are_weights_plus_block_io():
+    T, n = 4096, 255
+    m = method_bytes(D, I, K, S, T, n, w_bytes=2, x_bytes=2)
+    # the first matmul streams w1 and w3 (two thirds of each expert) and x once
+    assert m["gemm1"] == (n + 1) * (2 * PER_EXPERT // 3) * 2 + T * D * 2
+    # the second streams w2 (one third) and writes y in fp32
+    assert m["gemm2"] == (n + 1) * (PER_EXPERT // 3) * 2 + T * D * 4
+    # together with the router they are the block's bytes
+    b = block_work(D, E, I, K, S, T, n, w_bytes=2, x_bytes=2)
+    assert m["gemm1"] + m["gemm2"] + E * D * 4 + E * 4 == b.bytes
+    kw = kernel_work(D, E, I, K, S, T, n, w_bytes=2, x_bytes=2, scatter=True)
+    assert m["gemm1"] < kw["gemm1"].bytes and m["gemm2"] < kw["gemm2"].bytes
+
+
+def test_tensor_peak_by_operand_type():
+    p = {"bf16_tflops": 1600.0, "bf16_tflops_sustained": 1400.0}
+    assert tensor_peak(p, False, "bf16") == 1600.0
+    assert tensor_peak(p, True, "f16") == 1400.0
+    assert tensor_peak(p, False, "e4m3") == 3200.0

@@ -66,6 +66,16 @@ def test_no_alloc_dispatch_matches_workspace_dispatch_twice():
         for a, b in zip(ref, got):  # integer outputs: identical
             assert torch.equal(a, b)
         assert int(status.item()) == 0
+    # an empty batch, and a batch whose histograms fill the scratch array
+    # exactly (ceil(T / 64) * E = 262144 ints)
+    for T, seed in ((0, 3), (64 * (262144 // E), 4)):
+        idx = random_topk_indices(T, E, k, seed=seed, device="cuda")
+        ref = _with_workspace(cfg, idx, T, E, k)
+        got = _no_alloc(cfg, idx, T, E, k, status)
+        torch.cuda.synchronize()
+        for a, b in zip(ref, got):
+            assert torch.equal(a, b)
+        assert int(status.item()) == 0
     # beyond the fixed scratch size: a clear error and nothing launched
     big = 64 * (262144 // E + 1)
     rc = _lib.fn("moe_dispatch", "moe_dispatch_build_noalloc")(
