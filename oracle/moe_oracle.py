@@ -202,10 +202,11 @@ def quantize_e4m3_rows(v: np.ndarray, block: int = 128):
     """Per-row 1 x block e4m3 quantisation of activations, fp32 arithmetic.
 
     For each row and each run of `block` columns: amax = max |v| (exact),
-    scale = fp32(amax / 448) (an IEEE fp32 division), code = the e4m3 value
-    nearest fp32(v / scale) (IEEE fp32 division, ties to even, saturated);
-    an all-zero block has scale 0 and codes 0.  This is the weights' rule
-    (scale = block amax / 448) applied to 1 x 128 blocks of a row.
+    scale = fp32(amax / 448) (an IEEE fp32 division), r = fp32(1 / scale)
+    (IEEE fp32 reciprocal), code = the e4m3 value nearest fp32(v * r) (ties
+    to even, saturated); an all-zero block has scale 0 and codes 0.  This is
+    the weights' rule (scale = block amax / 448) applied to 1 x 128 blocks of
+    a row, with one reciprocal per block in place of a division per value.
     Returns (values [rows, cols] fp64 of the codes, scales [rows, cols/block] fp32);
     the dequantised activation is values * scale.
     """
@@ -215,7 +216,8 @@ def quantize_e4m3_rows(v: np.ndarray, block: int = 128):
     amax = np.abs(vb).max(axis=-1)
     scale = (amax / np.float32(E4M3_MAX)).astype(np.float32)
     safe = np.where(scale > 0, scale, np.float32(1.0)).astype(np.float32)
-    q = (vb / safe[:, :, None]).astype(np.float32)        # fp32 division
+    recip = (np.float32(1.0) / safe).astype(np.float32)     # fp32 reciprocal
+    q = (vb * recip[:, :, None]).astype(np.float32)         # fp32 product
     vals = round_to_e4m3(q.astype(np.float64))
     vals = np.where(scale[:, :, None] > 0, vals, 0.0)
     return vals.reshape(r, c), scale
