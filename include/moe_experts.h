@@ -120,6 +120,23 @@ moe_status moe_experts_down(const moe_cfg *cfg, int64_t T, moe_dtype x_dt,
                             int32_t *dev_status, moe_stream_t stream);
 
 /*
+ * The activation quantiser of the FP8 x FP8 path (act_e4m3 = 1), on its own:
+ * each row of src [rows, K] bf16 is cut into K / 128 blocks of 128 values;
+ * a block's scale is amax / 448 (fp32, IEEE division) and its codes are
+ * e4m3(v * fp32(1 / scale)) (IEEE reciprocal, round to nearest even,
+ * saturated to +-448); an all-zero block has scale 0 and codes 0.
+ *   q       [rows, K] uint8 out (e4m3 codes, row-major)
+ *   scales  [K / 128, ld] fp32 out, transposed: row r's scale of block b at
+ *           scales[b * ld + r]; ld >= rows
+ * No counterpart on the pages, which name FP8 experts but no activation
+ * format (the weights' 128 x 128 block rule applied to 1 x 128 blocks).
+ * Limits: K % 128 == 0, rows < 2^31.  Returns MOE_ERR_INVALID for bad
+ * sizes or NULL pointers (rows == 0 launches nothing).
+ */
+moe_status moe_quantize_e4m3_rows(const void *src, int64_t rows, int32_t K, uint8_t *q,
+                                  float *scales, int64_t ld, moe_stream_t stream);
+
+/*
  * Profiling: register up to five caller-owned cudaEvent_t handles that later
  * calls record on their stream: [0] before the row gather, [1] before the
  * first GEMM, [2] after it, [3] before the second GEMM, [4] after it.  n = 0

@@ -222,6 +222,10 @@ struct Params {
   float *y;                // [T, D], zeroed before the launch
   // e4m3 weights: fp32 scales of 128 x 128 blocks, [G, rows/128, cols/128]
   const float *sA0, *sA1;  // GEMM1: w1, w3; second GEMM: w2 (sA1 unused)
+  // FP8 x FP8 path: the activation rows' 1 x 128 block scales, transposed
+  // [K / 128][ld_sx] (row r's scale for k-block kb at kb * ld_sx + r)
+  const float *sX;
+  int ld_sx;
 };
 
 // CG = CTA group: 1 = one SM per tile; 2 = an SM pair per tile (cta_group::2),
@@ -821,6 +825,458 @@ __global__ void selftest_wait_kernel(int64_t limit_ns, int32_t *status) {
 
 }  // namespace tc
 
+// ------------------------------------------------ FP8 x FP8 (e4m3 activations)
+//
+// The optional path for e4m3 weights on which the activations are quantised
+// to e4m3 as well, so that the matmuls run as e4m3 x e4m3 tensor-core MMAs
+// (kind::f8f6f4, twice the bf16 rate).  Both operands carry fp32 block scales
+// along the reduction dimension: the weights per 128 x 128 block, the
+// activation rows per 1 x 128 block.  A k-block of 128 is one 128-byte
+// swizzle row of e4m3, so every k-block's partial sum is scaled by one weight
+// scale per CTA (its 128 weight rows lie in one scale block) times one
+// activation scale per token:
+//   acc[m, n] = sum_kb  s_w[kb] * s_x[n, kb] * (sum_{k in kb} q_w[m, k] q_x[n, k])
+// The MMAs of a k-block write a fresh TMEM partial (two buffers alternate)
+// and eight promotion warps fold it into fp32 running sums in registers.
+
+// Rows of a bf16 matrix [*, K] quantised to e4m3 in 1 x 128 blocks:
+// scale = amax / 448 (IEEE division), r = 1 / scale (IEEE reciprocal),
+// code = e4m3(v * r), rounded to nearest even and saturated; an all-zero
+// block has scale 0 and codes 0.  With GATHER, output row p < rows_routed
+// is token sorted_token[p] and row rows_routed + t is token t (the shared
+// expert's rows); otherwise row p is source row p.  Codes go to q [rows, K]
+// row-major; scales, transposed, to sc [K / 128][ld], so that the scales of
+// a tile's tokens for one k-block are contiguous.  A block of eight warps
+// takes 32 consecutive rows; a warp quantises one 128-column block per step,
+// four values per lane.
+template <bool GATHER>
+__global__ void __launch_bounds__(256) quant_rows_e4m3(const uint2 *__restrict__ src,
+                                                       const int32_t *__restrict__ sorted_token,
+                                                       uint32_t *__restrict__ q,
+                                                       float *__restrict__ sc, int rows_routed,
+                                                       int rows_total, int T, int K, int ld) {
+  extern __shared__ float s_sc[];  // [K / 128][32]
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int row0 = blockIdx.x * 32;
+  const int KB = K / 128;
+  for (int rr = warp; rr < 32; rr += 8) {
+    const int row = row0 + rr;
+    if (row >= rows_total) break;
+    const int srow = !GATHER ? row : row < rows_routed ? sorted_token[row] : row - rows_routed;
+    const uint2 *s = src + (size_t)srow * (K / 4);
+    uint32_t *d = q + (size_t)row * (K / 4);
+    for (int kb = 0; kb < KB; ++kb) {
+      const uint2 v = __ldg(s + kb * 32 + lane);  // four bf16
+      const float f0 = __uint_as_float(v.x << 16), f1 = __uint_as_float(v.x & 0xffff0000u);
+      const float f2 = __uint_as_float(v.y << 16), f3 = __uint_as_float(v.y & 0xffff0000u);
+      float m = fmaxf(fmaxf(fabsf(f0), fabsf(f1)), fmaxf(fabsf(f2), fabsf(f3)));
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+      const float scale = m / 448.0f;
+      uint32_t packed = 0;
+      if (scale > 0.0f) {
+        const float r = __frcp_rn(scale);
+        packed = (uint32_t)sm100::f32x2_to_e4m3x2(__fmul_rn(f0, r), __fmul_rn(f1, r)) |
+                 ((uint32_t)sm100::f32x2_to_e4m3x2(__fmul_rn(f2, r), __fmul_rn(f3, r)) << 16);
+      }
+      d[kb * 32 + lane] = packed;
+      if (lane == 0) s_sc[kb * 32 + rr] = scale;
+    }
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < KB * 32; i += 256) {
+    const int kb = i / 32, rr = i % 32;
+    if (row0 + rr < rows_total) sc[(size_t)kb * ld + row0 + rr] = s_sc[i];
+  }
+}
+
+namespace f8 {
+
+using tc::drain_wait;
+using tc::sleep_ns;
+using tc::swiglu_h;
+
+constexpr int BK = 128;                // K per stage: one 128-byte swizzle row of e4m3
+constexpr int BM = 128;                // weight rows per CTA
+constexpr int BN_MAX = 256;            // token rows per tile (per SM pair)
+constexpr int BOXN = 32;               // token rows per TMA box
+constexpr int EPI = 8;                 // promotion / epilogue warps (two per TMEM lane quarter)
+constexpr int NT = 32 * (2 + EPI);
+constexpr int A_BYTES = BM * BK;       // 16 KB
+constexpr int B_ROWS = BN_MAX / 2;     // token rows one CTA holds
+constexpr int B_BYTES = B_ROWS * BK;   // 16 KB
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr int NPBUF = 2;               // TMEM partial-sum buffers of BN_MAX columns
+constexpr int CHUNKS = BN_MAX / 32 / 2;  // 32-column chunks per promotion warp
+constexpr int XB_STRIDE = 17;
+
+template <int STAGES>
+struct Layout {
+  static constexpr int BAR_OFF = STAGES * STAGE_BYTES;
+  // full, empty per stage; partial full, partial empty per buffer; drain
+  static constexpr int NBARS = 2 * STAGES + 2 * NPBUF + 1;
+  static constexpr int MISC_OFF = BAR_OFF + NBARS * 8;
+  static constexpr int MISC_BYTES = 16 + 4 * STAGES;  // TMEM slot, abort flag, pending loads
+  static constexpr int SC_OFF = (MISC_OFF + MISC_BYTES + 127) / 128 * 128;
+  static constexpr int SC_BYTES = EPI * CHUNKS * 32 * 4;  // combined scales of one k-block
+  static constexpr int XBUF_OFF = SC_OFF + SC_BYTES;
+  // SwiGLU exchange of the four warp pairs (first matmul), or the tile's
+  // (token, gate) list (second matmul with the scatter)
+  static constexpr int XBUF_BYTES = 4 * 2 * 32 * XB_STRIDE * 4;
+  static constexpr int TAB_OFF = XBUF_OFF + XBUF_BYTES;
+  static size_t smem_bytes(int G, int E) {
+    return 1024 + TAB_OFF + sizeof(int32_t) * (size_t)((G + 1) + G + (E + 1));
+  }
+  static_assert(BN_MAX * 8 <= XBUF_BYTES, "token list");
+  static_assert(NPBUF * BN_MAX <= 512, "TMEM columns");
+};
+
+// MODE 1: h = silu(x w1^T) * (x w3^T), bf16 out (the pair's 256 weight rows
+// per tile are 64 rows of w1 over the same 64 rows of w3 in each CTA: 128
+// features).  MODE 2: o = h w2^T, fp32 per-slot outputs.  MODE 3: gate * o
+// added into y.  Warp 0 issues TMA loads, one thread of warp 1 the MMAs,
+// warps 2-9 promote the partial sums and run the epilogue.
+template <int MODE, int STAGES>
+__global__ void __maxnreg__(200)
+    tc_fp8_gemm(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA1,
+                const __grid_constant__ CUtensorMap tmB, const tc::Params p) {
+  using L = Layout<STAGES>;
+  using namespace sm100;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                            ~static_cast<uintptr_t>(1023));
+  uint64_t *full = reinterpret_cast<uint64_t *>(sm + L::BAR_OFF);
+  uint64_t *empty = full + STAGES;
+  uint64_t *pfull = empty + STAGES;
+  uint64_t *pempty = pfull + NPBUF;
+  uint64_t *drain = pempty + NPBUF;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + L::MISC_OFF);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + L::MISC_OFF + 4);
+  volatile int *pending = reinterpret_cast<volatile int *>(sm + L::MISC_OFF + 16);
+  float *s_comb = reinterpret_cast<float *>(sm + L::SC_OFF);
+  float *xbuf = reinterpret_cast<float *>(sm + L::XBUF_OFF);
+  int32_t *s_tstart = reinterpret_cast<int32_t *>(sm + L::TAB_OFF);
+  int32_t *s_tbase = s_tstart + p.G + 1;
+  int32_t *s_off = s_tbase + p.G;
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const uint32_t rank = cluster_rank();
+  const bool leader = rank == 0;
+  const int unit = (int)cluster_id_x();
+  const int nunits = (int)cluster_count_x();
+  const int KB = p.KB;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(full + s, 1);
+      mbar_init(empty + s, 1);
+      pending[s] = -1;
+    }
+    for (int b = 0; b < NPBUF; ++b) {
+      mbar_init(pfull + b, 1);
+      mbar_init(pempty + b, EPI * 2);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&tmA0);
+    if (MODE == 1) tma_prefetch_desc(&tmA1);
+    tma_prefetch_desc(&tmB);
+  }
+  for (int i = threadIdx.x; i <= p.G; i += NT) s_tstart[i] = p.tile_start[i];
+  for (int i = threadIdx.x; i < p.G; i += NT) s_tbase[i] = p.tile_base[i];
+  for (int i = threadIdx.x; i <= p.E; i += NT) s_off[i] = p.offsets[i];
+  if (warp == 1) {
+    tmem_alloc_pair(tmem_slot, 512);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();  // the pair's barriers exist before any remote arrive
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int total = s_tstart[p.G];
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---------------------------------------------------- TMA producer
+      // weights at normal L2 priority when their expert has several token
+      // tiles (which then share them in L2), else evict-first in the second
+      // matmul, whose scattered fp32 sums need L2 more; token rows evict-last
+      const uint64_t pol_normal = policy_evict_normal();
+      const uint64_t pol_first = MODE == 1 ? pol_normal : policy_evict_first();
+      const uint64_t pol_x = policy_evict_last();
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int tile = unit; ok && tile < total; tile += nunits) {
+        const Tile t = decode_tile(tile, s_tstart, s_tbase, s_off, p.G, p.E, p.T, p.rows_routed);
+        const uint64_t pol_w = t.ntt > 1 ? pol_normal : pol_first;
+        const int nmma = (t.nvalid + 15) & ~15;
+        const int brows = nmma / 2;
+        const int b0 = t.rowbase + t.n0 + (int)rank * brows;
+        const int arow = MODE == 1 ? t.g * p.I + t.ft * 128 + (int)rank * 64
+                                   : t.g * p.D + t.ft * 256 + (int)rank * BM;
+        const int nbox = (brows + BOXN - 1) / BOXN;
+        const uint32_t bytes = (uint32_t)(A_BYTES + nbox * BOXN * BK);
+        const int k0 = k_rotation(t, KB);
+        for (int i = 0; i < KB; ++i) {
+          const int kb = k0 + i < KB ? k0 + i : k0 + i - KB;
+          if (!wait_bounded(empty + stage, phase ^ 1u, abort_flag, p.timeout_ns, p.status)) {
+            ok = false;
+            break;
+          }
+          // the leader's full barrier counts the bytes of both CTAs
+          if (leader) mbar_arrive_expect_tx(full + stage, bytes * 2);
+          pending[stage] = (int)phase;
+          uint8_t *a_dst = sm + stage * STAGE_BYTES;
+          uint8_t *b_dst = a_dst + A_BYTES;
+          const uint32_t fb = mapa_shared(smem_u32(full + stage), 0);
+          if (MODE == 1) {
+            tma_load_2d_pair(&tmA0, a_dst, fb, kb * BK, arow, pol_w);
+            tma_load_2d_pair(&tmA1, a_dst + A_BYTES / 2, fb, kb * BK, arow, pol_w);
+          } else {
+            tma_load_2d_pair(&tmA0, a_dst, fb, kb * BK, arow, pol_w);
+          }
+          for (int b = 0; b < nbox; ++b)
+            tma_load_2d_pair(&tmB, b_dst + b * BOXN * BK, fb, kb * BK, b0 + b * BOXN, pol_x);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && leader) {
+      // ------------------------------------------------------ MMA issuer
+      int stage = 0, pb = 0;
+      uint32_t phase = 0, pphase = 0;
+      bool ok = true;
+      for (int tile = unit; ok && tile < total; tile += nunits) {
+        const Tile t = decode_tile(tile, s_tstart, s_tbase, s_off, p.G, p.E, p.T, p.rows_routed);
+        const int nmma = (t.nvalid + 15) & ~15;
+        const uint32_t idesc = idesc_e4m3_f32(2 * BM, nmma);
+        for (int i = 0; i < KB; ++i) {
+          if (!wait_bounded(pempty + pb, pphase ^ 1u, abort_flag, p.timeout_ns, p.status) ||
+              !wait_bounded(full + stage, phase, abort_flag, p.timeout_ns, p.status)) {
+            ok = false;
+            break;
+          }
+          pending[stage] = -1;
+          tc_fence_after();
+          const uint32_t a_addr = smem_u32(sm + stage * STAGE_BYTES);
+          const uint32_t b_addr = a_addr + A_BYTES;
+          const uint32_t d_tmem = tmem_base + (uint32_t)(pb * BN_MAX);
+#pragma unroll
+          for (int kk = 0; kk < BK / 32; ++kk)
+            mma_f8_pair(d_tmem, sdesc_sw128(a_addr + kk * 32), sdesc_sw128(b_addr + kk * 32), idesc,
+                        kk != 0 ? 1u : 0u);
+          mma_commit_pair_mc(empty + stage, 0x3);
+          mma_commit_pair_mc(pfull + pb, 0x3);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+          if (++pb == NPBUF) {
+            pb = 0;
+            pphase ^= 1u;
+          }
+        }
+      }
+      if (!ok) {
+        // make sure no MMA is still writing TMEM before it is freed
+        mma_commit_pair(drain);
+        drain_wait(drain, 0, p.timeout_ns);
+      }
+    }
+  } else {
+    // ------------------------------------------- promotion and epilogue
+    const int q = warp & 3;           // TMEM lane quarter this warp may access
+    const int half = (warp - 2) >> 2;  // the two warps of a quarter take alternate chunks
+    float *comb = s_comb + (warp - 2) * CHUNKS * 32;
+    const uint32_t lane_base = tmem_base + ((uint32_t)(q * 32) << 16);
+    int pb = 0;
+    uint32_t pphase = 0;
+    bool ok = true;
+    for (int tile = unit; ok && tile < total; tile += nunits) {
+      const Tile t = decode_tile(tile, s_tstart, s_tbase, s_off, p.G, p.E, p.T, p.rows_routed);
+      const int row0 = t.rowbase + t.n0;
+      // weight scales of this CTA's rows, one per k-block
+      const float *sw;
+      if (MODE == 1)
+        sw = (q < 2 ? p.sA0 : p.sA1) + ((size_t)t.g * (p.I / 128) + t.ft) * KB;
+      else
+        sw = p.sA0 + ((size_t)t.g * (p.D / 128) + t.ft * 2 + (int)rank) * KB;
+      const float *sx = p.sX + row0 + lane;
+      float acc[CHUNKS][32];
+#pragma unroll
+      for (int j = 0; j < CHUNKS; ++j)
+#pragma unroll
+        for (int e = 0; e < 32; ++e) acc[j][e] = 0.0f;
+      const int k0 = k_rotation(t, KB);
+      // scales are fetched two k-blocks ahead of their use
+      float nx[2][CHUNKS], nw[2];
+      auto fetch = [&](int i, float (&x)[CHUNKS], float &w) {
+        const int kb = k0 + i < KB ? k0 + i : k0 + i - KB;
+        w = __ldg(sw + kb);
+#pragma unroll
+        for (int j = 0; j < CHUNKS; ++j) {
+          const int c = (2 * j + half) * 32 + lane;
+          x[j] = c < t.nvalid ? __ldg(sx + (size_t)kb * p.ld_sx + (2 * j + half) * 32) : 0.0f;
+        }
+      };
+      fetch(0, nx[0], nw[0]);
+      if (KB > 1) fetch(1, nx[1], nw[1]);
+      for (int i = 0; i < KB; ++i) {
+        float cx[CHUNKS], cw = nw[0];
+#pragma unroll
+        for (int j = 0; j < CHUNKS; ++j) {
+          cx[j] = nx[0][j];
+          nx[0][j] = nx[1][j];
+        }
+        nw[0] = nw[1];
+        if (i + 2 < KB) fetch(i + 2, nx[1], nw[1]);
+        if (!wait_bounded(pfull + pb, pphase, abort_flag, p.timeout_ns, p.status)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+#pragma unroll
+        for (int j = 0; j < CHUNKS; ++j) comb[j * 32 + lane] = cw * cx[j];
+        __syncwarp();
+#pragma unroll
+        for (int j = 0; j < CHUNKS; ++j) {
+          const int c0 = (2 * j + half) * 32;
+          if (c0 < t.nvalid) {
+#pragma unroll
+            for (int hh = 0; hh < 32; hh += 16) {
+              uint32_t v[16];
+              tmem_ld_32x32b_x16(lane_base + (uint32_t)(pb * BN_MAX + c0 + hh), v);
+              tmem_wait_ld();
+#pragma unroll
+              for (int e = 0; e < 16; e += 4) {
+                const float4 c = *reinterpret_cast<const float4 *>(comb + j * 32 + hh + e);
+                acc[j][hh + e] = fmaf(__uint_as_float(v[e]), c.x, acc[j][hh + e]);
+                acc[j][hh + e + 1] = fmaf(__uint_as_float(v[e + 1]), c.y, acc[j][hh + e + 1]);
+                acc[j][hh + e + 2] = fmaf(__uint_as_float(v[e + 2]), c.z, acc[j][hh + e + 2]);
+                acc[j][hh + e + 3] = fmaf(__uint_as_float(v[e + 3]), c.w, acc[j][hh + e + 3]);
+              }
+            }
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(pempty + pb), 0));
+        if (++pb == NPBUF) {
+          pb = 0;
+          pphase ^= 1u;
+        }
+      }
+      if (!ok) break;
+
+      if (MODE == 1) {
+        // lanes 0-63 of the CTA hold w1.x (a), lanes 64-127 w3.x (u) of the
+        // same 64 features; warps q and q+2 of one half pair up through
+        // shared memory, each finishing 16 of the 32 columns of a chunk
+        const int pr = q & 1;
+        const bool is_a = q < 2;
+        float *buf_a = xbuf + (pr + 2 * half) * 2 * 32 * XB_STRIDE;
+        float *buf_u = buf_a + 32 * XB_STRIDE;
+        const int bar = 1 + pr + 2 * half;
+        const int f = t.ft * 128 + (int)rank * 64 + pr * 32 + lane;
+        bf16 *out = static_cast<bf16 *>(p.out);
+#pragma unroll
+        for (int j = 0; j < CHUNKS; ++j) {
+          const int c0 = (2 * j + half) * 32;
+          if (c0 >= t.nvalid) continue;
+          float *mine = is_a ? buf_a : buf_u;
+#pragma unroll
+          for (int e = 0; e < 16; ++e) mine[lane * XB_STRIDE + e] = is_a ? acc[j][16 + e] : acc[j][e];
+          named_bar_sync(bar, 64);
+          const float *other = is_a ? buf_u : buf_a;
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const int col = is_a ? e : 16 + e;
+            const float a = is_a ? acc[j][e] : other[lane * XB_STRIDE + e];
+            const float u = is_a ? other[lane * XB_STRIDE + e] : acc[j][16 + e];
+            if (c0 + col < t.nvalid)
+              out[(size_t)(row0 + c0 + col) * p.I + f] = __float2bfloat16_rn(swiglu_h(a, u));
+          }
+          named_bar_sync(bar, 64);
+        }
+      } else if (MODE == 2) {
+        float *out;
+        size_t r0;
+        if (t.g < p.E) {
+          out = static_cast<float *>(p.out);
+          r0 = (size_t)row0;
+        } else {
+          out = p.out_shared;
+          r0 = (size_t)(t.g - p.E) * p.T + t.n0;
+        }
+        const int d = t.ft * 256 + (int)rank * BM + q * 32 + lane;
+#pragma unroll
+        for (int j = 0; j < CHUNKS; ++j) {
+          const int c0 = (2 * j + half) * 32;
+#pragma unroll
+          for (int e = 0; e < 32; ++e)
+            if (c0 + e < t.nvalid) out[(r0 + c0 + e) * p.D + d] = acc[j][e];
+        }
+      } else {
+        // weighted scatter into y (gate 1 for the shared expert)
+        int32_t *s_tok = reinterpret_cast<int32_t *>(xbuf);
+        float *s_gate = reinterpret_cast<float *>(s_tok + BN_MAX);
+        const int et = threadIdx.x - 64;
+        named_bar_sync(5, 32 * EPI);  // the previous tile's readers are done
+        for (int c = et; c < t.nvalid; c += 32 * EPI) {
+          int tok;
+          float gate = 1.0f;
+          if (t.g < p.E) {
+            tok = p.sorted_token[row0 + c];
+            for (int jj = 0; jj < p.k; ++jj)
+              if (p.indices[(size_t)tok * p.k + jj] == t.g) gate = p.weights[(size_t)tok * p.k + jj];
+          } else {
+            tok = t.n0 + c;
+          }
+          s_tok[c] = tok;
+          s_gate[c] = gate;
+        }
+        named_bar_sync(5, 32 * EPI);
+        const int d = t.ft * 256 + (int)rank * BM + q * 32 + lane;
+#pragma unroll
+        for (int j = 0; j < CHUNKS; ++j) {
+          const int c0 = (2 * j + half) * 32;
+#pragma unroll
+          for (int e = 0; e < 32; ++e)
+            if (c0 + e < t.nvalid)
+              atomicAdd(p.y + (size_t)s_tok[c0 + e] * p.D + d, s_gate[c0 + e] * acc[j][e]);
+        }
+      }
+    }
+  }
+
+  __syncthreads();
+  if (threadIdx.x == 0 && *abort_flag) {
+    // a stalled pipeline stopped early: let copies already issued land (the
+    // leader's full barriers count both CTAs' copies)
+    if (leader) {
+      for (int s = 0; s < STAGES; ++s)
+        if (pending[s] >= 0) drain_wait(full + s, (uint32_t)pending[s], p.timeout_ns);
+    } else {
+      sleep_ns(200000);
+    }
+  }
+  __syncthreads();
+  cluster_sync();  // neither CTA leaves while the other may touch its memory
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, 512);
+  }
+}
+
+}  // namespace f8
+
 // ----------------------------------------------------------- CUDA-core path
 
 __device__ __forceinline__ float ld_f(const float *p, size_t i) { return p[i]; }
@@ -1007,6 +1463,9 @@ int sm_count() {
 struct WsLayout {
   size_t tab, xperm, h, total;
   int64_t rows_pad;
+  // FP8 x FP8 path (e4m3 weights): e4m3 codes and transposed 1 x 128 block
+  // scales of the expert rows (xq, xs) and of h (hq, hs), and h in bf16 (hb)
+  size_t xq, xs, hb, hq, hs;
 };
 
 constexpr int ROW_PAD = 256;  // spare rows so a TMA box never starts past a buffer
@@ -1028,6 +1487,22 @@ WsLayout ws_layout(const moe_cfg *c, int64_t T, moe_dtype x_dt, moe_dtype w_dt) 
   l.h = off;
   off = align_up(off + (size_t)l.rows_pad * c->inter * (tc ? 2 : 4), 1024);
   l.total = off;
+  l.xq = l.xs = l.hb = l.hq = l.hs = 0;
+  if (tc && w_dt == MOE_E4M3) {
+    size_t o = align_up(sizeof(int32_t) * (size_t)(4 * G + 4), 1024);
+    const size_t rp = (size_t)l.rows_pad;
+    l.xq = o;
+    o = align_up(o + rp * c->dim, 1024);
+    l.xs = o;
+    o = align_up(o + (size_t)(c->dim / 128) * rp * 4, 1024);
+    l.hb = o;
+    o = align_up(o + rp * c->inter * 2, 1024);
+    l.hq = o;
+    o = align_up(o + rp * c->inter, 1024);
+    l.hs = o;
+    o = align_up(o + (size_t)(c->inter / 128) * rp * 4, 1024);
+    if (o > l.total) l.total = o;
+  }
   return l;
 }
 
@@ -1066,6 +1541,41 @@ moe_status launch_tc(const CUtensorMap &a0, const CUtensorMap &a1, const CUtenso
       pairs = active;
     cfg.gridDim = dim3(2 * pairs);
   }
+  if (cudaLaunchKernelEx(&cfg, kern, a0, a1, b, p) != cudaSuccess) return MOE_ERR_CUDA;
+  return launch_status();
+}
+
+template <int MODE, int STAGES>
+moe_status launch_fp8(const CUtensorMap &a0, const CUtensorMap &a1, const CUtensorMap &b,
+                      const tc::Params &p, cudaStream_t s) {
+  using L = f8::Layout<STAGES>;
+  auto kern = f8::tc_fp8_gemm<MODE, STAGES>;
+  const size_t smem = L::smem_bytes(p.G, p.E);
+  if (smem > 232448) return MOE_ERR_UNSUPPORTED;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+      cudaSuccess)
+    return MOE_ERR_CUDA;
+  const int nsm = sm_count();
+  if (nsm < 2) return MOE_ERR_CUDA;
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  cfg.blockDim = dim3(f8::NT);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  // one persistent pair per co-resident SM pair
+  int pairs = nsm / 2;
+  cfg.gridDim = dim3(2 * pairs);
+  int active = 0;
+  if (cudaOccupancyMaxActiveClusters(&active, kern, &cfg) == cudaSuccess && active > 0 &&
+      active < pairs)
+    pairs = active;
+  cfg.gridDim = dim3(2 * pairs);
   if (cudaLaunchKernelEx(&cfg, kern, a0, a1, b, p) != cudaSuccess) return MOE_ERR_CUDA;
   return launch_status();
 }
@@ -1125,6 +1635,8 @@ tc::Params tc_params(const Job &j) {
   p.y = j.y;
   p.sA0 = nullptr;
   p.sA1 = nullptr;
+  p.sX = nullptr;
+  p.ld_sx = 0;
   return p;
 }
 
@@ -1206,6 +1718,96 @@ moe_status tc_down(const Job &j) {
     st = launch_tc<3, CG, AT, BN_MAX, BOXN, STAGES, F8>(mw2, mw2, mh, p, j.s);
   else
     st = launch_tc<2, CG, AT, BN_MAX, BOXN, STAGES, F8>(mw2, mw2, mh, p, j.s);
+  prof(4, j.s);
+  return st;
+}
+
+// ring depth of the FP8 x FP8 GEMMs: 32 KB per stage (16 KB of weight codes,
+// 128 token rows of 128 codes)
+#ifndef MOE_F8_STAGES
+#define MOE_F8_STAGES 6
+#endif
+
+bool e4m3_tmap(CUtensorMap *m, const void *base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+  return make_tmap(m, base, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, rows, cols, box_rows, 128);
+}
+
+moe_status quantise_rows(const Job &j, const void *src, bool gather, size_t q_off, size_t s_off,
+                         int K) {
+  const int rows = j.rows_total();
+  const unsigned grid = (unsigned)((rows + 31) / 32);
+  const size_t smem = (size_t)(K / 128) * 32 * sizeof(float);
+  uint32_t *q = reinterpret_cast<uint32_t *>(j.ws + q_off);
+  float *sc = reinterpret_cast<float *>(j.ws + s_off);
+  if (gather)
+    quant_rows_e4m3<true><<<grid, 256, smem, j.s>>>(static_cast<const uint2 *>(src),
+                                                    j.sorted_token, q, sc, j.rows_routed(), rows,
+                                                    (int)j.T, K, (int)j.l.rows_pad);
+  else
+    quant_rows_e4m3<false><<<grid, 256, smem, j.s>>>(static_cast<const uint2 *>(src), nullptr, q,
+                                                     sc, j.rows_routed(), rows, (int)j.T, K,
+                                                     (int)j.l.rows_pad);
+  return launch_status();
+}
+
+moe_status fp8_up(const Job &j) {
+  const int G = j.G(), D = j.c->dim, I = j.c->inter;
+  int32_t *tab = j.tab();
+  Tiling t1{f8::BN_MAX, I / 128, tab, tab + (G + 1)};
+  Tiling none{0, 0, nullptr, nullptr};
+  prep_tiles<<<1, 32, 0, j.s>>>(j.offsets, j.E(), G, (int)j.T, t1, none);
+  moe_status st = launch_status();
+  if (st != MOE_OK) return st;
+  prof(0, j.s);
+  if ((st = quantise_rows(j, j.x, true, j.l.xq, j.l.xs, D)) != MOE_OK) return st;
+  CUtensorMap mw1, mw3, mx;
+  if (!e4m3_tmap(&mw1, j.w->w1, (uint64_t)G * I, D, 64) ||
+      !e4m3_tmap(&mw3, j.w->w3, (uint64_t)G * I, D, 64) ||
+      !e4m3_tmap(&mx, j.ws + j.l.xq, (uint64_t)j.l.rows_pad, D, f8::BOXN))
+    return MOE_ERR_CUDA;
+  tc::Params p = tc_params(j);
+  p.tile_start = t1.tile_start;
+  p.tile_base = t1.tile_base;
+  p.KB = D / f8::BK;
+  p.out = j.ws + j.l.hb;
+  p.sA0 = j.w->s1;
+  p.sA1 = j.w->s3;
+  p.sX = reinterpret_cast<const float *>(j.ws + j.l.xs);
+  p.ld_sx = (int)j.l.rows_pad;
+  prof(1, j.s);
+  st = launch_fp8<1, MOE_F8_STAGES>(mw1, mw3, mx, p, j.s);
+  prof(2, j.s);
+  if (st != MOE_OK) return st;
+  // h (bf16) to e4m3 codes and scales for the second matmul
+  return quantise_rows(j, j.ws + j.l.hb, false, j.l.hq, j.l.hs, I);
+}
+
+moe_status fp8_down(const Job &j) {
+  const int G = j.G(), D = j.c->dim, I = j.c->inter;
+  int32_t *tab = j.tab();
+  Tiling t2{f8::BN_MAX, D / 256, tab + (2 * G + 1), tab + (3 * G + 2)};
+  Tiling none{0, 0, nullptr, nullptr};
+  prep_tiles<<<1, 32, 0, j.s>>>(j.offsets, j.E(), G, (int)j.T, t2, none);
+  moe_status st = launch_status();
+  if (st != MOE_OK) return st;
+  CUtensorMap mw2, mh;
+  if (!e4m3_tmap(&mw2, j.w->w2, (uint64_t)G * D, I, f8::BM) ||
+      !e4m3_tmap(&mh, j.ws + j.l.hq, (uint64_t)j.l.rows_pad, I, f8::BOXN))
+    return MOE_ERR_CUDA;
+  tc::Params p = tc_params(j);
+  p.tile_start = t2.tile_start;
+  p.tile_base = t2.tile_base;
+  p.KB = I / f8::BK;
+  p.out = j.out_perm;
+  p.sA0 = j.w->s2;
+  p.sA1 = j.w->s2;
+  p.sX = reinterpret_cast<const float *>(j.ws + j.l.hs);
+  p.ld_sx = (int)j.l.rows_pad;
+  prof(3, j.s);
+  if (j.y)
+    st = launch_fp8<3, MOE_F8_STAGES>(mw2, mw2, mh, p, j.s);
+  else
+    st = launch_fp8<2, MOE_F8_STAGES>(mw2, mw2, mh, p, j.s);
   prof(4, j.s);
   return st;
 }
@@ -1354,12 +1956,14 @@ moe_status run_down_t(const Job &j) {
 }
 
 moe_status run_up(const Job &j) {
+  if (j.w->act_e4m3) return fp8_up(j);
   if (tc_path(j.c, j.x_dt, j.w->w_dt))
     return j.w->w_dt == MOE_E4M3 ? run_up_t<true>(j) : run_up_t<false>(j);
   return j.x_dt == MOE_BF16 ? simt_up_x<bf16>(j) : simt_up_x<float>(j);
 }
 
 moe_status run_down(const Job &j) {
+  if (j.w->act_e4m3) return fp8_down(j);
   if (tc_path(j.c, j.x_dt, j.w->w_dt))
     return j.w->w_dt == MOE_E4M3 ? run_down_t<true>(j) : run_down_t<false>(j);
   return simt_down_w(j);
@@ -1385,7 +1989,10 @@ moe_status make_job(Job &j, const moe_cfg *cfg, int64_t T, const void *x, moe_dt
     if (!w->s1 || !w->s3 || !w->s2) return MOE_ERR_INVALID;
     if (cfg->dim % 128 != 0 || cfg->inter % 128 != 0) return MOE_ERR_UNSUPPORTED;
   }
-  if (w->act_e4m3) return MOE_ERR_UNSUPPORTED;
+  if (w->act_e4m3 != 0 && w->act_e4m3 != 1) return MOE_ERR_INVALID;
+  if (w->act_e4m3 && (w->w_dt != MOE_E4M3 || x_dt != MOE_BF16 || cfg->dim % 256 != 0 ||
+                      cfg->inter % 128 != 0))
+    return MOE_ERR_UNSUPPORTED;
   j.l = ws_layout(cfg, T, x_dt, w->w_dt);
   if (ws_bytes < j.l.total) return MOE_ERR_WORKSPACE;
   j.c = cfg;
@@ -1476,6 +2083,23 @@ MOE_EXPORT moe_status moe_experts_forward_combine(const moe_cfg *cfg, int64_t T,
     return MOE_ERR_CUDA;
   if ((st = run_up(j)) != MOE_OK) return st;
   return run_down(j);
+}
+
+MOE_EXPORT moe_status moe_quantize_e4m3_rows(const void *src, int64_t rows, int32_t K,
+                                             uint8_t *q, float *scales, int64_t ld,
+                                             moe_stream_t stream) {
+  if (rows < 0 || rows >= ((int64_t)1 << 31) || K <= 0 || K % 128 != 0 || ld < rows ||
+      ld >= ((int64_t)1 << 31))
+    return MOE_ERR_INVALID;
+  if (rows == 0) return MOE_OK;
+  if (!src || !q || !scales) return MOE_ERR_INVALID;
+  const unsigned grid = (unsigned)((rows + 31) / 32);
+  const size_t smem = (size_t)(K / 128) * 32 * sizeof(float);
+  if (smem > 48 * 1024) return MOE_ERR_UNSUPPORTED;
+  quant_rows_e4m3<false><<<grid, 256, smem, as_stream(stream)>>>(
+      static_cast<const uint2 *>(src), nullptr, reinterpret_cast<uint32_t *>(q), scales, 0,
+      (int)rows, 0, K, (int)ld);
+  return launch_status();
 }
 
 MOE_EXPORT moe_status moe_experts_set_profile_events(void *const *events, int32_t n) {

@@ -208,6 +208,21 @@ def combine(shape: BlockShape, weights: torch.Tensor, slot_of: torch.Tensor,
     return y
 
 
+def quantize_e4m3_rows(src: torch.Tensor):
+    """moe_quantize_e4m3_rows: (codes [rows, K] uint8, scales [K/128, rows] fp32)
+    of a bf16 [rows, K] matrix, 1 x 128 blocks."""
+    _check_cuda(src)
+    if src.dtype != torch.bfloat16 or src.dim() != 2:
+        raise ValueError("src must be a 2-D bf16 tensor")
+    rows, K = src.shape
+    q = torch.empty(rows, K, dtype=torch.uint8, device=src.device)
+    sc = torch.empty(K // 128, rows, dtype=torch.float32, device=src.device)
+    check(fn("moe_experts", "moe_quantize_e4m3_rows")(src.data_ptr(), rows, K, q.data_ptr(),
+                                                      sc.data_ptr(), rows, _stream()),
+          "moe_quantize_e4m3_rows")
+    return q, sc
+
+
 def selftest_wait(limit_ns: int, status: torch.Tensor) -> None:
     check(fn("moe_experts", "moe_experts_selftest_wait")(limit_ns, status.data_ptr(), _stream()),
           "moe_experts_selftest_wait")
@@ -302,8 +317,9 @@ class MoEBlock:
         tc_experts = (self.x_dtype == torch.bfloat16 and sh.dim % 128 == 0
                       and sh.inter % 128 == 0
                       and self.p.w1.dtype in (torch.bfloat16, torch.uint8, torch.float8_e4m3fn))
+        # the FP8 x FP8 path adds the quantisation of h (six expert launches)
         return ((2 if tc_router and self.router_prep is not None else 3 if tc_router else 2)
-                + 3 + (5 if tc_experts else 4)
+                + 3 + (6 if self.fp8_act else 5 if tc_experts else 4)
                 + (1 if self.combine_mode == "ordered" else 0))
 
     def _router(self, x, cfgp, s):

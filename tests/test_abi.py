@@ -151,6 +151,25 @@ def test_experts_validation():
               None) == 0
 
 
+def test_fp8_activation_path_validation():
+    f = fn("moe_experts", "moe_experts_forward")
+    c = v3_cfg()
+    call = lambda cfg, wt, x_dt=1: f(ctypes.byref(cfg), 8, P, x_dt, ctypes.byref(wt), P, P, P, P,
+                                     P, 1 << 40, None, None)
+    fp8 = lambda act: MoEExpertWeights(0x1000, 0x1000, 0x1000, 2, 0x1000, 0x1000, 0x1000, act)
+    assert call(c, fp8(2)) == INVALID                          # the flag is 0 or 1
+    bf = MoEExpertWeights(0x1000, 0x1000, 0x1000, 1, None, None, None, 1)
+    assert call(c, bf) == UNSUPPORTED                          # e4m3 weights only
+    assert call(c, fp8(1), x_dt=0) == UNSUPPORTED              # bf16 activations in
+    assert call(v3_cfg(dim=7296), fp8(1)) == UNSUPPORTED       # dim % 256 != 0
+    q = fn("moe_experts", "moe_quantize_e4m3_rows")
+    assert q(P, 4, 100, P, P, 4, None) == INVALID              # K % 128 != 0
+    assert q(P, 4, 128, P, P, 3, None) == INVALID              # ld < rows
+    assert q(None, 4, 128, P, P, 4, None) == INVALID
+    assert q(P, -1, 128, P, P, 4, None) == INVALID
+    assert q(None, 0, 128, None, None, 0, None) == 0           # nothing to do
+
+
 def test_combine_and_selftest_validation():
     f = fn("moe_combine", "moe_combine")
     c = v3_cfg()

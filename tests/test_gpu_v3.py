@@ -28,8 +28,15 @@ from sparse_moe_layer_sum_b200.inputs import WORKLOADS, make_block, sample_token
 pytestmark = pytest.mark.gpu
 
 TOL = {"bf16": 2e-2, "e4m3": 5e-2}
-# per-expert rows: max |d| / rms(expert output) (the same bounds) and mean
-MEAN_TOL = {"bf16": 2e-4, "e4m3": 1e-3}
+# per-expert rows: max |d| / rms(expert output) (the same bounds) and the
+# mean.  At dim 7168 the kernel's fp32 h (tensor-core accumulation over 7168
+# terms, silu with the hardware exp2) differs from the oracle's fp64 h by
+# about 2e-5 relative, so about 2 * 2e-5 / 2^-8 = 1% of the h elements round
+# to the neighbouring bf16 value; over the 2048 terms of an output that is
+# sqrt(0.01) * 2^-8 / sqrt(3) = 2.3e-4 rms, a mean |error| near 1.8e-4 rms
+# (measured 1.8e-4 to 2.0e-4).  The bound is 2.5 times that.  e4m3 weights
+# add the fp16 roundings of the expanded weights (about 4.5e-4).
+MEAN_TOL = {"bf16": 5e-4, "e4m3": 1.5e-3}
 CASES = ["v3_decode_t64", "v3_prefill_t4096", "v3_skew_t16384", "v3_fp8_t8192"]
 N_Y = 64
 
