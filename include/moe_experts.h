@@ -100,6 +100,48 @@ moe_status moe_experts_forward_combine(const moe_cfg *cfg, int64_t T, const void
                                        moe_stream_t stream);
 
 /*
+ * Expert parallelism: the experts split over `world` ranks (GPUs), as the
+ * moe-init excerpt of "DeepSeek-V3.2-Exp · Mixture of experts" splits them
+ * (n_local_experts = n_routed / world_size, experts_start_idx = rank *
+ * n_local_experts) and the moe-forward excerpt sums the ranks' partial
+ * outputs (dist.all_reduce(y)).  Rank r runs the routed experts
+ * [r * E / world, (r + 1) * E / world) on the tokens routed to them, and the
+ * shared expert on its slice of the tokens [floor(r * T / world),
+ * floor((r + 1) * T / world)) -- every shared-expert row is computed by
+ * exactly one rank, so the sum over ranks is the block output.  The router
+ * and the dispatch run on every rank on the full batch (x is replicated).
+ */
+typedef struct {
+  int32_t rank, world;
+} moe_ep_shard;
+
+/*
+ * The shard of `shard->rank`: out[0..3] = first and end routed expert, first
+ * and end token of the shared expert's slice.  Host only (no device call).
+ * Returns MOE_ERR_INVALID for a bad config, T < 0 or rank outside
+ * [0, world), MOE_ERR_UNSUPPORTED when world does not divide n_routed.
+ */
+moe_status moe_ep_plan(const moe_cfg *cfg, int64_t T, const moe_ep_shard *shard, int32_t *out);
+
+/*
+ * moe_experts_forward_combine for one expert-parallel rank: y (zeroed
+ * first) receives the rank's partial sum, gate * expert output for the
+ * routed rows of its experts plus the shared expert's output on its token
+ * slice; the caller adds the ranks' y (an all-reduce).  w holds only the
+ * rank's weights: its n_routed / world routed experts in order, then the
+ * shared expert ([n_routed / world + n_shared, ...] stacked as above).
+ * offsets, sorted_token, indices and weights are those of the whole batch.
+ * Limits and errors as moe_experts_forward_combine and moe_ep_plan.
+ */
+moe_status moe_experts_forward_combine_ep(const moe_cfg *cfg, int64_t T, const void *x,
+                                          moe_dtype x_dt, const moe_expert_weights *w,
+                                          const moe_ep_shard *shard, const int32_t *offsets,
+                                          const int32_t *sorted_token, const int32_t *indices,
+                                          const float *weights, float *y, void *ws,
+                                          size_t ws_bytes, int32_t *dev_status,
+                                          moe_stream_t stream);
+
+/*
  * The two halves of moe_experts_forward, for callers that schedule them
  * separately (moe_experts_forward(...) == moe_experts_up(...) followed by
  * moe_experts_down(...) on the same stream and workspace).

@@ -38,6 +38,12 @@ class MoEExpertWeights(ctypes.Structure):
     ]
 
 
+class MoEEpShard(ctypes.Structure):
+    """Mirror of moe_ep_shard in include/moe_experts.h."""
+
+    _fields_ = [("rank", ctypes.c_int32), ("world", ctypes.c_int32)]
+
+
 _vp, _i32, _i64, _sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
 _cfgp = ctypes.POINTER(MoECfg)
 
@@ -62,6 +68,11 @@ SIGNATURES = {
     ("moe_experts", "moe_experts_forward_combine"): (
         _i32, [_cfgp, _i64, _vp, _i32, ctypes.POINTER(MoEExpertWeights), _vp, _vp, _vp, _vp, _vp,
                _vp, _sz, _vp, _vp]),
+    ("moe_experts", "moe_ep_plan"): (
+        _i32, [_cfgp, _i64, ctypes.POINTER(MoEEpShard), ctypes.POINTER(ctypes.c_int32)]),
+    ("moe_experts", "moe_experts_forward_combine_ep"): (
+        _i32, [_cfgp, _i64, _vp, _i32, ctypes.POINTER(MoEExpertWeights),
+               ctypes.POINTER(MoEEpShard), _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp, _vp]),
     ("moe_experts", "moe_experts_up"): (
         _i32, [_cfgp, _i64, _vp, _i32, ctypes.POINTER(MoEExpertWeights), _vp, _vp, _vp, _sz, _vp,
                _vp]),

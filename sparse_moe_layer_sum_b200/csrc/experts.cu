@@ -36,6 +36,8 @@
 #include <cuda_fp8.h>
 #include <cudaTypedefs.h>
 #include <math.h>
+#include <stdio.h>
+#include <stdlib.h>
 
 #include "common.cuh"
 #include "moe_experts.h"
@@ -70,9 +72,23 @@ __device__ __forceinline__ void group_tiles(int n, int rows_max, int &base, int 
   ntt = (n + base - 1) / base;
 }
 
+// The part of the experts' work one call runs: routed experts [e0, e1) and
+// the shared expert on tokens [st0, st1).  A single-GPU call runs all of it;
+// an expert-parallel rank runs its own experts and its slice of the tokens.
+struct Shard {
+  int e0, e1, st0, st1;
+};
+
+// Rows of group g in this call: an expert's tokens when it is one of the
+// call's experts, else none; the shared expert's token slice.
+__device__ __forceinline__ int group_rows(int g, const int32_t *off, int E, const Shard &sh) {
+  if (g < E) return g >= sh.e0 && g < sh.e1 ? off[g + 1] - off[g] : 0;
+  return sh.st1 - sh.st0;
+}
+
 // One warp: lane l owns a contiguous run of groups.
 __global__ void __launch_bounds__(32) prep_tiles(const int32_t *__restrict__ offsets, int E,
-                                                 int G, int T, Tiling t0, Tiling t1) {
+                                                 int G, Shard sh, Tiling t0, Tiling t1) {
   const int lane = threadIdx.x;
   const int per = (G + 31) / 32;
   const int g0 = min(G, lane * per), g1 = min(G, g0 + per);
@@ -81,7 +97,7 @@ __global__ void __launch_bounds__(32) prep_tiles(const int32_t *__restrict__ off
     if (!tl.tile_start) continue;
     int local = 0;
     for (int g = g0; g < g1; ++g) {
-      const int n = g < E ? offsets[g + 1] - offsets[g] : T;
+      const int n = group_rows(g, offsets, E, sh);
       int base, ntt;
       group_tiles(n, tl.rows_max, base, ntt);
       tl.tile_base[g] = base;
@@ -95,7 +111,7 @@ __global__ void __launch_bounds__(32) prep_tiles(const int32_t *__restrict__ off
     }
     int run = inc - local;
     for (int g = g0; g < g1; ++g) {
-      const int n = g < E ? offsets[g + 1] - offsets[g] : T;
+      const int n = group_rows(g, offsets, E, sh);
       int base, ntt;
       group_tiles(n, tl.rows_max, base, ntt);
       tl.tile_start[g] = run;
@@ -105,8 +121,11 @@ __global__ void __launch_bounds__(32) prep_tiles(const int32_t *__restrict__ off
   }
 }
 
+// g: group (routed expert, then the shared expert); wg: its index in the
+// call's weight tensors (the call's experts e0.. first, then the shared one);
+// tok0: first token of a shared-expert tile.
 struct Tile {
-  int g, ft, tt, ntt, n0, nvalid, rowbase;
+  int g, wg, ft, tt, ntt, n0, nvalid, rowbase, tok0;
 };
 
 // First k-block of a tile.  Tiles that run at the same time share operands
@@ -120,7 +139,7 @@ __device__ __forceinline__ int k_rotation(const Tile &t, int KB) { return (t.ft 
 // buffers (routed: offsets[g]; shared: after the T*k routed rows).
 __device__ __forceinline__ Tile decode_tile(int tile, const int32_t *tstart, const int32_t *tbase,
                                             const int32_t *off, int G, int E, int T,
-                                            int rows_routed) {
+                                            int rows_routed, const Shard &sh) {
   int lo = 0, hi = G;
   while (hi - lo > 1) {
     const int mid = (lo + hi) >> 1;
@@ -131,7 +150,8 @@ __device__ __forceinline__ Tile decode_tile(int tile, const int32_t *tstart, con
   }
   Tile t;
   t.g = lo;
-  const int n = lo < E ? off[lo + 1] - off[lo] : T;
+  t.wg = lo < E ? lo - sh.e0 : (sh.e1 - sh.e0) + (lo - E);
+  const int n = group_rows(lo, off, E, sh);
   const int base = tbase[lo];
   const int ntt = (n + base - 1) / base;
   const int local = tile - tstart[lo];
@@ -140,7 +160,8 @@ __device__ __forceinline__ Tile decode_tile(int tile, const int32_t *tstart, con
   t.ntt = ntt;
   t.n0 = t.tt * base;
   t.nvalid = min(base, n - t.n0);
-  t.rowbase = lo < E ? off[lo] : rows_routed + (lo - E) * T;
+  t.rowbase = lo < E ? off[lo] : rows_routed + (lo - E) * T + sh.st0;
+  t.tok0 = sh.st0 + t.n0;
   return t;
 }
 
@@ -148,13 +169,24 @@ __device__ __forceinline__ Tile decode_tile(int tile, const int32_t *tstart, con
 
 // X_perm[p] = x[sorted_token[p]] for p < rows_routed, then x itself for the
 // shared expert's rows.  One warp per row, 16-byte vectors.
+// Whether row p of the expert-contiguous buffers belongs to this call's share
+// (every row when the call is not sharded: off == NULL).
+__device__ __forceinline__ bool row_in_shard(int row, int rows_routed, int T,
+                                             const int32_t *off, const Shard &sh) {
+  if (!off) return true;
+  if (row < rows_routed) return row >= off[sh.e0] && row < off[sh.e1];
+  const int t = (row - rows_routed) % T;
+  return t >= sh.st0 && t < sh.st1;
+}
+
 __global__ void __launch_bounds__(256) gather_rows(const uint4 *__restrict__ x,
                                                    const int32_t *__restrict__ sorted_token,
                                                    uint4 *__restrict__ xp, int rows_routed,
-                                                   int rows_total, int T, int vec_per_row) {
+                                                   int rows_total, int T, int vec_per_row,
+                                                   const int32_t *off, Shard sh) {
   const int row = (int)((blockIdx.x * (size_t)blockDim.x + threadIdx.x) / 32);
   const int lane = threadIdx.x % 32;
-  if (row >= rows_total) return;
+  if (row >= rows_total || !row_in_shard(row, rows_routed, T, off, sh)) return;
   const int src = row < rows_routed ? sorted_token[row] : (row - rows_routed) % T;
   const uint4 *s = x + (size_t)src * vec_per_row;
   uint4 *d = xp + (size_t)row * vec_per_row;
@@ -166,10 +198,11 @@ __global__ void __launch_bounds__(256) gather_rows(const uint4 *__restrict__ x,
 __global__ void __launch_bounds__(256) gather_rows_f16(const __nv_bfloat162 *__restrict__ x,
                                                        const int32_t *__restrict__ sorted_token,
                                                        __half2 *__restrict__ xp, int rows_routed,
-                                                       int rows_total, int T, int pairs_per_row) {
+                                                       int rows_total, int T, int pairs_per_row,
+                                                       const int32_t *off, Shard sh) {
   const int row = (int)((blockIdx.x * (size_t)blockDim.x + threadIdx.x) / 32);
   const int lane = threadIdx.x % 32;
-  if (row >= rows_total) return;
+  if (row >= rows_total || !row_in_shard(row, rows_routed, T, off, sh)) return;
   const int src = row < rows_routed ? sorted_token[row] : (row - rows_routed) % T;
   const __nv_bfloat162 *s = x + (size_t)src * pairs_per_row;
   __half2 *d = xp + (size_t)row * pairs_per_row;
@@ -226,6 +259,7 @@ struct Params {
   // [K / 128][ld_sx] (row r's scale for k-block kb at kb * ld_sx + r)
   const float *sX;
   int ld_sx;
+  Shard sh;
 };
 
 // CG = CTA group: 1 = one SM per tile; 2 = an SM pair per tile (cta_group::2),
@@ -393,15 +427,15 @@ __global__ void __launch_bounds__(threads_of(F8, AT), 1)
       uint32_t phase = 0;
       bool ok = true;
       for (int tile = unit; ok && tile < total; tile += nunits) {
-        const Tile t = decode_tile(tile, s_tstart, s_tbase, s_off, p.G, p.E, p.T, p.rows_routed);
+        const Tile t = decode_tile(tile, s_tstart, s_tbase, s_off, p.G, p.E, p.T, p.rows_routed, p.sh);
         const uint64_t pol_w = t.ntt > 1 ? pol_normal : pol_first;
         const int nmma = (t.nvalid + 15) & ~15;
         const int brows = nmma / CG;  // this CTA's share of the token rows
         const int b0 = t.rowbase + t.n0 + (int)rank * brows;
         // first weight row of this CTA's part 0; part i of GEMM2 lies
         // i * 128 * CG rows further, GEMM1's part 1 is w3 at the same rows
-        const int arow = MODE == 1 ? t.g * p.I + t.ft * L::FEAT + (int)rank * L::PART_ROWS
-                                   : t.g * p.D + t.ft * L::FEAT + (int)rank * BM;
+        const int arow = MODE == 1 ? t.wg * p.I + t.ft * L::FEAT + (int)rank * L::PART_ROWS
+                                   : t.wg * p.D + t.ft * L::FEAT + (int)rank * BM;
         const int nbox = (brows + BOXN - 1) / BOXN;
         // with e4m3 weights the full barrier counts only the token rows; the
         // weight tile arrives on this CTA's own a8_full barrier
@@ -469,7 +503,7 @@ __global__ void __launch_bounds__(threads_of(F8, AT), 1)
       uint32_t phase = 0, acc_phase = 0;
       bool ok = true;
       for (int tile = unit; ok && tile < total; tile += nunits) {
-        const Tile t = decode_tile(tile, s_tstart, s_tbase, s_off, p.G, p.E, p.T, p.rows_routed);
+        const Tile t = decode_tile(tile, s_tstart, s_tbase, s_off, p.G, p.E, p.T, p.rows_routed, p.sh);
         if (!wait_bounded(acce + acc, acc_phase ^ 1u, abort_flag, p.timeout_ns, p.status)) {
           ok = false;
           break;
@@ -544,11 +578,11 @@ __global__ void __launch_bounds__(threads_of(F8, AT), 1)
       uint32_t phase = 0;
       bool ok = true;
       for (int tile = unit; ok && tile < total; tile += nunits) {
-        const Tile t = decode_tile(tile, s_tstart, s_tbase, s_off, p.G, p.E, p.T, p.rows_routed);
+        const Tile t = decode_tile(tile, s_tstart, s_tbase, s_off, p.G, p.E, p.T, p.rows_routed, p.sh);
         // scale rows of part 0 and part 1 (GEMM1: w1 and w3 at the same
         // rows; GEMM2 with two parts: 128 * CG rows apart)
         const int r0 = t.ft * L::FEAT + (int)rank * L::PART_ROWS;
-        const size_t srow = ((size_t)t.g * (rows_w / 128) + r0 / 128) * (cols_w / 128);
+        const size_t srow = ((size_t)t.wg * (rows_w / 128) + r0 / 128) * (cols_w / 128);
         const size_t srow1 =
             MODE != 1 && AT == 2 ? srow + (size_t)CG * (cols_w / 128) : srow;
         const float *sc1 = MODE == 1 ? p.sA1 : p.sA0;
@@ -635,7 +669,7 @@ __global__ void __launch_bounds__(threads_of(F8, AT), 1)
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int tile = unit; tile < total; tile += nunits) {
-      const Tile t = decode_tile(tile, s_tstart, s_tbase, s_off, p.G, p.E, p.T, p.rows_routed);
+      const Tile t = decode_tile(tile, s_tstart, s_tbase, s_off, p.G, p.E, p.T, p.rows_routed, p.sh);
       if (!wait_bounded(accf + acc, acc_phase, abort_flag, p.timeout_ns, p.status)) break;
       tc_fence_after();
       const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * L::ACC_COLS);
@@ -667,7 +701,7 @@ __global__ void __launch_bounds__(threads_of(F8, AT), 1)
             for (int jj = 0; jj < p.k; ++jj)
               if (p.indices[(size_t)tok * p.k + jj] == t.g) gate = p.weights[(size_t)tok * p.k + jj];
           } else {
-            tok = t.n0 + c;
+            tok = t.tok0 + c;
           }
           s_tok[c] = tok;
           s_gate[c] = gate;
@@ -696,7 +730,7 @@ __global__ void __launch_bounds__(threads_of(F8, AT), 1)
           row0 = (size_t)t.rowbase + t.n0;
         } else {
           out = p.out_shared;
-          row0 = (size_t)(t.g - p.E) * p.T + t.n0;
+          row0 = (size_t)(t.g - p.E) * p.T + t.tok0;
         }
 #pragma unroll
         for (int a = 0; a < AT; ++a) {
@@ -854,7 +888,8 @@ __global__ void __launch_bounds__(256) quant_rows_e4m3(const uint2 *__restrict__
                                                        const int32_t *__restrict__ sorted_token,
                                                        uint32_t *__restrict__ q,
                                                        float *__restrict__ sc, int rows_routed,
-                                                       int rows_total, int T, int K, int ld) {
+                                                       int rows_total, int T, int K, int ld,
+                                                       const int32_t *off, Shard sh) {
   extern __shared__ float s_sc[];  // [K / 128][32]
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int row0 = blockIdx.x * 32;
@@ -862,6 +897,7 @@ __global__ void __launch_bounds__(256) quant_rows_e4m3(const uint2 *__restrict__
   for (int rr = warp; rr < 32; rr += 8) {
     const int row = row0 + rr;
     if (row >= rows_total) break;
+    if (!row_in_shard(row, rows_routed, T, off, sh)) continue;
     const int srow = !GATHER ? row : row < rows_routed ? sorted_token[row] : row - rows_routed;
     const uint2 *s = src + (size_t)srow * (K / 4);
     uint32_t *d = q + (size_t)row * (K / 4);
@@ -901,7 +937,17 @@ constexpr int BM = 128;                // weight rows per CTA
 constexpr int BN_MAX = 256;            // token rows per tile (per SM pair)
 constexpr int BOXN = 32;               // token rows per TMA box
 constexpr int EPI = 8;                 // promotion / epilogue warps (two per TMEM lane quarter)
-constexpr int NT = 32 * (2 + EPI);
+// warpgroup 0: warp 0 TMA, warp 1 MMA, warps 2-3 idle; warpgroups 1-2: the
+// promotion / epilogue warps.  A thread's registers are split unevenly with
+// setmaxnreg: the block launches with REG_LAUNCH per thread (the most that
+// three warps per SM sub-partition allow), warpgroup 0 gives all but
+// REG_LOW back and the two epilogue warpgroups take REG_HIGH, which holds
+// their fp32 running sums (128 per thread) without spilling.  The shares
+// add up to the launch's total: 4 * 56 + 8 * 224 = 12 * 168 (per warp, x32).
+constexpr int EPI0 = 4;                // first epilogue warp
+constexpr int NT = 32 * (EPI0 + EPI);
+constexpr int REG_LAUNCH = 168, REG_LOW = 56, REG_HIGH = 224;
+static_assert(4 * REG_LOW + EPI * REG_HIGH == (NT / 32) * REG_LAUNCH, "register split");
 constexpr int A_BYTES = BM * BK;       // 16 KB
 constexpr int B_ROWS = BN_MAX / 2;     // token rows one CTA holds
 constexpr int B_BYTES = B_ROWS * BK;   // 16 KB
@@ -937,7 +983,7 @@ struct Layout {
 // added into y.  Warp 0 issues TMA loads, one thread of warp 1 the MMAs,
 // warps 2-9 promote the partial sums and run the epilogue.
 template <int MODE, int STAGES>
-__global__ void __maxnreg__(200)
+__global__ void __launch_bounds__(NT, 1)
     tc_fp8_gemm(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA1,
                 const __grid_constant__ CUtensorMap tmB, const tc::Params p) {
   using L = Layout<STAGES>;
@@ -997,8 +1043,10 @@ __global__ void __maxnreg__(200)
   const uint32_t tmem_base = *tmem_slot;
   const int total = s_tstart[p.G];
 
-  if (warp == 0) {
-    if (lane == 0) {
+  if (warp < EPI0) {
+    // warpgroup 0 as a whole gives registers back, then splits into roles
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(REG_LOW));
+    if (warp == 0 && lane == 0) {
       // ---------------------------------------------------- TMA producer
       // weights at normal L2 priority when their expert has several token
       // tiles (which then share them in L2), else evict-first in the second
@@ -1010,13 +1058,13 @@ __global__ void __maxnreg__(200)
       uint32_t phase = 0;
       bool ok = true;
       for (int tile = unit; ok && tile < total; tile += nunits) {
-        const Tile t = decode_tile(tile, s_tstart, s_tbase, s_off, p.G, p.E, p.T, p.rows_routed);
+        const Tile t = decode_tile(tile, s_tstart, s_tbase, s_off, p.G, p.E, p.T, p.rows_routed, p.sh);
         const uint64_t pol_w = t.ntt > 1 ? pol_normal : pol_first;
         const int nmma = (t.nvalid + 15) & ~15;
         const int brows = nmma / 2;
         const int b0 = t.rowbase + t.n0 + (int)rank * brows;
-        const int arow = MODE == 1 ? t.g * p.I + t.ft * 128 + (int)rank * 64
-                                   : t.g * p.D + t.ft * 256 + (int)rank * BM;
+        const int arow = MODE == 1 ? t.wg * p.I + t.ft * 128 + (int)rank * 64
+                                   : t.wg * p.D + t.ft * 256 + (int)rank * BM;
         const int nbox = (brows + BOXN - 1) / BOXN;
         const uint32_t bytes = (uint32_t)(A_BYTES + nbox * BOXN * BK);
         const int k0 = k_rotation(t, KB);
@@ -1046,15 +1094,13 @@ __global__ void __maxnreg__(200)
           }
         }
       }
-    }
-  } else if (warp == 1) {
-    if (lane == 0 && leader) {
+    } else if (warp == 1 && lane == 0 && leader) {
       // ------------------------------------------------------ MMA issuer
       int stage = 0, pb = 0;
       uint32_t phase = 0, pphase = 0;
       bool ok = true;
       for (int tile = unit; ok && tile < total; tile += nunits) {
-        const Tile t = decode_tile(tile, s_tstart, s_tbase, s_off, p.G, p.E, p.T, p.rows_routed);
+        const Tile t = decode_tile(tile, s_tstart, s_tbase, s_off, p.G, p.E, p.T, p.rows_routed, p.sh);
         const int nmma = (t.nvalid + 15) & ~15;
         const uint32_t idesc = idesc_e4m3_f32(2 * BM, nmma);
         for (int i = 0; i < KB; ++i) {
@@ -1091,23 +1137,24 @@ __global__ void __maxnreg__(200)
       }
     }
   } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(REG_HIGH));
     // ------------------------------------------- promotion and epilogue
-    const int q = warp & 3;           // TMEM lane quarter this warp may access
-    const int half = (warp - 2) >> 2;  // the two warps of a quarter take alternate chunks
-    float *comb = s_comb + (warp - 2) * CHUNKS * 32;
+    const int q = warp & 3;              // TMEM lane quarter this warp may access
+    const int half = (warp - EPI0) >> 2;  // the two warps of a quarter take alternate chunks
+    float *comb = s_comb + (warp - EPI0) * CHUNKS * 32;
     const uint32_t lane_base = tmem_base + ((uint32_t)(q * 32) << 16);
     int pb = 0;
     uint32_t pphase = 0;
     bool ok = true;
     for (int tile = unit; ok && tile < total; tile += nunits) {
-      const Tile t = decode_tile(tile, s_tstart, s_tbase, s_off, p.G, p.E, p.T, p.rows_routed);
+      const Tile t = decode_tile(tile, s_tstart, s_tbase, s_off, p.G, p.E, p.T, p.rows_routed, p.sh);
       const int row0 = t.rowbase + t.n0;
       // weight scales of this CTA's rows, one per k-block
       const float *sw;
       if (MODE == 1)
-        sw = (q < 2 ? p.sA0 : p.sA1) + ((size_t)t.g * (p.I / 128) + t.ft) * KB;
+        sw = (q < 2 ? p.sA0 : p.sA1) + ((size_t)t.wg * (p.I / 128) + t.ft) * KB;
       else
-        sw = p.sA0 + ((size_t)t.g * (p.D / 128) + t.ft * 2 + (int)rank) * KB;
+        sw = p.sA0 + ((size_t)t.wg * (p.D / 128) + t.ft * 2 + (int)rank) * KB;
       const float *sx = p.sX + row0 + lane;
       float acc[CHUNKS][32];
 #pragma unroll
@@ -1213,7 +1260,7 @@ __global__ void __maxnreg__(200)
           r0 = (size_t)row0;
         } else {
           out = p.out_shared;
-          r0 = (size_t)(t.g - p.E) * p.T + t.n0;
+          r0 = (size_t)(t.g - p.E) * p.T + t.tok0;
         }
         const int d = t.ft * 256 + (int)rank * BM + q * 32 + lane;
 #pragma unroll
@@ -1227,7 +1274,7 @@ __global__ void __maxnreg__(200)
         // weighted scatter into y (gate 1 for the shared expert)
         int32_t *s_tok = reinterpret_cast<int32_t *>(xbuf);
         float *s_gate = reinterpret_cast<float *>(s_tok + BN_MAX);
-        const int et = threadIdx.x - 64;
+        const int et = threadIdx.x - 32 * EPI0;
         named_bar_sync(5, 32 * EPI);  // the previous tile's readers are done
         for (int c = et; c < t.nvalid; c += 32 * EPI) {
           int tok;
@@ -1237,7 +1284,7 @@ __global__ void __maxnreg__(200)
             for (int jj = 0; jj < p.k; ++jj)
               if (p.indices[(size_t)tok * p.k + jj] == t.g) gate = p.weights[(size_t)tok * p.k + jj];
           } else {
-            tok = t.n0 + c;
+            tok = t.tok0 + c;
           }
           s_tok[c] = tok;
           s_gate[c] = gate;
@@ -1308,6 +1355,7 @@ struct SimtArgs {
   const float *weights;
   int k;
   float *y;
+  Shard sh;
 };
 
 template <typename XT, typename WT>
@@ -1319,10 +1367,10 @@ __global__ void __launch_bounds__(256) simt_gemm1(const XT *__restrict__ x, cons
   const int tile = blockIdx.x;
   if (tile >= a.tile_start[a.G]) return;
   const Tile t = decode_tile(tile, a.tile_start, a.tile_base, a.offsets, a.G, a.E, a.T,
-                             a.rows_routed);
+                             a.rows_routed, a.sh);
   if (threadIdx.x < ST) {
     const int r = threadIdx.x;
-    tok[r] = r < t.nvalid ? (t.g < a.E ? a.sorted_token[t.rowbase + t.n0 + r] : t.n0 + r) : -1;
+    tok[r] = r < t.nvalid ? (t.g < a.E ? a.sorted_token[t.rowbase + t.n0 + r] : t.tok0 + r) : -1;
   }
   const int r = threadIdx.x / 8, fq = (threadIdx.x % 8) * 4;
   float acc_a[4] = {0.f, 0.f, 0.f, 0.f}, acc_u[4] = {0.f, 0.f, 0.f, 0.f};
@@ -1333,8 +1381,8 @@ __global__ void __launch_bounds__(256) simt_gemm1(const XT *__restrict__ x, cons
       xs[rr][kk] = (tok[rr] >= 0 && kd < a.D) ? ld_f(x, (size_t)tok[rr] * a.D + kd) : 0.f;
       const int f = t.ft * ST + rr;
       const bool in = f < a.I && kd < a.D;
-      as_[rr][kk] = in ? w_at(w1, s1, t.g, f, kd, a.I, a.D) : 0.f;
-      us[rr][kk] = in ? w_at(w3, s3, t.g, f, kd, a.I, a.D) : 0.f;
+      as_[rr][kk] = in ? w_at(w1, s1, t.wg, f, kd, a.I, a.D) : 0.f;
+      us[rr][kk] = in ? w_at(w3, s3, t.wg, f, kd, a.I, a.D) : 0.f;
     }
     __syncthreads();
 #pragma unroll 8
@@ -1365,7 +1413,7 @@ __global__ void __launch_bounds__(256) simt_gemm2(const WT *w2, const float *s2,
   const int tile = blockIdx.x;
   if (tile >= a.tile_start[a.G]) return;
   const Tile t = decode_tile(tile, a.tile_start, a.tile_base, a.offsets, a.G, a.E, a.T,
-                             a.rows_routed);
+                             a.rows_routed, a.sh);
   const int r = threadIdx.x / 8, dq = (threadIdx.x % 8) * 4;
   float acc[4] = {0.f, 0.f, 0.f, 0.f};
   for (int k0 = 0; k0 < a.I; k0 += ST) {
@@ -1376,7 +1424,7 @@ __global__ void __launch_bounds__(256) simt_gemm2(const WT *w2, const float *s2,
                        ? a.h[((size_t)t.rowbase + t.n0 + rr) * a.I + ki]
                        : 0.f;
       const int d = t.ft * ST + rr;
-      ws[rr][kk] = (d < a.D && ki < a.I) ? w_at(w2, s2, t.g, d, ki, a.D, a.I) : 0.f;
+      ws[rr][kk] = (d < a.D && ki < a.I) ? w_at(w2, s2, t.wg, d, ki, a.D, a.I) : 0.f;
     }
     __syncthreads();
 #pragma unroll 8
@@ -1388,7 +1436,7 @@ __global__ void __launch_bounds__(256) simt_gemm2(const WT *w2, const float *s2,
   }
   if (r < t.nvalid) {
     if (a.y) {
-      int tok = t.n0 + r;
+      int tok = t.tok0 + r;
       float gate = 1.0f;
       if (t.g < a.E) {
         tok = a.sorted_token[t.rowbase + t.n0 + r];
@@ -1409,7 +1457,7 @@ __global__ void __launch_bounds__(256) simt_gemm2(const WT *w2, const float *s2,
       row = (size_t)t.rowbase + t.n0 + r;
     } else {
       out = a.out_shared;
-      row = (size_t)(t.g - a.E) * a.T + t.n0 + r;
+      row = (size_t)(t.g - a.E) * a.T + t.tok0 + r;
     }
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
@@ -1545,6 +1593,19 @@ moe_status launch_tc(const CUtensorMap &a0, const CUtensorMap &a1, const CUtenso
   return launch_status();
 }
 
+// MOE_ERR_CUDA for a failed runtime call; with MOE_DEBUG set in the
+// environment the call site and the runtime's error name go to stderr.
+moe_status cuda_fail(const char *where, cudaError_t e) {
+  if (getenv("MOE_DEBUG"))
+    fprintf(stderr, "moe_experts: %s: %s\n", where, cudaGetErrorName(e));
+  return MOE_ERR_CUDA;
+}
+
+moe_status checked_launch(const char *where) {
+  const cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? MOE_OK : cuda_fail(where, e);
+}
+
 template <int MODE, int STAGES>
 moe_status launch_fp8(const CUtensorMap &a0, const CUtensorMap &a1, const CUtensorMap &b,
                       const tc::Params &p, cudaStream_t s) {
@@ -1552,9 +1613,10 @@ moe_status launch_fp8(const CUtensorMap &a0, const CUtensorMap &a1, const CUtens
   auto kern = f8::tc_fp8_gemm<MODE, STAGES>;
   const size_t smem = L::smem_bytes(p.G, p.E);
   if (smem > 232448) return MOE_ERR_UNSUPPORTED;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
-      cudaSuccess)
-    return MOE_ERR_CUDA;
+  cudaError_t e = cudaGetLastError();  // nothing earlier may be reported as this launch's
+  if (e != cudaSuccess) return cuda_fail("before the FP8 GEMM", e);
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return cuda_fail("FP8 GEMM shared memory", e);
   const int nsm = sm_count();
   if (nsm < 2) return MOE_ERR_CUDA;
   cudaLaunchConfig_t cfg = {};
@@ -1572,12 +1634,17 @@ moe_status launch_fp8(const CUtensorMap &a0, const CUtensorMap &a1, const CUtens
   int pairs = nsm / 2;
   cfg.gridDim = dim3(2 * pairs);
   int active = 0;
-  if (cudaOccupancyMaxActiveClusters(&active, kern, &cfg) == cudaSuccess && active > 0 &&
-      active < pairs)
+  e = cudaOccupancyMaxActiveClusters(&active, kern, &cfg);
+  if (e != cudaSuccess) {
+    cudaGetLastError();  // not sticky: the launch below decides
+    if (getenv("MOE_DEBUG")) cuda_fail("FP8 GEMM occupancy query", e);
+  } else if (active > 0 && active < pairs) {
     pairs = active;
+  }
   cfg.gridDim = dim3(2 * pairs);
-  if (cudaLaunchKernelEx(&cfg, kern, a0, a1, b, p) != cudaSuccess) return MOE_ERR_CUDA;
-  return launch_status();
+  e = cudaLaunchKernelEx(&cfg, kern, a0, a1, b, p);
+  if (e != cudaSuccess) return cuda_fail("FP8 GEMM launch", e);
+  return checked_launch("FP8 GEMM launch");
 }
 
 // Optional profiling events (caller-owned cudaEvent_t), recorded on the call's
@@ -1611,6 +1678,12 @@ struct Job {
 
   int E() const { return c->n_routed; }
   int G() const { return c->n_routed + c->n_shared; }
+  // the call's share of the work (all of it unless expert-parallel) and
+  // whether it is a strict part (then rows outside it are skipped)
+  Shard sh;
+  bool sharded;
+  int wgroups() const { return (sh.e1 - sh.e0) + c->n_shared; }  // groups in the weight tensors
+  const int32_t *shard_off() const { return sharded ? offsets : nullptr; }
   int rows_routed() const { return (int)(T * c->topk); }
   int rows_total() const { return (int)(T * c->topk + T * c->n_shared); }
   int32_t *tab() const { return reinterpret_cast<int32_t *>(ws + l.tab); }
@@ -1637,6 +1710,7 @@ tc::Params tc_params(const Job &j) {
   p.sA1 = nullptr;
   p.sX = nullptr;
   p.ld_sx = 0;
+  p.sh = j.sh;
   return p;
 }
 
@@ -1655,7 +1729,7 @@ moe_status tc_up(const Job &j) {
   int32_t *tab = j.tab();
   Tiling t1{BN_MAX, I / L::FEAT, tab, tab + (G + 1)};
   Tiling none{0, 0, nullptr, nullptr};
-  prep_tiles<<<1, 32, 0, j.s>>>(j.offsets, j.E(), G, (int)j.T, t1, none);
+  prep_tiles<<<1, 32, 0, j.s>>>(j.offsets, j.E(), G, j.sh, t1, none);
   moe_status st = launch_status();
   if (st != MOE_OK) return st;
   bf16 *xperm = reinterpret_cast<bf16 *>(j.ws + j.l.xperm);
@@ -1665,16 +1739,17 @@ moe_status tc_up(const Job &j) {
   if (F8)
     gather_rows_f16<<<(unsigned)((threads + 255) / 256), 256, 0, j.s>>>(
         static_cast<const __nv_bfloat162 *>(j.x), j.sorted_token,
-        reinterpret_cast<__half2 *>(xperm), j.rows_routed(), j.rows_total(), (int)j.T, D / 2);
+        reinterpret_cast<__half2 *>(xperm), j.rows_routed(), j.rows_total(), (int)j.T, D / 2,
+        j.shard_off(), j.sh);
   else
     gather_rows<<<(unsigned)((threads + 255) / 256), 256, 0, j.s>>>(
         static_cast<const uint4 *>(j.x), j.sorted_token, reinterpret_cast<uint4 *>(xperm),
-        j.rows_routed(), j.rows_total(), (int)j.T, D * 2 / 16);
+        j.rows_routed(), j.rows_total(), (int)j.T, D * 2 / 16, j.shard_off(), j.sh);
   if ((st = launch_status()) != MOE_OK) return st;
   CUtensorMap mw1, mw3, mx;
   const CUtensorMapDataType BF = F8 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
-  if (!weight_tmap(&mw1, j.w->w1, F8, (uint64_t)G * I, D, L::PART_ROWS) ||
-      !weight_tmap(&mw3, j.w->w3, F8, (uint64_t)G * I, D, L::PART_ROWS) ||
+  if (!weight_tmap(&mw1, j.w->w1, F8, (uint64_t)j.wgroups() * I, D, L::PART_ROWS) ||
+      !weight_tmap(&mw3, j.w->w3, F8, (uint64_t)j.wgroups() * I, D, L::PART_ROWS) ||
       !make_tmap(&mx, xperm, BF, 2, (uint64_t)j.l.rows_pad, D, BOXN, 64))
     return MOE_ERR_CUDA;
   tc::Params p = tc_params(j);
@@ -1697,13 +1772,13 @@ moe_status tc_down(const Job &j) {
   int32_t *tab = j.tab();
   Tiling t2{BN_MAX, D / L::FEAT, tab + (2 * G + 1), tab + (3 * G + 2)};
   Tiling none{0, 0, nullptr, nullptr};
-  prep_tiles<<<1, 32, 0, j.s>>>(j.offsets, j.E(), G, (int)j.T, t2, none);
+  prep_tiles<<<1, 32, 0, j.s>>>(j.offsets, j.E(), G, j.sh, t2, none);
   moe_status st = launch_status();
   if (st != MOE_OK) return st;
   bf16 *h = reinterpret_cast<bf16 *>(j.ws + j.l.h);
   CUtensorMap mw2, mh;
   const CUtensorMapDataType BF = F8 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
-  if (!weight_tmap(&mw2, j.w->w2, F8, (uint64_t)G * D, I, tc::BM) ||
+  if (!weight_tmap(&mw2, j.w->w2, F8, (uint64_t)j.wgroups() * D, I, tc::BM) ||
       !make_tmap(&mh, h, BF, 2, (uint64_t)j.l.rows_pad, I, BOXN, 64))
     return MOE_ERR_CUDA;
   tc::Params p = tc_params(j);
@@ -1742,12 +1817,13 @@ moe_status quantise_rows(const Job &j, const void *src, bool gather, size_t q_of
   if (gather)
     quant_rows_e4m3<true><<<grid, 256, smem, j.s>>>(static_cast<const uint2 *>(src),
                                                     j.sorted_token, q, sc, j.rows_routed(), rows,
-                                                    (int)j.T, K, (int)j.l.rows_pad);
+                                                    (int)j.T, K, (int)j.l.rows_pad, j.shard_off(),
+                                                    j.sh);
   else
     quant_rows_e4m3<false><<<grid, 256, smem, j.s>>>(static_cast<const uint2 *>(src), nullptr, q,
                                                      sc, j.rows_routed(), rows, (int)j.T, K,
-                                                     (int)j.l.rows_pad);
-  return launch_status();
+                                                     (int)j.l.rows_pad, j.shard_off(), j.sh);
+  return checked_launch("e4m3 row quantiser");
 }
 
 moe_status fp8_up(const Job &j) {
@@ -1755,16 +1831,16 @@ moe_status fp8_up(const Job &j) {
   int32_t *tab = j.tab();
   Tiling t1{f8::BN_MAX, I / 128, tab, tab + (G + 1)};
   Tiling none{0, 0, nullptr, nullptr};
-  prep_tiles<<<1, 32, 0, j.s>>>(j.offsets, j.E(), G, (int)j.T, t1, none);
+  prep_tiles<<<1, 32, 0, j.s>>>(j.offsets, j.E(), G, j.sh, t1, none);
   moe_status st = launch_status();
   if (st != MOE_OK) return st;
   prof(0, j.s);
   if ((st = quantise_rows(j, j.x, true, j.l.xq, j.l.xs, D)) != MOE_OK) return st;
   CUtensorMap mw1, mw3, mx;
-  if (!e4m3_tmap(&mw1, j.w->w1, (uint64_t)G * I, D, 64) ||
-      !e4m3_tmap(&mw3, j.w->w3, (uint64_t)G * I, D, 64) ||
+  if (!e4m3_tmap(&mw1, j.w->w1, (uint64_t)j.wgroups() * I, D, 64) ||
+      !e4m3_tmap(&mw3, j.w->w3, (uint64_t)j.wgroups() * I, D, 64) ||
       !e4m3_tmap(&mx, j.ws + j.l.xq, (uint64_t)j.l.rows_pad, D, f8::BOXN))
-    return MOE_ERR_CUDA;
+    return cuda_fail("FP8 first matmul tensor maps", cudaErrorInvalidValue);
   tc::Params p = tc_params(j);
   p.tile_start = t1.tile_start;
   p.tile_base = t1.tile_base;
@@ -1787,13 +1863,13 @@ moe_status fp8_down(const Job &j) {
   int32_t *tab = j.tab();
   Tiling t2{f8::BN_MAX, D / 256, tab + (2 * G + 1), tab + (3 * G + 2)};
   Tiling none{0, 0, nullptr, nullptr};
-  prep_tiles<<<1, 32, 0, j.s>>>(j.offsets, j.E(), G, (int)j.T, t2, none);
+  prep_tiles<<<1, 32, 0, j.s>>>(j.offsets, j.E(), G, j.sh, t2, none);
   moe_status st = launch_status();
   if (st != MOE_OK) return st;
   CUtensorMap mw2, mh;
-  if (!e4m3_tmap(&mw2, j.w->w2, (uint64_t)G * D, I, f8::BM) ||
+  if (!e4m3_tmap(&mw2, j.w->w2, (uint64_t)j.wgroups() * D, I, f8::BM) ||
       !e4m3_tmap(&mh, j.ws + j.l.hq, (uint64_t)j.l.rows_pad, I, f8::BOXN))
-    return MOE_ERR_CUDA;
+    return cuda_fail("FP8 second matmul tensor maps", cudaErrorInvalidValue);
   tc::Params p = tc_params(j);
   p.tile_start = t2.tile_start;
   p.tile_base = t2.tile_base;
@@ -1832,6 +1908,7 @@ SimtArgs simt_args(const Job &j, const Tiling &t) {
   a.weights = j.weights;
   a.k = j.c->topk;
   a.y = j.y;
+  a.sh = j.sh;
   return a;
 }
 
@@ -1844,7 +1921,7 @@ moe_status simt_up(const Job &j) {
   int32_t *tab = j.tab();
   Tiling t1{ST, (j.c->inter + ST - 1) / ST, tab, tab + (G + 1)};
   Tiling none{0, 0, nullptr, nullptr};
-  prep_tiles<<<1, 32, 0, j.s>>>(j.offsets, j.E(), G, (int)j.T, t1, none);
+  prep_tiles<<<1, 32, 0, j.s>>>(j.offsets, j.E(), G, j.sh, t1, none);
   moe_status st = launch_status();
   if (st != MOE_OK) return st;
   const SimtArgs a = simt_args(j, t1);
@@ -1865,7 +1942,7 @@ moe_status simt_down(const Job &j) {
   int32_t *tab = j.tab();
   Tiling t2{ST, (j.c->dim + ST - 1) / ST, tab + (2 * G + 1), tab + (3 * G + 2)};
   Tiling none{0, 0, nullptr, nullptr};
-  prep_tiles<<<1, 32, 0, j.s>>>(j.offsets, j.E(), G, (int)j.T, t2, none);
+  prep_tiles<<<1, 32, 0, j.s>>>(j.offsets, j.E(), G, j.sh, t2, none);
   moe_status st = launch_status();
   if (st != MOE_OK) return st;
   const SimtArgs a = simt_args(j, t2);
@@ -2009,6 +2086,8 @@ moe_status make_job(Job &j, const moe_cfg *cfg, int64_t T, const void *x, moe_dt
   j.y = nullptr;
   j.ws = static_cast<uint8_t *>(ws);
   j.status = dev_status;
+  j.sh = Shard{0, cfg->n_routed, 0, (int)T};
+  j.sharded = false;
   j.s = as_stream(stream);
   return MOE_OK;
 }
@@ -2085,6 +2164,59 @@ MOE_EXPORT moe_status moe_experts_forward_combine(const moe_cfg *cfg, int64_t T,
   return run_down(j);
 }
 
+// The rank's share of the expert work (host only; no device call).
+static moe_status ep_plan(const moe_cfg *cfg, int64_t T, const moe_ep_shard *shard, Shard *out) {
+  if (check_cfg(cfg) != MOE_OK || !shard || T < 0) return MOE_ERR_INVALID;
+  const int W = shard->world, r = shard->rank;
+  if (W < 1 || r < 0 || r >= W) return MOE_ERR_INVALID;
+  if (cfg->n_routed % W != 0) return MOE_ERR_UNSUPPORTED;
+  const int per = cfg->n_routed / W;
+  out->e0 = r * per;
+  out->e1 = (r + 1) * per;
+  out->st0 = (int)(T * r / W);
+  out->st1 = (int)(T * (r + 1) / W);
+  return MOE_OK;
+}
+
+MOE_EXPORT moe_status moe_ep_plan(const moe_cfg *cfg, int64_t T, const moe_ep_shard *shard,
+                                  int32_t *out) {
+  if (!out) return MOE_ERR_INVALID;
+  Shard sh;
+  const moe_status st = ep_plan(cfg, T, shard, &sh);
+  if (st != MOE_OK) return st;
+  out[0] = sh.e0;
+  out[1] = sh.e1;
+  out[2] = sh.st0;
+  out[3] = sh.st1;
+  return MOE_OK;
+}
+
+MOE_EXPORT moe_status moe_experts_forward_combine_ep(
+    const moe_cfg *cfg, int64_t T, const void *x, moe_dtype x_dt, const moe_expert_weights *w,
+    const moe_ep_shard *shard, const int32_t *offsets, const int32_t *sorted_token,
+    const int32_t *indices, const float *weights, float *y, void *ws, size_t ws_bytes,
+    int32_t *dev_status, moe_stream_t stream) {
+  Job j;
+  moe_status st = make_job(j, cfg, T, x, x_dt, w, offsets, sorted_token, y, y, ws, ws_bytes,
+                           dev_status, stream, true, true);
+  if (st != MOE_OK) return st;
+  Shard sh;
+  if ((st = ep_plan(cfg, T, shard, &sh)) != MOE_OK) return st;
+  if (T == 0) return MOE_OK;
+  if (!indices || !weights || !y) return MOE_ERR_INVALID;
+  j.out_perm = nullptr;
+  j.out_shared = nullptr;
+  j.indices = indices;
+  j.weights = weights;
+  j.y = y;
+  j.sh = sh;
+  j.sharded = shard->world > 1;
+  if (cudaMemsetAsync(y, 0, (size_t)T * cfg->dim * sizeof(float), j.s) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  if ((st = run_up(j)) != MOE_OK) return st;
+  return run_down(j);
+}
+
 MOE_EXPORT moe_status moe_quantize_e4m3_rows(const void *src, int64_t rows, int32_t K,
                                              uint8_t *q, float *scales, int64_t ld,
                                              moe_stream_t stream) {
@@ -2098,7 +2230,7 @@ MOE_EXPORT moe_status moe_quantize_e4m3_rows(const void *src, int64_t rows, int3
   if (smem > 48 * 1024) return MOE_ERR_UNSUPPORTED;
   quant_rows_e4m3<false><<<grid, 256, smem, as_stream(stream)>>>(
       static_cast<const uint2 *>(src), nullptr, reinterpret_cast<uint32_t *>(q), scales, 0,
-      (int)rows, 0, K, (int)ld);
+      (int)rows, 1, K, (int)ld, nullptr, Shard{0, 0, 0, 0});
   return launch_status();
 }
 

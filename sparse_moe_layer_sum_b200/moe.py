@@ -20,7 +20,7 @@ from typing import Optional
 import torch
 
 from . import _lib
-from ._lib import MoECfg, MoEExpertWeights, check, fn
+from ._lib import MoECfg, MoEEpShard, MoEExpertWeights, check, fn
 
 
 @dataclass(frozen=True)
@@ -223,6 +223,33 @@ def quantize_e4m3_rows(src: torch.Tensor):
     return q, sc
 
 
+def ep_plan(shape: BlockShape, T: int, rank: int, world: int) -> tuple:
+    """moe_ep_plan: (first expert, end expert, first token, end token) of the
+    shared expert's slice for expert-parallel rank `rank` of `world`."""
+    cfg = shape.cfg()
+    out = (ctypes.c_int32 * 4)()
+    check(fn("moe_experts", "moe_ep_plan")(ctypes.byref(cfg), T,
+                                           ctypes.byref(MoEEpShard(rank, world)), out),
+          "moe_ep_plan")
+    return tuple(out)
+
+
+def shard_params(shape: BlockShape, params: "BlockParams", rank: int, world: int) -> "BlockParams":
+    """The weights expert-parallel rank `rank` holds: its routed experts in
+    order, then the shared expert(s); the router weight and bias whole."""
+    e0, e1, _, _ = ep_plan(shape, 0, rank, world)
+    E = shape.n_routed
+
+    def part(t):
+        if t is None:
+            return None
+        return torch.cat([t[e0:e1], t[E:]]).contiguous()
+
+    p = params
+    return BlockParams(p.w_r, p.bias, part(p.w1), part(p.w3), part(p.w2), part(p.s1),
+                       part(p.s3), part(p.s2))
+
+
 def selftest_wait(limit_ns: int, status: torch.Tensor) -> None:
     check(fn("moe_experts", "moe_experts_selftest_wait")(limit_ns, status.data_ptr(), _stream()),
           "moe_experts_selftest_wait")
@@ -260,9 +287,17 @@ class MoEBlock:
     """
 
     def __init__(self, shape: BlockShape, params: BlockParams, T: int, x_dtype: torch.dtype,
-                 device=None, combine: str = "scatter", fp8_act: bool = False):
+                 device=None, combine: str = "scatter", fp8_act: bool = False,
+                 ep: tuple = (0, 1), ep_group=None):
         if combine not in ("scatter", "ordered"):
             raise ValueError(combine)
+        # expert parallelism: (rank, world); params then hold the rank's
+        # shard (shard_params) and y is summed over the ranks of ep_group by
+        # an all-reduce (left partial when ep_group is None)
+        self.ep_rank, self.ep_world = ep
+        self.ep_group = ep_group
+        if self.ep_world > 1 and combine != "scatter":
+            raise ValueError("expert parallelism uses the scatter combine")
         if fp8_act and params.s1 is None:
             raise ValueError("fp8_act needs e4m3 expert weights")
         self.fp8_act = fp8_act
@@ -345,6 +380,15 @@ class MoEBlock:
             "moe_dispatch_build")
 
     def _experts(self, x, cfgp, s, y):
+        if self.ep_world > 1:
+            shard = MoEEpShard(self.ep_rank, self.ep_world)
+            check(fn("moe_experts", "moe_experts_forward_combine_ep")(
+                cfgp, self.T, x.data_ptr(), _dt(x), ctypes.byref(self.wstruct),
+                ctypes.byref(shard), self.offsets.data_ptr(), self.sorted_token.data_ptr(),
+                self.indices.data_ptr(), self.weights.data_ptr(), y.data_ptr(),
+                self.ws_experts.data_ptr(), self.ws_experts.numel(), self.status.data_ptr(), s),
+                "moe_experts_forward_combine_ep")
+            return
         if self.combine_mode == "scatter":
             check(fn("moe_experts", "moe_experts_forward_combine")(
                 cfgp, self.T, x.data_ptr(), _dt(x), ctypes.byref(self.wstruct),
@@ -360,6 +404,10 @@ class MoEBlock:
             self.status.data_ptr(), s), "moe_experts_forward")
 
     def _combine(self, cfgp, s, y):
+        if self.ep_world > 1 and self.ep_group is not None:
+            # the ranks' partial sums (the moe-forward excerpt's all_reduce)
+            torch.distributed.all_reduce(y, group=self.ep_group)
+            return
         if self.combine_mode == "scatter":
             return  # done inside the experts' second matmul
         check(fn("moe_combine", "moe_combine")(

@@ -170,6 +170,31 @@ def test_fp8_activation_path_validation():
     assert q(None, 0, 128, None, None, 0, None) == 0           # nothing to do
 
 
+def test_expert_parallel_plan_and_validation():
+    from sparse_moe_layer_sum_b200._lib import MoEEpShard
+    plan = fn("moe_experts", "moe_ep_plan")
+    c = v3_cfg()
+    out = (ctypes.c_int32 * 4)()
+    assert plan(ctypes.byref(c), 4096, ctypes.byref(MoEEpShard(3, 8)), out) == 0
+    assert list(out) == [96, 128, 1536, 2048]          # experts 96..127, tokens 1536..2047
+    assert plan(ctypes.byref(c), 10, ctypes.byref(MoEEpShard(2, 3)), out) == UNSUPPORTED
+    assert plan(ctypes.byref(c), 10, ctypes.byref(MoEEpShard(8, 8)), out) == INVALID
+    assert plan(ctypes.byref(c), 10, ctypes.byref(MoEEpShard(0, 0)), out) == INVALID
+    assert plan(ctypes.byref(c), -1, ctypes.byref(MoEEpShard(0, 1)), out) == INVALID
+    assert plan(ctypes.byref(c), 10, None, out) == INVALID
+    f = fn("moe_experts", "moe_experts_forward_combine_ep")
+    w = MoEExpertWeights(0x1000, 0x1000, 0x1000, 1, None, None, None)
+    sh = MoEEpShard(1, 4)
+    assert f(ctypes.byref(c), 8, P, 1, ctypes.byref(w), None, P, P, P, P, P, P, 1 << 40, None,
+             None) == INVALID                                   # no shard
+    assert f(ctypes.byref(c), 8, P, 1, ctypes.byref(w), ctypes.byref(MoEEpShard(1, 3)), P, P, P,
+             P, P, P, 1 << 40, None, None) == UNSUPPORTED
+    assert f(ctypes.byref(c), 8, P, 1, ctypes.byref(w), ctypes.byref(sh), P, P, None, P, P, P,
+             1 << 40, None, None) == INVALID                    # no router indices
+    assert f(ctypes.byref(c), 0, P, 1, ctypes.byref(w), ctypes.byref(sh), P, P, P, P, P, P,
+             1 << 40, None, None) == 0                          # empty batch
+
+
 def test_combine_and_selftest_validation():
     f = fn("moe_combine", "moe_combine")
     c = v3_cfg()

@@ -35,7 +35,7 @@ def _worker(rank, world, port, out):
 
 def test_two_replicas_report_the_slowest_rank():
     world, port = 2, _free_port()
-    out = mp.Manager().dict()
+    out = mp.get_context("spawn").Manager().dict()
     mp.spawn(_worker, args=(world, port, out), nprocs=world, join=True)
     assert out[0] == out[1]
     m, tps = out[0]
