@@ -44,8 +44,8 @@ Readings of points the pages leave open:
 6. FP8 activations (the optional FP8 x FP8 path of the FP8-weight
    configuration; the pages name FP8 experts but no activation format):
    each row of x, and each row of h after its bf16 rounding, is quantised to
-   e4m3 in 1 x 128 blocks with the weights' rule, scale = block amax / 448,
-   in fp32 arithmetic.
+   e4m3 with the weights' rule applied to the row, scale = row amax / 448,
+   in fp32 arithmetic (one scale per token and matrix).
 
 Parity pins for every function live in ``tests/test_oracle_*.py``.
 """
@@ -198,8 +198,9 @@ def e4m3_code(values: np.ndarray) -> np.ndarray:
     return np.vectorize(lambda x: lut[float(x)], otypes=[np.uint8])(np.asarray(values))
 
 
-def quantize_e4m3_rows(v: np.ndarray, block: int = 128):
-    """Per-row 1 x block e4m3 quantisation of activations, fp32 arithmetic.
+def quantize_e4m3_rows(v: np.ndarray, block: Optional[int] = None):
+    """Per-row e4m3 quantisation of activations in 1 x block runs (the whole
+    row when block is None), fp32 arithmetic.
 
     For each row and each run of `block` columns: amax = max |v| (exact),
     scale = fp32(amax / 448) (an IEEE fp32 division), r = fp32(1 / scale)
@@ -212,6 +213,7 @@ def quantize_e4m3_rows(v: np.ndarray, block: int = 128):
     """
     v = np.asarray(v, dtype=np.float32)
     r, c = v.shape
+    block = c if block is None else block
     vb = v.reshape(r, c // block, block)
     amax = np.abs(vb).max(axis=-1)
     scale = (amax / np.float32(E4M3_MAX)).astype(np.float32)
@@ -223,9 +225,11 @@ def quantize_e4m3_rows(v: np.ndarray, block: int = 128):
     return vals.reshape(r, c), scale
 
 
-def dequant_e4m3_rows(vals: np.ndarray, scales: np.ndarray, block: int = 128) -> np.ndarray:
-    """fp64 activation from the e4m3 values and per-row 1 x block scales."""
-    s = np.repeat(np.asarray(scales, dtype=np.float64), block, axis=-1)
+def dequant_e4m3_rows(vals: np.ndarray, scales: np.ndarray) -> np.ndarray:
+    """fp64 activation from the e4m3 values and their per-row scales
+    (one or more equal runs of columns per scale)."""
+    s = np.asarray(scales, dtype=np.float64)
+    s = np.repeat(s, np.asarray(vals).shape[-1] // s.shape[-1], axis=-1)
     return np.asarray(vals, dtype=np.float64) * s
 
 
@@ -378,9 +382,10 @@ def expert_ffn(x_rows: np.ndarray, w1: np.ndarray, w3: np.ndarray, w2: np.ndarra
     x_rows [n, D]; w1, w3 [I, D]; w2 [D, I] in the nn.Linear [out, in] layout.
     The hidden activation h is rounded once, through fp32, to the type of
     the second matmul's operand (reading 3): ``act_dtype`` "bf16", "f16" or
-    "f32".  "e4m3" (reading 6): the rows of x and the bf16-rounded h are
-    each quantised to e4m3 in 1 x 128 blocks (quantize_e4m3_rows) and the
-    matmuls take the dequantised values.  Returns fp64 [n, D].
+    "f32".  "e4m3" (reading 6): each row of x and each row of the
+    bf16-rounded h is quantised to e4m3 with one scale per row
+    (quantize_e4m3_rows) and the matmuls take the dequantised values.
+    Returns fp64 [n, D].
     """
     x64 = np.asarray(x_rows, dtype=np.float64)
     if act_dtype == "e4m3":

@@ -132,18 +132,29 @@ def test_e4m3_code_inverts_the_table():
 
 def test_activation_quantisation_worked_example():
     g = read_golden("e4m3_act_quant.txt")
-    v = np.zeros((2, 256), dtype=np.float32)
+    v = np.zeros((3, 256), dtype=np.float32)
     v[0, [int(c) for c in g["row0_cols"]]] = [float(x) for x in g["row0_vals"]]
     v[1, [int(c) for c in g["row1_cols"]]] = [float(x) for x in g["row1_vals"]]
     vals, scales = quantize_e4m3_rows(v)
-    assert scales.dtype == np.float32
-    assert list(scales[0]) == [float(x) for x in g["row0_scales"]]
-    assert list(scales[1]) == [float(x) for x in g["row1_scales"]]
+    assert scales.dtype == np.float32 and scales.shape == (3, 1)
+    assert list(scales[:, 0]) == [float(x) for x in g["scales"]]
     deq = dequant_e4m3_rows(vals, scales)
-    want0 = [float(x) for x in g["row0_codes_times_scale"]]
-    assert list(deq[0, [int(c) for c in g["row0_cols"]]]) == want0
+    assert list(deq[0, [int(c) for c in g["row0_cols"]]]) == [float(x) for x in g["row0_deq"]]
     assert list(deq[1, [int(c) for c in g["row1_cols"]]]) == [float(x) for x in g["row1_deq"]]
-    assert np.count_nonzero(deq) == 7                    # zeros stay zero, block 1 empty
+    assert np.count_nonzero(deq) == 8                    # zeros stay zero, row 2 empty
+
+
+def test_activation_quantisation_blocks_are_independent_rows():
+    # with 1 x 128 runs, each run is quantised as a row of its own
+    rng = np.random.default_rng(10)
+    v = (rng.standard_normal((5, 384)) * np.exp(rng.standard_normal((5, 3)).repeat(128, 1)))
+    v = v.astype(np.float32)
+    vals, scales = quantize_e4m3_rows(v, block=128)
+    assert scales.shape == (5, 3)
+    for b in range(3):
+        vb, sb = quantize_e4m3_rows(v[:, 128 * b:128 * (b + 1)])
+        assert np.array_equal(vals[:, 128 * b:128 * (b + 1)], vb)
+        assert np.array_equal(scales[:, b:b + 1], sb)
 
 
 def test_activation_quantisation_error_bound():
@@ -153,10 +164,8 @@ def test_activation_quantisation_error_bound():
     v = (rng.standard_normal((64, 512)) * np.exp(rng.standard_normal((64, 1)))).astype(np.float32)
     vals, scales = quantize_e4m3_rows(v)
     deq = dequant_e4m3_rows(vals, scales)
-    s = np.repeat(scales.astype(np.float64), 128, axis=1)
+    s = scales.astype(np.float64)
     bound = np.maximum(np.abs(v) * 2.0 ** -4, s * 2.0 ** -10) * (1 + 1e-6)
     assert np.all(np.abs(deq - v) <= bound)
-    # the block maximum itself is kept to fp32 rounding of the scale
-    amax = np.abs(v.reshape(64, 4, 128)).max(-1)
-    deq_max = np.abs(deq.reshape(64, 4, 128)).max(-1)
-    assert np.allclose(deq_max, amax, rtol=2e-7)
+    # the row maximum itself is kept to fp32 rounding of the scale
+    assert np.allclose(np.abs(deq).max(-1), np.abs(v).max(-1), rtol=2e-7)
