@@ -36,7 +36,8 @@ METRIC = "MoE block tokens/s (V3 shape, bf16, T=4096) and % of roofline on 1 B20
 N_X_BATCHES = 4  # rotating input batches: with the 22.6 GB of weights, > L2 per step
 # the other configurations timed in short loops after the headline one:
 # (workload, FP8 x FP8 activations)
-OTHER_CONFIGS = [("v3_decode_t64", False), ("v3_skew_t16384", False), ("v3_fp8_t8192", False)]
+OTHER_CONFIGS = [("v3_decode_t64", False), ("v3_skew_t16384", False), ("v3_fp8_t8192", False),
+                 ("v3_fp8_t8192", True)]
 
 
 def parse():

@@ -37,13 +37,13 @@ extern "C" {
  * For MOE_E4M3 the weight is value(q) * scale of its 128 x 128 block.
  *   act_e4m3  0: the matmuls take bf16 activations (e4m3 weights are
  *             expanded to fp16 on the fly, fp16 x fp16 MMAs).
- *             1 (MOE_E4M3 weights only): FP8 x FP8 -- the expert rows of x
- *             and the hidden h (after its bf16 rounding) are quantised to
- *             e4m3 in 1 x 128 blocks along the reduction dimension, each
- *             block with fp32 scale = block amax / 448 (the weights' rule;
- *             an all-zero block has scale 0), and the matmuls run as
- *             e4m3 x e4m3 tensor-core MMAs whose per-block partial sums are
- *             scaled by weight scale x activation scale in fp32.  The pages
+ *             1 (MOE_E4M3 weights only): FP8 x FP8 -- each expert row of x
+ *             and each row of the hidden h (after its bf16 rounding) is
+ *             quantised to e4m3 with one fp32 scale per row, row amax / 448
+ *             (the weights' rule; an all-zero row has scale 0), and the
+ *             matmuls run as e4m3 x e4m3 tensor-core MMAs; each 128-wide
+ *             k-block's partial sum is scaled by its weight block's scale in
+ *             fp32, and the row's scale is applied to the total.  The pages
  *             name FP8 experts but no activation format; this path trades
  *             about 5% rms of extra error for twice the tensor throughput.
  *             Needs dim % 256 == 0 and inter % 128 == 0.
@@ -163,20 +163,19 @@ moe_status moe_experts_down(const moe_cfg *cfg, int64_t T, moe_dtype x_dt,
 
 /*
  * The activation quantiser of the FP8 x FP8 path (act_e4m3 = 1), on its own:
- * each row of src [rows, K] bf16 is cut into K / 128 blocks of 128 values;
- * a block's scale is amax / 448 (fp32, IEEE division) and its codes are
- * e4m3(v * fp32(1 / scale)) (IEEE reciprocal, round to nearest even,
- * saturated to +-448); an all-zero block has scale 0 and codes 0.
+ * each row of src [rows, K] bf16 gets one scale, amax / 448 (fp32, IEEE
+ * division), and codes e4m3(v * fp32(1 / scale)) (IEEE reciprocal, round to
+ * nearest even, saturated to +-448); an all-zero row has scale 0 and codes 0.
  *   q       [rows, K] uint8 out (e4m3 codes, row-major)
- *   scales  [K / 128, ld] fp32 out, transposed: row r's scale of block b at
- *           scales[b * ld + r]; ld >= rows
+ *   scales  [rows] fp32 out
  * No counterpart on the pages, which name FP8 experts but no activation
- * format (the weights' 128 x 128 block rule applied to 1 x 128 blocks).
- * Limits: K % 128 == 0, rows < 2^31.  Returns MOE_ERR_INVALID for bad
- * sizes or NULL pointers (rows == 0 launches nothing).
+ * format (the weights' amax / 448 block rule applied to a row).
+ * Limits: K % 4 == 0, rows < 2^31, src and q 8- and 4-byte aligned.
+ * Returns MOE_ERR_INVALID for bad sizes or NULL pointers (rows == 0
+ * launches nothing).
  */
 moe_status moe_quantize_e4m3_rows(const void *src, int64_t rows, int32_t K, uint8_t *q,
-                                  float *scales, int64_t ld, moe_stream_t stream);
+                                  float *scales, moe_stream_t stream);
 
 /*
  * Profiling: register up to five caller-owned cudaEvent_t handles that later

@@ -79,7 +79,7 @@ SIGNATURES = {
     ("moe_experts", "moe_experts_down"): (
         _i32, [_cfgp, _i64, _i32, ctypes.POINTER(MoEExpertWeights), _vp, _vp, _vp, _vp, _sz, _vp,
                _vp]),
-    ("moe_experts", "moe_quantize_e4m3_rows"): (_i32, [_vp, _i64, _i32, _vp, _vp, _i64, _vp]),
+    ("moe_experts", "moe_quantize_e4m3_rows"): (_i32, [_vp, _i64, _i32, _vp, _vp, _vp]),
     ("moe_experts", "moe_experts_set_profile_events"): (_i32, [ctypes.POINTER(_vp), _i32]),
     ("moe_experts", "moe_experts_selftest_wait"): (_i32, [_i64, _vp, _vp]),
     ("moe_combine", "moe_combine"): (_i32, [_cfgp, _i64, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),

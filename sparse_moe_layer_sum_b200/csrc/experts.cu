@@ -255,10 +255,8 @@ struct Params {
   float *y;                // [T, D], zeroed before the launch
   // e4m3 weights: fp32 scales of 128 x 128 blocks, [G, rows/128, cols/128]
   const float *sA0, *sA1;  // GEMM1: w1, w3; second GEMM: w2 (sA1 unused)
-  // FP8 x FP8 path: the activation rows' 1 x 128 block scales, transposed
-  // [K / 128][ld_sx] (row r's scale for k-block kb at kb * ld_sx + r)
+  // FP8 x FP8 path: the activation rows' scales, one per row
   const float *sX;
-  int ld_sx;
   Shard sh;
 };
 
@@ -863,67 +861,61 @@ __global__ void selftest_wait_kernel(int64_t limit_ns, int32_t *status) {
 //
 // The optional path for e4m3 weights on which the activations are quantised
 // to e4m3 as well, so that the matmuls run as e4m3 x e4m3 tensor-core MMAs
-// (kind::f8f6f4, twice the bf16 rate).  Both operands carry fp32 block scales
-// along the reduction dimension: the weights per 128 x 128 block, the
-// activation rows per 1 x 128 block.  A k-block of 128 is one 128-byte
-// swizzle row of e4m3, so every k-block's partial sum is scaled by one weight
-// scale per CTA (its 128 weight rows lie in one scale block) times one
-// activation scale per token:
-//   acc[m, n] = sum_kb  s_w[kb] * s_x[n, kb] * (sum_{k in kb} q_w[m, k] q_x[n, k])
+// (kind::f8f6f4, twice the bf16 rate).  The weights carry fp32 scales per
+// 128 x 128 block, the activation rows one fp32 scale per row.  A k-block of
+// 128 is one 128-byte swizzle row of e4m3, so every k-block's partial sum is
+// scaled by one weight scale per CTA (its 128 weight rows lie in one scale
+// block), and the token's scale factors out of the whole sum:
+//   acc[m, n] = s_x[n] * sum_kb  s_w[kb] * (sum_{k in kb} q_w[m, k] q_x[n, k])
 // The MMAs of a k-block write a fresh TMEM partial (two buffers alternate)
-// and eight promotion warps fold it into fp32 running sums in registers.
+// and eight promotion warps fold it into fp32 running sums in registers with
+// one warp-uniform scale; s_x is applied once per tile.
 
-// Rows of a bf16 matrix [*, K] quantised to e4m3 in 1 x 128 blocks:
+// Rows of a bf16 matrix [*, K] quantised to e4m3 with one scale per row:
 // scale = amax / 448 (IEEE division), r = 1 / scale (IEEE reciprocal),
-// code = e4m3(v * r), rounded to nearest even and saturated; an all-zero
-// block has scale 0 and codes 0.  With GATHER, output row p < rows_routed
-// is token sorted_token[p] and row rows_routed + t is token t (the shared
-// expert's rows); otherwise row p is source row p.  Codes go to q [rows, K]
-// row-major; scales, transposed, to sc [K / 128][ld], so that the scales of
-// a tile's tokens for one k-block are contiguous.  A block of eight warps
-// takes 32 consecutive rows; a warp quantises one 128-column block per step,
-// four values per lane.
+// code = e4m3(v * r), rounded to nearest even and saturated; an all-zero row
+// has scale 0 and codes 0.  With GATHER, output row p < rows_routed is token
+// sorted_token[p] and row rows_routed + t is token t (the shared expert's
+// rows); otherwise row p is source row p.  Codes go to q [rows, K]
+// row-major, scales to sc [rows].  One warp per row: a pass for the row's
+// amax, a second (from L1/L2) for the codes, four values per lane and step.
 template <bool GATHER>
 __global__ void __launch_bounds__(256) quant_rows_e4m3(const uint2 *__restrict__ src,
                                                        const int32_t *__restrict__ sorted_token,
                                                        uint32_t *__restrict__ q,
                                                        float *__restrict__ sc, int rows_routed,
-                                                       int rows_total, int T, int K, int ld,
+                                                       int rows_total, int T, int K,
                                                        const int32_t *off, Shard sh) {
-  extern __shared__ float s_sc[];  // [K / 128][32]
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  const int row0 = blockIdx.x * 32;
-  const int KB = K / 128;
-  for (int rr = warp; rr < 32; rr += 8) {
-    const int row = row0 + rr;
-    if (row >= rows_total) break;
-    if (!row_in_shard(row, rows_routed, T, off, sh)) continue;
-    const int srow = !GATHER ? row : row < rows_routed ? sorted_token[row] : row - rows_routed;
-    const uint2 *s = src + (size_t)srow * (K / 4);
-    uint32_t *d = q + (size_t)row * (K / 4);
-    for (int kb = 0; kb < KB; ++kb) {
-      const uint2 v = __ldg(s + kb * 32 + lane);  // four bf16
+  const int row = blockIdx.x * 8 + warp;
+  if (row >= rows_total) return;
+  if (!row_in_shard(row, rows_routed, T, off, sh)) return;
+  const int srow = !GATHER ? row : row < rows_routed ? sorted_token[row] : row - rows_routed;
+  const uint2 *s = src + (size_t)srow * (K / 4);
+  uint32_t *d = q + (size_t)row * (K / 4);
+  const int n4 = K / 4;  // groups of four values in the row
+  float m = 0.0f;
+  for (int i = lane; i < n4; i += 32) {
+    const uint2 v = __ldg(s + i);
+    m = fmaxf(m, fmaxf(fmaxf(fabsf(__uint_as_float(v.x << 16)), fabsf(__uint_as_float(v.x & 0xffff0000u))),
+                       fmaxf(fabsf(__uint_as_float(v.y << 16)), fabsf(__uint_as_float(v.y & 0xffff0000u)))));
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  const float scale = m / 448.0f;
+  const float r = scale > 0.0f ? __frcp_rn(scale) : 0.0f;
+  for (int i = lane; i < n4; i += 32) {
+    uint32_t packed = 0;
+    if (scale > 0.0f) {
+      const uint2 v = __ldg(s + i);
       const float f0 = __uint_as_float(v.x << 16), f1 = __uint_as_float(v.x & 0xffff0000u);
       const float f2 = __uint_as_float(v.y << 16), f3 = __uint_as_float(v.y & 0xffff0000u);
-      float m = fmaxf(fmaxf(fabsf(f0), fabsf(f1)), fmaxf(fabsf(f2), fabsf(f3)));
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
-      const float scale = m / 448.0f;
-      uint32_t packed = 0;
-      if (scale > 0.0f) {
-        const float r = __frcp_rn(scale);
-        packed = (uint32_t)sm100::f32x2_to_e4m3x2(__fmul_rn(f0, r), __fmul_rn(f1, r)) |
-                 ((uint32_t)sm100::f32x2_to_e4m3x2(__fmul_rn(f2, r), __fmul_rn(f3, r)) << 16);
-      }
-      d[kb * 32 + lane] = packed;
-      if (lane == 0) s_sc[kb * 32 + rr] = scale;
+      packed = (uint32_t)sm100::f32x2_to_e4m3x2(__fmul_rn(f0, r), __fmul_rn(f1, r)) |
+               ((uint32_t)sm100::f32x2_to_e4m3x2(__fmul_rn(f2, r), __fmul_rn(f3, r)) << 16);
     }
+    d[i] = packed;
   }
-  __syncthreads();
-  for (int i = threadIdx.x; i < KB * 32; i += 256) {
-    const int kb = i / 32, rr = i % 32;
-    if (row0 + rr < rows_total) sc[(size_t)kb * ld + row0 + rr] = s_sc[i];
-  }
+  if (lane == 0) sc[row] = scale;
 }
 
 namespace f8 {
@@ -964,7 +956,7 @@ struct Layout {
   static constexpr int MISC_OFF = BAR_OFF + NBARS * 8;
   static constexpr int MISC_BYTES = 16 + 4 * STAGES;  // TMEM slot, abort flag, pending loads
   static constexpr int SC_OFF = (MISC_OFF + MISC_BYTES + 127) / 128 * 128;
-  static constexpr int SC_BYTES = EPI * CHUNKS * 32 * 4;  // combined scales of one k-block
+  static constexpr int SC_BYTES = EPI * CHUNKS * 32 * 4;  // the tile's token scales, per warp
   static constexpr int XBUF_OFF = SC_OFF + SC_BYTES;
   // SwiGLU exchange of the four warp pairs (first matmul), or the tile's
   // (token, gate) list (second matmul with the scatter)
@@ -1155,62 +1147,63 @@ __global__ void __launch_bounds__(NT, 1)
         sw = (q < 2 ? p.sA0 : p.sA1) + ((size_t)t.wg * (p.I / 128) + t.ft) * KB;
       else
         sw = p.sA0 + ((size_t)t.wg * (p.D / 128) + t.ft * 2 + (int)rank) * KB;
-      const float *sx = p.sX + row0 + lane;
+      // what the tile's end needs from memory is fetched now, so that its
+      // latency passes during the k-loop: each lane's token scales and (second
+      // matmul with the scatter) the tile's token and gate list
+      float sxr[CHUNKS];
+#pragma unroll
+      for (int j = 0; j < CHUNKS; ++j) {
+        const int c = (2 * j + half) * 32 + lane;
+        sxr[j] = c < t.nvalid ? __ldg(p.sX + row0 + c) : 0.0f;
+      }
+      int32_t *s_tok = reinterpret_cast<int32_t *>(xbuf);
+      float *s_gate = reinterpret_cast<float *>(s_tok + BN_MAX);
+      if (MODE == 3) {
+        const int et = threadIdx.x - 32 * EPI0;
+        named_bar_sync(5, 32 * EPI);  // the previous tile's readers are done
+        for (int c = et; c < t.nvalid; c += 32 * EPI) {
+          int tok;
+          float gate = 1.0f;
+          if (t.g < p.E) {
+            tok = p.sorted_token[row0 + c];
+            for (int jj = 0; jj < p.k; ++jj)
+              if (p.indices[(size_t)tok * p.k + jj] == t.g) gate = p.weights[(size_t)tok * p.k + jj];
+          } else {
+            tok = t.tok0 + c;
+          }
+          s_tok[c] = tok;
+          s_gate[c] = gate;
+        }
+      }
+      // running sums: this lane's row, the warp's columns
       float acc[CHUNKS][32];
 #pragma unroll
       for (int j = 0; j < CHUNKS; ++j)
 #pragma unroll
         for (int e = 0; e < 32; ++e) acc[j][e] = 0.0f;
+#define ACC(j, e) acc[j][e]
       const int k0 = k_rotation(t, KB);
-      // scales are fetched two k-blocks ahead of their use
-      float nx[2][CHUNKS], nw[2];
-      auto fetch = [&](int i, float (&x)[CHUNKS], float &w) {
-        const int kb = k0 + i < KB ? k0 + i : k0 + i - KB;
-        w = __ldg(sw + kb);
-#pragma unroll
-        for (int j = 0; j < CHUNKS; ++j) {
-          const int c = (2 * j + half) * 32 + lane;
-          x[j] = c < t.nvalid ? __ldg(sx + (size_t)kb * p.ld_sx + (2 * j + half) * 32) : 0.0f;
-        }
-      };
-      fetch(0, nx[0], nw[0]);
-      if (KB > 1) fetch(1, nx[1], nw[1]);
+      // the weight scale of each k-block, fetched one k-block ahead of its use
+      float nw = __ldg(sw + k0);
       for (int i = 0; i < KB; ++i) {
-        float cx[CHUNKS], cw = nw[0];
-#pragma unroll
-        for (int j = 0; j < CHUNKS; ++j) {
-          cx[j] = nx[0][j];
-          nx[0][j] = nx[1][j];
-        }
-        nw[0] = nw[1];
-        if (i + 2 < KB) fetch(i + 2, nx[1], nw[1]);
+        const float cw = nw;
+        if (i + 1 < KB) nw = __ldg(sw + (k0 + i + 1 < KB ? k0 + i + 1 : k0 + i + 1 - KB));
         if (!wait_bounded(pfull + pb, pphase, abort_flag, p.timeout_ns, p.status)) {
           ok = false;
           break;
         }
         tc_fence_after();
-#pragma unroll
-        for (int j = 0; j < CHUNKS; ++j) comb[j * 32 + lane] = cw * cx[j];
-        __syncwarp();
+        // acc += s_w[kb] * partial: a chunk's 32 columns per TMEM load, with
+        // the (warp-uniform) weight scale
 #pragma unroll
         for (int j = 0; j < CHUNKS; ++j) {
           const int c0 = (2 * j + half) * 32;
-          if (c0 < t.nvalid) {
+          if (c0 >= t.nvalid) continue;
+          uint32_t v[32];
+          tmem_ld_32x32b_x32(lane_base + (uint32_t)(pb * BN_MAX + c0), v);
+          tmem_wait_ld();
 #pragma unroll
-            for (int hh = 0; hh < 32; hh += 16) {
-              uint32_t v[16];
-              tmem_ld_32x32b_x16(lane_base + (uint32_t)(pb * BN_MAX + c0 + hh), v);
-              tmem_wait_ld();
-#pragma unroll
-              for (int e = 0; e < 16; e += 4) {
-                const float4 c = *reinterpret_cast<const float4 *>(comb + j * 32 + hh + e);
-                acc[j][hh + e] = fmaf(__uint_as_float(v[e]), c.x, acc[j][hh + e]);
-                acc[j][hh + e + 1] = fmaf(__uint_as_float(v[e + 1]), c.y, acc[j][hh + e + 1]);
-                acc[j][hh + e + 2] = fmaf(__uint_as_float(v[e + 2]), c.z, acc[j][hh + e + 2]);
-                acc[j][hh + e + 3] = fmaf(__uint_as_float(v[e + 3]), c.w, acc[j][hh + e + 3]);
-              }
-            }
-          }
+          for (int e = 0; e < 32; ++e) acc[j][e] = fmaf(__uint_as_float(v[e]), cw, acc[j][e]);
         }
         tc_fence_before();
         __syncwarp();
@@ -1221,6 +1214,17 @@ __global__ void __launch_bounds__(NT, 1)
         }
       }
       if (!ok) break;
+      // times each token's activation scale (one per row, the same for every
+      // k-block), handed from the lane that holds it to all lanes through
+      // this warp's shared-memory slots
+#pragma unroll
+      for (int j = 0; j < CHUNKS; ++j) comb[j * 32 + lane] = sxr[j];
+      __syncwarp();
+#pragma unroll
+      for (int j = 0; j < CHUNKS; ++j)
+#pragma unroll
+        for (int e = 0; e < 32; ++e) acc[j][e] *= comb[j * 32 + e];
+      __syncwarp();
 
       if (MODE == 1) {
         // lanes 0-63 of the CTA hold w1.x (a), lanes 64-127 w3.x (u) of the
@@ -1239,14 +1243,14 @@ __global__ void __launch_bounds__(NT, 1)
           if (c0 >= t.nvalid) continue;
           float *mine = is_a ? buf_a : buf_u;
 #pragma unroll
-          for (int e = 0; e < 16; ++e) mine[lane * XB_STRIDE + e] = is_a ? acc[j][16 + e] : acc[j][e];
+          for (int e = 0; e < 16; ++e) mine[lane * XB_STRIDE + e] = is_a ? ACC(j, 16 + e) : ACC(j, e);
           named_bar_sync(bar, 64);
           const float *other = is_a ? buf_u : buf_a;
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
             const int col = is_a ? e : 16 + e;
-            const float a = is_a ? acc[j][e] : other[lane * XB_STRIDE + e];
-            const float u = is_a ? other[lane * XB_STRIDE + e] : acc[j][16 + e];
+            const float a = is_a ? ACC(j, e) : other[lane * XB_STRIDE + e];
+            const float u = is_a ? other[lane * XB_STRIDE + e] : ACC(j, 16 + e);
             if (c0 + col < t.nvalid)
               out[(size_t)(row0 + c0 + col) * p.I + f] = __float2bfloat16_rn(swiglu_h(a, u));
           }
@@ -1268,27 +1272,11 @@ __global__ void __launch_bounds__(NT, 1)
           const int c0 = (2 * j + half) * 32;
 #pragma unroll
           for (int e = 0; e < 32; ++e)
-            if (c0 + e < t.nvalid) out[(r0 + c0 + e) * p.D + d] = acc[j][e];
+            if (c0 + e < t.nvalid) out[(r0 + c0 + e) * p.D + d] = ACC(j, e);
         }
       } else {
-        // weighted scatter into y (gate 1 for the shared expert)
-        int32_t *s_tok = reinterpret_cast<int32_t *>(xbuf);
-        float *s_gate = reinterpret_cast<float *>(s_tok + BN_MAX);
-        const int et = threadIdx.x - 32 * EPI0;
-        named_bar_sync(5, 32 * EPI);  // the previous tile's readers are done
-        for (int c = et; c < t.nvalid; c += 32 * EPI) {
-          int tok;
-          float gate = 1.0f;
-          if (t.g < p.E) {
-            tok = p.sorted_token[row0 + c];
-            for (int jj = 0; jj < p.k; ++jj)
-              if (p.indices[(size_t)tok * p.k + jj] == t.g) gate = p.weights[(size_t)tok * p.k + jj];
-          } else {
-            tok = t.tok0 + c;
-          }
-          s_tok[c] = tok;
-          s_gate[c] = gate;
-        }
+        // weighted scatter into y (gate 1 for the shared expert); the tile's
+        // token and gate list was written at its start
         named_bar_sync(5, 32 * EPI);
         const int d = t.ft * 256 + (int)rank * BM + q * 32 + lane;
 #pragma unroll
@@ -1297,12 +1285,13 @@ __global__ void __launch_bounds__(NT, 1)
 #pragma unroll
           for (int e = 0; e < 32; ++e)
             if (c0 + e < t.nvalid)
-              atomicAdd(p.y + (size_t)s_tok[c0 + e] * p.D + d, s_gate[c0 + e] * acc[j][e]);
+              atomicAdd(p.y + (size_t)s_tok[c0 + e] * p.D + d, s_gate[c0 + e] * ACC(j, e));
         }
       }
     }
   }
 
+#undef ACC
   __syncthreads();
   if (threadIdx.x == 0 && *abort_flag) {
     // a stalled pipeline stopped early: let copies already issued land (the
@@ -1511,8 +1500,8 @@ int sm_count() {
 struct WsLayout {
   size_t tab, xperm, h, total;
   int64_t rows_pad;
-  // FP8 x FP8 path (e4m3 weights): e4m3 codes and transposed 1 x 128 block
-  // scales of the expert rows (xq, xs) and of h (hq, hs), and h in bf16 (hb)
+  // FP8 x FP8 path (e4m3 weights): e4m3 codes and per-row scales of the
+  // expert rows (xq, xs) and of h (hq, hs), and h in bf16 (hb)
   size_t xq, xs, hb, hq, hs;
 };
 
@@ -1542,13 +1531,13 @@ WsLayout ws_layout(const moe_cfg *c, int64_t T, moe_dtype x_dt, moe_dtype w_dt) 
     l.xq = o;
     o = align_up(o + rp * c->dim, 1024);
     l.xs = o;
-    o = align_up(o + (size_t)(c->dim / 128) * rp * 4, 1024);
+    o = align_up(o + rp * 4, 1024);
     l.hb = o;
     o = align_up(o + rp * c->inter * 2, 1024);
     l.hq = o;
     o = align_up(o + rp * c->inter, 1024);
     l.hs = o;
-    o = align_up(o + (size_t)(c->inter / 128) * rp * 4, 1024);
+    o = align_up(o + rp * 4, 1024);
     if (o > l.total) l.total = o;
   }
   return l;
@@ -1709,7 +1698,6 @@ tc::Params tc_params(const Job &j) {
   p.sA0 = nullptr;
   p.sA1 = nullptr;
   p.sX = nullptr;
-  p.ld_sx = 0;
   p.sh = j.sh;
   return p;
 }
@@ -1810,19 +1798,17 @@ bool e4m3_tmap(CUtensorMap *m, const void *base, uint64_t rows, uint64_t cols, u
 moe_status quantise_rows(const Job &j, const void *src, bool gather, size_t q_off, size_t s_off,
                          int K) {
   const int rows = j.rows_total();
-  const unsigned grid = (unsigned)((rows + 31) / 32);
-  const size_t smem = (size_t)(K / 128) * 32 * sizeof(float);
+  const unsigned grid = (unsigned)((rows + 7) / 8);
   uint32_t *q = reinterpret_cast<uint32_t *>(j.ws + q_off);
   float *sc = reinterpret_cast<float *>(j.ws + s_off);
   if (gather)
-    quant_rows_e4m3<true><<<grid, 256, smem, j.s>>>(static_cast<const uint2 *>(src),
-                                                    j.sorted_token, q, sc, j.rows_routed(), rows,
-                                                    (int)j.T, K, (int)j.l.rows_pad, j.shard_off(),
-                                                    j.sh);
+    quant_rows_e4m3<true><<<grid, 256, 0, j.s>>>(static_cast<const uint2 *>(src), j.sorted_token,
+                                                 q, sc, j.rows_routed(), rows, (int)j.T, K,
+                                                 j.shard_off(), j.sh);
   else
-    quant_rows_e4m3<false><<<grid, 256, smem, j.s>>>(static_cast<const uint2 *>(src), nullptr, q,
-                                                     sc, j.rows_routed(), rows, (int)j.T, K,
-                                                     (int)j.l.rows_pad, j.shard_off(), j.sh);
+    quant_rows_e4m3<false><<<grid, 256, 0, j.s>>>(static_cast<const uint2 *>(src), nullptr, q, sc,
+                                                  j.rows_routed(), rows, (int)j.T, K,
+                                                  j.shard_off(), j.sh);
   return checked_launch("e4m3 row quantiser");
 }
 
@@ -1849,7 +1835,6 @@ moe_status fp8_up(const Job &j) {
   p.sA0 = j.w->s1;
   p.sA1 = j.w->s3;
   p.sX = reinterpret_cast<const float *>(j.ws + j.l.xs);
-  p.ld_sx = (int)j.l.rows_pad;
   prof(1, j.s);
   st = launch_fp8<1, MOE_F8_STAGES>(mw1, mw3, mx, p, j.s);
   prof(2, j.s);
@@ -1878,7 +1863,6 @@ moe_status fp8_down(const Job &j) {
   p.sA0 = j.w->s2;
   p.sA1 = j.w->s2;
   p.sX = reinterpret_cast<const float *>(j.ws + j.l.hs);
-  p.ld_sx = (int)j.l.rows_pad;
   prof(3, j.s);
   if (j.y)
     st = launch_fp8<3, MOE_F8_STAGES>(mw2, mw2, mh, p, j.s);
@@ -2218,19 +2202,13 @@ MOE_EXPORT moe_status moe_experts_forward_combine_ep(
 }
 
 MOE_EXPORT moe_status moe_quantize_e4m3_rows(const void *src, int64_t rows, int32_t K,
-                                             uint8_t *q, float *scales, int64_t ld,
-                                             moe_stream_t stream) {
-  if (rows < 0 || rows >= ((int64_t)1 << 31) || K <= 0 || K % 128 != 0 || ld < rows ||
-      ld >= ((int64_t)1 << 31))
-    return MOE_ERR_INVALID;
+                                             uint8_t *q, float *scales, moe_stream_t stream) {
+  if (rows < 0 || rows >= ((int64_t)1 << 31) || K <= 0 || K % 4 != 0) return MOE_ERR_INVALID;
   if (rows == 0) return MOE_OK;
   if (!src || !q || !scales) return MOE_ERR_INVALID;
-  const unsigned grid = (unsigned)((rows + 31) / 32);
-  const size_t smem = (size_t)(K / 128) * 32 * sizeof(float);
-  if (smem > 48 * 1024) return MOE_ERR_UNSUPPORTED;
-  quant_rows_e4m3<false><<<grid, 256, smem, as_stream(stream)>>>(
+  quant_rows_e4m3<false><<<(unsigned)((rows + 7) / 8), 256, 0, as_stream(stream)>>>(
       static_cast<const uint2 *>(src), nullptr, reinterpret_cast<uint32_t *>(q), scales, 0,
-      (int)rows, 1, K, (int)ld, nullptr, Shard{0, 0, 0, 0});
+      (int)rows, 1, K, nullptr, Shard{0, 0, 0, 0});
   return launch_status();
 }
 

@@ -209,16 +209,16 @@ def combine(shape: BlockShape, weights: torch.Tensor, slot_of: torch.Tensor,
 
 
 def quantize_e4m3_rows(src: torch.Tensor):
-    """moe_quantize_e4m3_rows: (codes [rows, K] uint8, scales [K/128, rows] fp32)
-    of a bf16 [rows, K] matrix, 1 x 128 blocks."""
+    """moe_quantize_e4m3_rows: (codes [rows, K] uint8, scales [rows] fp32) of
+    a bf16 [rows, K] matrix, one scale per row."""
     _check_cuda(src)
     if src.dtype != torch.bfloat16 or src.dim() != 2:
         raise ValueError("src must be a 2-D bf16 tensor")
     rows, K = src.shape
     q = torch.empty(rows, K, dtype=torch.uint8, device=src.device)
-    sc = torch.empty(K // 128, rows, dtype=torch.float32, device=src.device)
+    sc = torch.empty(rows, dtype=torch.float32, device=src.device)
     check(fn("moe_experts", "moe_quantize_e4m3_rows")(src.data_ptr(), rows, K, q.data_ptr(),
-                                                      sc.data_ptr(), rows, _stream()),
+                                                      sc.data_ptr(), _stream()),
           "moe_quantize_e4m3_rows")
     return q, sc
 

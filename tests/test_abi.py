@@ -163,11 +163,11 @@ def test_fp8_activation_path_validation():
     assert call(c, fp8(1), x_dt=0) == UNSUPPORTED              # bf16 activations in
     assert call(v3_cfg(dim=7296), fp8(1)) == UNSUPPORTED       # dim % 256 != 0
     q = fn("moe_experts", "moe_quantize_e4m3_rows")
-    assert q(P, 4, 100, P, P, 4, None) == INVALID              # K % 128 != 0
-    assert q(P, 4, 128, P, P, 3, None) == INVALID              # ld < rows
-    assert q(None, 4, 128, P, P, 4, None) == INVALID
-    assert q(P, -1, 128, P, P, 4, None) == INVALID
-    assert q(None, 0, 128, None, None, 0, None) == 0           # nothing to do
+    assert q(P, 4, 102, P, P, None) == INVALID                 # K % 4 != 0
+    assert q(None, 4, 128, P, P, None) == INVALID
+    assert q(P, 4, 128, P, None, None) == INVALID
+    assert q(P, -1, 128, P, P, None) == INVALID
+    assert q(None, 0, 128, None, None, None) == 0              # nothing to do
 
 
 def test_expert_parallel_plan_and_validation():

@@ -37,7 +37,13 @@ TOL = {"bf16": 2e-2, "e4m3": 5e-2}
 # (measured 1.8e-4 to 2.0e-4).  The bound is 2.5 times that.  e4m3 weights
 # add the fp16 roundings of the expanded weights (about 4.5e-4).
 MEAN_TOL = {"bf16": 5e-4, "e4m3": 1.5e-3}
-CASES = ["v3_decode_t64", "v3_prefill_t4096", "v3_skew_t16384", "v3_fp8_t8192"]
+# (workload, FP8 x FP8 activations)
+CASES = [("v3_decode_t64", False), ("v3_prefill_t4096", False), ("v3_skew_t16384", False),
+         ("v3_fp8_t8192", False), ("v3_fp8_t8192", True)]
+IDS = [n + ("_fp8act" if f else "") for n, f in CASES]
+# the FP8 x FP8 path against the oracle that quantises x and h the same way
+# (bound and mean as derived in test_gpu_fp8act.py)
+FP8ACT_TOL, FP8ACT_MEAN = 5e-2, 2e-3
 N_Y = 64
 
 
@@ -76,11 +82,11 @@ def report(line: dict):
             f.write(json.dumps(line) + "\n")
 
 
-@pytest.mark.parametrize("name", CASES)
-def test_v3_block(name):
+@pytest.mark.parametrize("name,fp8", CASES, ids=IDS)
+def test_v3_block(name, fp8):
     w = WORKLOADS[name]
     x, p = make_block(w)
-    blk = moe.MoEBlock(w.shape, p, w.T, x.dtype)
+    blk = moe.MoEBlock(w.shape, p, w.T, x.dtype, fp8_act=fp8)
     y = blk.forward(x)
     torch.cuda.synchronize()
     assert blk.device_status() == 0
@@ -98,9 +104,11 @@ def test_v3_block(name):
     gpu_flagged = int((gap < 1e-6).sum())
     tokens = sample_tokens(w.T, N_Y).numpy()
     tokens = tokens[rep.same_set[tokens]]
-    y_orc = oracle_y(w, x, p, r, tokens=tokens)
-    err = y_close(y[torch.from_numpy(tokens).cuda()].cpu().numpy(), y_orc, TOL[w.w_format])
-    line = {"workload": name, "T": w.T, "near_ties_oracle": rep.flagged,
+    y_orc = oracle_y(w, x, p, r, tokens=tokens, fp8_act=fp8)
+    err = y_close(y[torch.from_numpy(tokens).cuda()].cpu().numpy(), y_orc,
+                  FP8ACT_TOL if fp8 else TOL[w.w_format])
+    line = {"workload": name + ("_fp8act" if fp8 else ""), "T": w.T,
+            "near_ties_oracle": rep.flagged,
             "near_ties_gpu": gpu_flagged, "set_flips": rep.set_flips,
             "order_flips": rep.order_flips, "max_gate_rel_err": rep.max_w_rel,
             "y_tokens": int(tokens.size), "y_max_err_rms": err,
@@ -115,13 +123,13 @@ def test_v3_block(name):
     torch.cuda.empty_cache()
 
 
-@pytest.mark.parametrize("name", CASES)
-def test_v3_expert_rows(name):
+@pytest.mark.parametrize("name,fp8", CASES, ids=IDS)
+def test_v3_expert_rows(name, fp8):
     """Expert outputs of the full-size launch, row by row, against the oracle."""
     w = WORKLOADS[name]
     sh = w.shape
     x, p = make_block(w)
-    blk = moe.MoEBlock(sh, p, w.T, x.dtype, combine="ordered")
+    blk = moe.MoEBlock(sh, p, w.T, x.dtype, combine="ordered", fp8_act=fp8)
     blk.forward(x)
     torch.cuda.synchronize()
     assert blk.device_status() == 0
@@ -129,8 +137,9 @@ def test_v3_expert_rows(name):
     offsets = blk.offsets.cpu().numpy()
     st = blk.sorted_token.cpu().numpy()
     # the tile height the experts' kernels use for this batch (decode: 32-row
-    # tiles on one SM; otherwise 256-row tiles on an SM pair)
-    rows_max = 32 if w.T * sh.topk <= 16 * sh.n_routed else 256
+    # tiles on one SM; otherwise, and always on the FP8 x FP8 path, 256-row
+    # tiles on an SM pair)
+    rows_max = 32 if w.T * sh.topk <= 16 * sh.n_routed and not fp8 else 256
     nz = np.nonzero(counts)[0]
     chosen = {"hottest": int(nz[np.argmax(counts[nz])]), "smallest": int(nz[np.argmin(counts[nz])])}
     multi = [e for e in nz if len(token_tiles(counts[e], rows_max)) > 1]
@@ -138,10 +147,11 @@ def test_v3_expert_rows(name):
         chosen["straddles_tile"] = int(min(multi, key=lambda e: counts[e]))
     rng = np.random.default_rng(3)
     xs = to_host_f32(x)
-    act = oracle_act(w)
+    act = oracle_act(w, fp8)
+    tol, mean_tol = (FP8ACT_TOL, FP8ACT_MEAN) if fp8 else (TOL[w.w_format], MEAN_TOL[w.w_format])
     get = _expert_getter(p, w.w_format)
     out_perm = blk.out_perm
-    line = {"workload": name}
+    line = {"workload": name + ("_fp8act" if fp8 else "")}
     for tag, e in chosen.items():
         rows = rows_to_check(int(counts[e]), rows_max, rng)
         ref = O.expert_ffn(xs[st[offsets[e] + rows]], *get(e), act)
@@ -151,8 +161,8 @@ def test_v3_expert_rows(name):
         mean = float(np.mean(np.abs(got - ref)) / rms)
         line[tag] = {"expert": e, "rows": int(counts[e]), "checked": int(rows.size),
                      "max": mx, "mean": mean}
-        assert mx <= TOL[w.w_format], (tag, e, mx)
-        assert mean <= MEAN_TOL[w.w_format], (tag, e, mean)
+        assert mx <= tol, (tag, e, mx)
+        assert mean <= mean_tol, (tag, e, mean)
     # shared expert: rows of its first and last token tiles (all T tokens)
     rows = rows_to_check(w.T, rows_max, rng)
     ref = O.expert_ffn(xs[rows], *get(sh.n_routed), act)
@@ -161,7 +171,7 @@ def test_v3_expert_rows(name):
     mx = float(np.max(np.abs(got - ref)) / rms)
     mean = float(np.mean(np.abs(got - ref)) / rms)
     line["shared"] = {"rows": w.T, "checked": int(rows.size), "max": mx, "mean": mean}
-    assert mx <= TOL[w.w_format] and mean <= MEAN_TOL[w.w_format], line["shared"]
+    assert mx <= tol and mean <= mean_tol, line["shared"]
     print(line)
     report(line)
     del blk, x, p, out_perm
