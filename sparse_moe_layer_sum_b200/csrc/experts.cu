@@ -321,6 +321,22 @@ __device__ __forceinline__ float swiglu_h(float a, float u) {
   return __fdividef(a, 1.0f + __expf(-a)) * u;
 }
 
+// L2 priority of the token rows a matmul streams (the expert-ordered x rows
+// in the first, h in the second): 0 evict-first, 1 normal, 2 evict-last.
+// The rows of an expert are re-read by its feature tiles, which run at about
+// the same time, and are dead afterwards.
+#ifndef MOE_TOKEN_L2_UP
+#define MOE_TOKEN_L2_UP 2
+#endif
+#ifndef MOE_TOKEN_L2_DOWN
+#define MOE_TOKEN_L2_DOWN 2
+#endif
+__device__ __forceinline__ uint64_t token_policy(bool up) {
+  const int k = up ? MOE_TOKEN_L2_UP : MOE_TOKEN_L2_DOWN;
+  return k == 0 ? sm100::policy_evict_first()
+                : k == 1 ? sm100::policy_evict_normal() : sm100::policy_evict_last();
+}
+
 // Waits for a barrier phase with a time limit but ignores the abort flag;
 // used only to drain copies already in flight before the CTA exits.
 __device__ __forceinline__ void drain_wait(uint64_t *bar, uint32_t parity, int64_t limit_ns) {
@@ -420,7 +436,7 @@ __global__ void __launch_bounds__(threads_of(F8, AT), 1)
       // fp32 sums it scatters into y need L2 more
       const uint64_t pol_normal = policy_evict_normal();
       const uint64_t pol_first = MODE == 1 ? pol_normal : policy_evict_first();
-      const uint64_t pol_x = policy_evict_last();   // activations: re-read per feature tile
+      const uint64_t pol_x = token_policy(MODE == 1);  // re-read per feature tile
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
@@ -923,6 +939,7 @@ namespace f8 {
 using tc::drain_wait;
 using tc::sleep_ns;
 using tc::swiglu_h;
+using tc::token_policy;
 
 constexpr int BK = 128;                // K per stage: one 128-byte swizzle row of e4m3
 constexpr int BM = 128;                // weight rows per CTA
@@ -1045,7 +1062,7 @@ __global__ void __launch_bounds__(NT, 1)
       // matmul, whose scattered fp32 sums need L2 more; token rows evict-last
       const uint64_t pol_normal = policy_evict_normal();
       const uint64_t pol_first = MODE == 1 ? pol_normal : policy_evict_first();
-      const uint64_t pol_x = policy_evict_last();
+      const uint64_t pol_x = token_policy(MODE == 1);
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
