@@ -964,8 +964,7 @@ constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr int NPBUF = 2;               // TMEM partial-sum buffers of BN_MAX columns
 constexpr int CHUNKS = BN_MAX / 32 / 2;  // 32-column chunks per promotion warp
 constexpr int XB_STRIDE = 17;
-
-template <int STAGES>
+template <int MODE, int STAGES>
 struct Layout {
   static constexpr int BAR_OFF = STAGES * STAGE_BYTES;
   // full, empty per stage; partial full, partial empty per buffer; drain
@@ -995,7 +994,7 @@ template <int MODE, int STAGES>
 __global__ void __launch_bounds__(NT, 1)
     tc_fp8_gemm(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA1,
                 const __grid_constant__ CUtensorMap tmB, const tc::Params p) {
-  using L = Layout<STAGES>;
+  using L = Layout<MODE, STAGES>;
   using namespace sm100;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -1292,8 +1291,8 @@ __global__ void __launch_bounds__(NT, 1)
             if (c0 + e < t.nvalid) out[(r0 + c0 + e) * p.D + d] = ACC(j, e);
         }
       } else {
-        // weighted scatter into y (gate 1 for the shared expert); the tile's
-        // token and gate list was written at its start
+        // weighted scatter into y (gate 1 for the shared expert) with fp32
+        // atomic adds; the tile's token and gate list was written at its start
         named_bar_sync(5, 32 * EPI);
         const int d = t.ft * 256 + (int)rank * BM + q * 32 + lane;
 #pragma unroll
@@ -1307,7 +1306,6 @@ __global__ void __launch_bounds__(NT, 1)
       }
     }
   }
-
 #undef ACC
   __syncthreads();
   if (threadIdx.x == 0 && *abort_flag) {
@@ -1615,7 +1613,7 @@ moe_status checked_launch(const char *where) {
 template <int MODE, int STAGES>
 moe_status launch_fp8(const CUtensorMap &a0, const CUtensorMap &a1, const CUtensorMap &b,
                       const tc::Params &p, cudaStream_t s) {
-  using L = f8::Layout<STAGES>;
+  using L = f8::Layout<MODE, STAGES>;
   auto kern = f8::tc_fp8_gemm<MODE, STAGES>;
   const size_t smem = L::smem_bytes(p.G, p.E);
   if (smem > 232448) return MOE_ERR_UNSUPPORTED;
