@@ -57,6 +57,10 @@ def parse():
     ap.add_argument("--fp8-act", action="store_true",
                     help="e4m3-weight workloads: quantise the activations to e4m3 too "
                          "(FP8 x FP8 matmuls)")
+    ap.add_argument("--parallel", choices=["replicas", "ep"], default="replicas",
+                    help="N>1: independent replicas (weak scaling), or expert parallelism: "
+                         "one batch, the experts split over the ranks, y all-reduced "
+                         "(strong scaling)")
     ap.add_argument("--combine", choices=["scatter", "ordered"], default="scatter",
                     help="weighted sum into y inside the second matmul, or ordered and "
                          "bit-reproducible in a separate pass")
@@ -271,8 +275,10 @@ def time_block(w, blk, xs, K, warmup, world, dev, local_rank):
             "near_ties": ties, "clocks": clk}
 
 
-def rooflines(w, blk, K, tm, fp8_act=False):
-    """Dominant-kernel and whole-step rooflines from the measured timings."""
+def rooflines(w, blk, K, tm, fp8_act=False, share=1.0):
+    """Dominant-kernel and whole-step rooflines from the measured timings.
+    share: the part of the block's expert work one GPU does (1/world under
+    expert parallelism)."""
     sh = w.shape
     peaks, peak_src = load_peaks(ROOT)
     w_bytes = {"bf16": 2, "f32": 4, "e4m3": 1}[w.w_format]
@@ -292,9 +298,10 @@ def rooflines(w, blk, K, tm, fp8_act=False):
 
     dur = tm["dur"]
     dominant = max(("gemm1", "gemm2", "router", "combine", "gather", "dispatch"), key=dur.get)
-    bytes_dom = avg(lambda b: kw[b][dominant].bytes)
-    bytes_meth = avg(lambda b: mb[b][dominant]) if dominant in ("gemm1", "gemm2") else bytes_dom
-    flops_dom = avg(lambda b: kw[b][dominant].flops)
+    bytes_dom = share * avg(lambda b: kw[b][dominant].bytes)
+    bytes_meth = (share * avg(lambda b: mb[b][dominant]) if dominant in ("gemm1", "gemm2")
+                  else bytes_dom)
+    flops_dom = share * avg(lambda b: kw[b][dominant].flops)
     # tensor peak: the sustained (power-capped) figure when the timed loop runs
     # long enough for the clocks to settle under the power cap, else the burst one
     sustained = tm["ms_total"] > 500.0 and "bf16_tflops_sustained" in peaks
@@ -324,8 +331,8 @@ def rooflines(w, blk, K, tm, fp8_act=False):
     roof["method_bytes_per_launch"] = bytes_meth
     roof["impl_bytes_per_launch"] = bytes_dom
     roof["algorithmic_flops_per_launch"] = flops_dom
-    b_alg = avg(lambda b: bw[b].bytes)
-    f_alg = avg(lambda b: bw[b].flops)
+    b_alg = share * avg(lambda b: bw[b].bytes)
+    f_alg = share * avg(lambda b: bw[b].flops)
     ms_step = tm["ms_step"]
     t_roof = max(b_alg / (hbm * 1e9), f_alg / (tflops * 1e12))
     step_roof = {"bytes": b_alg, "flops": f_alg, "t_roof_ms": t_roof * 1e3,
@@ -379,15 +386,25 @@ def run_ours(args, rank, local_rank, world):
     build.build_all()
     w = WORKLOADS[args.workload]
     sh = w.shape
-    xs, params = make_inputs(w, dev, rank)
+    ep = args.parallel == "ep" and world > 1
+    # expert parallelism: every rank holds the same batches and its shard of
+    # the experts; replicas: every rank its own batches and all the experts
+    xs, params = make_inputs(w, dev, 0 if ep else rank)
+    if ep:
+        params = moe.shard_params(sh, params, rank, world)
+        torch.cuda.empty_cache()
     x0 = xs[0]
     blk = moe.MoEBlock(sh, params, w.T, w.x_dtype, device=dev, combine=args.combine,
-                       fp8_act=args.fp8_act)
+                       fp8_act=args.fp8_act, ep=(rank, world) if ep else (0, 1),
+                       ep_group=torch.distributed.group.WORLD if ep else None)
     K = args.steps
     tm = time_block(w, blk, xs, K, args.warmup, world, dev, local_rank)
     ms_total, ms_step = tm["ms_total"], tm["ms_step"]
-    value = job_tokens_per_s(world, w.T, K, ms_total)
-    roof, step_roof, touched = rooflines(w, blk, K, tm, args.fp8_act)
+    # the job's tokens: one batch per step under expert parallelism, one per
+    # replica and step otherwise
+    value = job_tokens_per_s(1 if ep else world, w.T, K, ms_total)
+    roof, step_roof, touched = rooflines(w, blk, K, tm, args.fp8_act,
+                                         share=1.0 / world if ep else 1.0)
     x_bytes = 2 if w.x_dtype == torch.bfloat16 else 4
     w_bytes = {"bf16": 2, "f32": 4, "e4m3": 1}[w.w_format]
 
@@ -412,7 +429,7 @@ def run_ours(args, rank, local_rank, world):
     e1.record()
     torch.cuda.synchronize()
     ms_e2e = max_over_ranks(e0.elapsed_time(e1), world, dev)
-    e2e = {"value": job_tokens_per_s(world, w.T, Ke, ms_e2e), "unit": "tokens/s",
+    e2e = {"value": job_tokens_per_s(1 if ep else world, w.T, Ke, ms_e2e), "unit": "tokens/s",
            "h2d_bytes_per_step": w.T * sh.dim * x_bytes, "d2h_bytes_per_step": w.T * sh.dim * 4,
            "steps": Ke}
 
@@ -420,7 +437,7 @@ def run_ours(args, rank, local_rank, world):
     # launch gaps between the kernels cost (each step copies its batch into
     # the graph's input buffer first, inside the timed region)
     graph = None
-    if not args.no_graph:
+    if not args.no_graph and not ep:  # (no NCCL call inside a captured graph)
         x_g = xs[0].clone()
         side = torch.cuda.Stream(device=dev)
         side.wait_stream(torch.cuda.current_stream())
@@ -488,7 +505,7 @@ def run_ours(args, rank, local_rank, world):
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None,
+        "scaling": "strong" if ep else "weak", "vs_baseline": None,
         # arithmetic type of the matmuls: e4m3 weights are expanded to f16
         # unless the activations are quantised to e4m3 as well
         "dtype": mma_type(w, args.fp8_act),
@@ -498,7 +515,8 @@ def run_ours(args, rank, local_rank, world):
                    "topk": sh.topk, "inter": sh.inter, "weights": w.w_format,
                    "activations": "e4m3 (1x128 blocks)" if args.fp8_act else
                    ("bf16" if w.x_dtype == torch.bfloat16 else "f32"),
-                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                   "parallelism": (f"expert parallel x{world} (NCCL all-reduce of y)" if ep else
+                                   f"replicas x{world}" if world > 1 else "single GPU"),
                    "l2": f"inputs larger than L2: {N_X_BATCHES} rotating x batches and "
                          f"{(sh.n_routed + 1) * 3 * sh.dim * sh.inter * w_bytes / 1e9:.1f} GB "
                          "of expert weights per step"},
