@@ -142,6 +142,36 @@ moe_status moe_experts_forward_combine_ep(const moe_cfg *cfg, int64_t T, const v
                                           moe_stream_t stream);
 
 /*
+ * The whole block for a decode-sized batch in one launch: routing (as
+ * moe_router_forward, with fp32 FMA scores), the token grouping (as
+ * moe_dispatch_build), the experts and the weighted scatter into y (as
+ * moe_experts_forward_combine) run as phases of one persistent kernel with
+ * one block per SM, separated by grid-wide barriers; a CUDA cooperative
+ * launch keeps every block resident.  Each barrier wait is bounded (1 s):
+ * a block that gives up records MOE_ERR_TIMEOUT in dev_status and returns.
+ * No counterpart on the pages beyond the block itself; it removes the
+ * launch gaps between the block's kernels at decode.
+ *   x         [T, dim] bf16; w_r [n_routed, dim] fp32; bias [n_routed] fp32
+ *   w         bf16 expert weights (act_e4m3 = 0)
+ *   weights, indices [T, topk], sel_gap [T] (may be NULL): as moe_router_forward
+ *   counts [n_routed], offsets [n_routed + 1], sorted_token, slot_of
+ *             [T * topk]: as moe_dispatch_build
+ *   y         [T, dim] fp32 out (zeroed by the call first)
+ *   ws        moe_block_decode_workspace_size(cfg, T) bytes
+ * Limits: the decode regime, T * topk <= 16 * n_routed; n_routed <= 256,
+ * n_groups <= 32, topk <= 32, n_shared == 1, dim and inter multiples of 128;
+ * otherwise MOE_ERR_UNSUPPORTED.  T == 0 launches nothing.
+ */
+size_t moe_block_decode_workspace_size(const moe_cfg *cfg, int64_t T);
+moe_status moe_block_forward_decode(const moe_cfg *cfg, int64_t T, const void *x, moe_dtype x_dt,
+                                    const float *w_r, const float *bias,
+                                    const moe_expert_weights *w, float *weights,
+                                    int32_t *indices, float *sel_gap, int32_t *counts,
+                                    int32_t *offsets, int32_t *sorted_token, int32_t *slot_of,
+                                    float *y, void *ws, size_t ws_bytes, int32_t *dev_status,
+                                    moe_stream_t stream);
+
+/*
  * The two halves of moe_experts_forward, for callers that schedule them
  * separately (moe_experts_forward(...) == moe_experts_up(...) followed by
  * moe_experts_down(...) on the same stream and workspace).

@@ -73,6 +73,10 @@ SIGNATURES = {
     ("moe_experts", "moe_experts_forward_combine_ep"): (
         _i32, [_cfgp, _i64, _vp, _i32, ctypes.POINTER(MoEExpertWeights),
                ctypes.POINTER(MoEEpShard), _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp, _vp]),
+    ("moe_experts", "moe_block_decode_workspace_size"): (_sz, [_cfgp, _i64]),
+    ("moe_experts", "moe_block_forward_decode"): (
+        _i32, [_cfgp, _i64, _vp, _i32, _vp, _vp, ctypes.POINTER(MoEExpertWeights), _vp, _vp, _vp,
+               _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp, _vp]),
     ("moe_experts", "moe_experts_up"): (
         _i32, [_cfgp, _i64, _vp, _i32, ctypes.POINTER(MoEExpertWeights), _vp, _vp, _vp, _sz, _vp,
                _vp]),

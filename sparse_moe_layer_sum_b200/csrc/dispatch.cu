@@ -20,31 +20,19 @@
 #include <mutex>
 
 #include "common.cuh"
+#include "dispatch_dev.cuh"
 #include "moe_dispatch.h"
 
 namespace moe {
 namespace {
 
-constexpr int CHUNK_TOKENS = 64;
+using grouping::CHUNK_TOKENS;
 
 __global__ void __launch_bounds__(256) dispatch_hist(const int32_t *__restrict__ idx, int T, int k,
                                                      int E, int32_t *__restrict__ chunk_hist,
                                                      int32_t *status) {
   extern __shared__ int32_t h[];
-  for (int e = threadIdx.x; e < E; e += blockDim.x) h[e] = 0;
-  __syncthreads();
-  const int t0 = blockIdx.x * CHUNK_TOKENS;
-  const int n = min(CHUNK_TOKENS, T - t0) * k;
-  const int32_t *src = idx + (size_t)t0 * k;
-  for (int i = threadIdx.x; i < n; i += blockDim.x) {
-    const int e = src[i];
-    if (e < 0 || e >= E)
-      set_status(status, MOE_ERR_RANGE);
-    else
-      atomicAdd(&h[e], 1);
-  }
-  __syncthreads();
-  for (int e = threadIdx.x; e < E; e += blockDim.x) chunk_hist[(size_t)blockIdx.x * E + e] = h[e];
+  grouping::hist_chunk(idx, T, k, E, blockIdx.x, chunk_hist, status, h);
 }
 
 // One block of >= E threads (E <= 1024).
@@ -53,45 +41,7 @@ __global__ void __launch_bounds__(1024) dispatch_scan(int32_t *__restrict__ chun
                                                       int32_t *__restrict__ counts,
                                                       int32_t *__restrict__ offsets) {
   __shared__ int32_t warp_tot[32];
-  const int e = threadIdx.x;
-  int run = 0;
-  if (e < E) {
-    for (int c = 0; c < nchunks; ++c) {
-      const int v = chunk_hist[(size_t)c * E + e];
-      chunk_hist[(size_t)c * E + e] = run;
-      run += v;
-    }
-    counts[e] = run;
-  }
-  // exclusive scan of run over e: warp inclusive scans, then warp totals
-  const int lane = threadIdx.x % 32, w = threadIdx.x / 32;
-  int v = (e < E) ? run : 0;
-  int inc = v;
-#pragma unroll
-  for (int off = 1; off < 32; off <<= 1) {
-    const int o = __shfl_up_sync(0xffffffffu, inc, off);
-    if (lane >= off) inc += o;
-  }
-  if (lane == 31) warp_tot[w] = inc;
-  __syncthreads();
-  if (w == 0) {
-    const int nw = (blockDim.x + 31) / 32;
-    int t = lane < nw ? warp_tot[lane] : 0;
-    int tinc = t;
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-      const int o = __shfl_up_sync(0xffffffffu, tinc, off);
-      if (lane >= off) tinc += o;
-    }
-    warp_tot[lane] = tinc - t;  // exclusive prefix of the warp totals
-  }
-  __syncthreads();
-  const int excl = inc - v + warp_tot[w];
-  if (e < E) {
-    offsets[e] = excl;
-    if (e == E - 1) offsets[E] = excl + v;
-    for (int c = 0; c < nchunks; ++c) chunk_hist[(size_t)c * E + e] += excl;
-  }
+  grouping::scan_chunks(chunk_hist, nchunks, E, counts, offsets, warp_tot);
 }
 
 // One warp per chunk.
@@ -101,31 +51,7 @@ __global__ void __launch_bounds__(32) dispatch_scatter(const int32_t *__restrict
                                                        int32_t *__restrict__ sorted_token,
                                                        int32_t *__restrict__ slot_of) {
   extern __shared__ int32_t base[];
-  const int lane = threadIdx.x;
-  for (int e = lane; e < E; e += 32) base[e] = chunk_base[(size_t)blockIdx.x * E + e];
-  __syncwarp();
-  const int t0 = blockIdx.x * CHUNK_TOKENS;
-  const int n = min(CHUNK_TOKENS, T - t0) * k;
-  const size_t flat0 = (size_t)t0 * k;
-  const unsigned lt = (1u << lane) - 1u;
-  for (int i0 = 0; i0 < n; i0 += 32) {
-    const int i = i0 + lane;
-    int e = -1;
-    if (i < n) e = idx[flat0 + i];
-    const bool ok = i < n && e >= 0 && e < E;
-    const int key = ok ? e : -1 - lane;  // invalid lanes get a key of their own
-    const unsigned same = __match_any_sync(0xffffffffu, key);
-    if (ok) {
-      const int rank = __popc(same & lt);
-      const int pos = base[e] + rank;
-      sorted_token[pos] = t0 + i / k;
-      slot_of[flat0 + i] = pos;
-    }
-    __syncwarp();
-    // the highest lane of each group advances that expert's next free row
-    if (ok && (same >> lane) == 1u) base[e] += __popc(same);
-    __syncwarp();
-  }
+  grouping::scatter_chunk(idx, T, k, E, blockIdx.x, chunk_base, sorted_token, slot_of, base);
 }
 
 // ------------------------------------------------- no-allocation variant

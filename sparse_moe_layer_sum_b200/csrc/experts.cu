@@ -41,6 +41,8 @@
 
 #include "common.cuh"
 #include "moe_experts.h"
+#include "dispatch_dev.cuh"
+#include "route.cuh"
 #include "sm100.cuh"
 
 namespace moe {
@@ -87,9 +89,9 @@ __device__ __forceinline__ int group_rows(int g, const int32_t *off, int E, cons
 }
 
 // One warp: lane l owns a contiguous run of groups.
-__global__ void __launch_bounds__(32) prep_tiles(const int32_t *__restrict__ offsets, int E,
-                                                 int G, Shard sh, Tiling t0, Tiling t1) {
-  const int lane = threadIdx.x;
+__device__ __forceinline__ void prep_tiles_warp(const int32_t *__restrict__ offsets, int E, int G,
+                                                Shard sh, Tiling t0, Tiling t1) {
+  const int lane = threadIdx.x % 32;
   const int per = (G + 31) / 32;
   const int g0 = min(G, lane * per), g1 = min(G, g0 + per);
   for (int which = 0; which < 2; ++which) {
@@ -119,6 +121,11 @@ __global__ void __launch_bounds__(32) prep_tiles(const int32_t *__restrict__ off
     }
     if (lane == 31) tl.tile_start[G] = inc;
   }
+}
+
+__global__ void __launch_bounds__(32) prep_tiles(const int32_t *__restrict__ offsets, int E,
+                                                 int G, Shard sh, Tiling t0, Tiling t1) {
+  prep_tiles_warp(offsets, E, G, sh, t0, t1);
 }
 
 // g: group (routed expert, then the shared expert); wg: its index in the
@@ -352,15 +359,17 @@ __device__ __forceinline__ void sleep_ns(int64_t ns) {
   }
 }
 
+// The body of the expert GEMM kernel, over the shared memory `sm` (1024-byte
+// aligned).  Warps beyond the variant's roles (in a larger block that runs
+// it as one phase) take no part but the block-wide barriers.  A CTA that will
+// allocate tensor memory again later (a later phase) passes last_alloc =
+// false, so that it keeps its right to allocate.
 template <int MODE, int CG, int AT, int BN_MAX, int BOXN, int STAGES, bool F8>
-__global__ void __launch_bounds__(threads_of(F8, AT), 1)
-    tc_expert_gemm(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA1,
-                   const __grid_constant__ CUtensorMap tmB, const Params p) {
+__device__ __forceinline__ void gemm_body(const CUtensorMap &tmA0, const CUtensorMap &tmA1,
+                                          const CUtensorMap &tmB, const Params &p, uint8_t *sm,
+                                          bool last_alloc = true) {
   using L = Layout<MODE, CG, AT, BN_MAX, BOXN, STAGES, F8>;
   using namespace sm100;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                            ~static_cast<uintptr_t>(1023));
   uint64_t *full = reinterpret_cast<uint64_t *>(sm + L::BAR_OFF);
   uint64_t *empty = full + STAGES;
   uint64_t *a8full = empty + STAGES;                 // F8 only
@@ -406,17 +415,17 @@ __global__ void __launch_bounds__(threads_of(F8, AT), 1)
     if (MODE == 1) tma_prefetch_desc(&tmA1);
     tma_prefetch_desc(&tmB);
   }
-  constexpr int NT = L::NT;
+  const int NT = blockDim.x;
   for (int i = threadIdx.x; i <= p.G; i += NT) s_tstart[i] = p.tile_start[i];
   for (int i = threadIdx.x; i < p.G; i += NT) s_tbase[i] = p.tile_base[i];
   for (int i = threadIdx.x; i <= p.E; i += NT) s_off[i] = p.offsets[i];
   if (warp == 1) {
     if (CG == 2) {
       tmem_alloc_pair(tmem_slot, L::TMEM_COLS);
-      tmem_relinquish_pair();
+      if (last_alloc) tmem_relinquish_pair();
     } else {
       tmem_alloc(tmem_slot, L::TMEM_COLS);
-      tmem_relinquish();
+      if (last_alloc) tmem_relinquish();
     }
   }
   tc_fence_before();
@@ -853,6 +862,16 @@ __global__ void __launch_bounds__(threads_of(F8, AT), 1)
     else
       tmem_dealloc(tmem_base, L::TMEM_COLS);
   }
+}
+
+template <int MODE, int CG, int AT, int BN_MAX, int BOXN, int STAGES, bool F8>
+__global__ void __launch_bounds__(threads_of(F8, AT), 1)
+    tc_expert_gemm(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA1,
+                   const __grid_constant__ CUtensorMap tmB, const Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                            ~static_cast<uintptr_t>(1023));
+  gemm_body<MODE, CG, AT, BN_MAX, BOXN, STAGES, F8>(tmA0, tmA1, tmB, p, sm);
 }
 
 // single-CTA self-test of the bounded wait: nothing ever arrives
@@ -1327,6 +1346,167 @@ __global__ void __launch_bounds__(NT, 1)
 }
 
 }  // namespace f8
+
+// ------------------------------------------------ fused decode block
+//
+// The whole block for a decode-sized batch in one persistent, cooperative
+// launch (one CTA per SM): the router (fp32 FMA scores, then the selection),
+// the token grouping and both tile tables, the row gather, the first matmul
+// and the second with the weighted scatter into y, as phases separated by
+// grid-wide barriers.  Each phase runs the same device code as the separate
+// kernels; the launch gaps between them go away.  Every barrier wait is
+// bounded: a CTA that waits too long records MOE_ERR_TIMEOUT and returns.
+
+namespace fused {
+
+constexpr int THREADS = 256;  // the router's tile shape; the GEMM phases use six warps of it
+
+struct Args {
+  const __nv_bfloat16 *x;  // [T, D]
+  const float *w_r;        // [E, D]
+  float *z_part;           // [nsplit, T, E]
+  int nsplit, cols_per_split;
+  route::SelectArgs sel;   // the selection's inputs and outputs
+  int32_t *chunk_hist;     // [nchunks, E]
+  int nchunks;
+  int32_t *counts, *offsets, *sorted_token, *slot_of;
+  Tiling t1, t2;           // the two matmuls' tile tables
+  Shard sh;
+  uint4 *xperm;            // expert-contiguous rows of x
+  float *y;                // [T, D]
+  int32_t *status;
+  unsigned *bar;           // grid barrier: arrivals, generation (zero at launch)
+  int64_t timeout_ns;
+  int T, D, E, G, k, rows_routed, rows_total;
+};
+
+// All CTAs meet; false (after recording MOE_ERR_TIMEOUT) when this CTA gave
+// up waiting.  Thread 0 arrives on the arrival counter and waits for the
+// generation to move on; the last to arrive resets the counter and moves it.
+__device__ __forceinline__ bool grid_sync(const Args &a, int *flag) {
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int ok = 1;
+    volatile unsigned *gen = a.bar + 1;
+    __threadfence();
+    const unsigned g = *gen;
+    if (atomicAdd(a.bar, 1u) == gridDim.x - 1) {
+      atomicExch(a.bar, 0u);
+      __threadfence();
+      atomicAdd(a.bar + 1, 1u);
+    } else {
+      const uint64_t t0 = sm100::globaltimer_ns();
+      while (*gen == g) {
+        if ((int64_t)(sm100::globaltimer_ns() - t0) > a.timeout_ns) {
+          set_status(a.status, MOE_ERR_TIMEOUT);
+          ok = 0;
+          break;
+        }
+        __nanosleep(100);
+      }
+    }
+    __threadfence();
+    *flag = ok;
+  }
+  __syncthreads();
+  return *flag != 0;
+}
+
+template <int BN, int STAGES>
+__global__ void __launch_bounds__(THREADS, 1)
+    decode_block(const __grid_constant__ CUtensorMap tmW1, const __grid_constant__ CUtensorMap tmW3,
+                 const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW2,
+                 const __grid_constant__ CUtensorMap tmH, const Args a, const tc::Params p1,
+                 const tc::Params p2) {
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ int s_flag;
+  uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                            ~static_cast<uintptr_t>(1023));
+  const int warp = threadIdx.x / 32;
+  const int nwarps = gridDim.x * (THREADS / 32);
+  const int gwarp = blockIdx.x * (THREADS / 32) + warp;
+  const int T = a.T, E = a.E, D = a.D;
+
+  // 1. y = 0; router scores z = x W_r^T in tiles of 64 tokens x 64 experts
+  //    x one split of dim
+  {
+    float4 *y4 = reinterpret_cast<float4 *>(a.y);
+    const size_t n4 = (size_t)T * D / 4;
+    for (size_t i = (size_t)blockIdx.x * THREADS + threadIdx.x; i < n4;
+         i += (size_t)gridDim.x * THREADS)
+      y4[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+    auto xs = reinterpret_cast<float(*)[route::SC_BM + 4]>(sm);
+    auto ws = reinterpret_cast<float(*)[route::SC_BN + 4]>(
+        sm + route::SC_BK * (route::SC_BM + 4) * sizeof(float));
+    const int mt = (T + route::SC_BM - 1) / route::SC_BM;
+    const int nt = (E + route::SC_BN - 1) / route::SC_BN;
+    const int ntiles = mt * nt * a.nsplit;
+    for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
+      const int split = tile / (mt * nt), r = tile - split * (mt * nt);
+      route::scores_tile(a.x, a.w_r, a.z_part, T, E, D, a.cols_per_split,
+                         (r / nt) * route::SC_BM, (r % nt) * route::SC_BN, split, xs, ws);
+      __syncthreads();
+    }
+  }
+  if (!grid_sync(a, &s_flag)) return;
+
+  // 2. selection: one warp per token
+  {
+    float *s = reinterpret_cast<float *>(sm) + (size_t)warp * 2 * E;
+    for (int t = gwarp; t < T; t += nwarps) route::select_token(a.sel, t, s, s + E);
+  }
+  if (!grid_sync(a, &s_flag)) return;
+
+  // 3. the grouping and both tile tables (one CTA)
+  if (blockIdx.x == 0) {
+    int32_t *h = reinterpret_cast<int32_t *>(sm);
+    int32_t *wt = h + E;
+    int32_t *base = wt + 32;
+    for (int c = 0; c < a.nchunks; ++c) {
+      grouping::hist_chunk(a.sel.indices, T, a.k, E, c, a.chunk_hist, a.status, h);
+      __syncthreads();
+    }
+    grouping::scan_chunks(a.chunk_hist, a.nchunks, E, a.counts, a.offsets, wt);
+    __syncthreads();
+    if (warp == 0)
+      for (int c = 0; c < a.nchunks; ++c)
+        grouping::scatter_chunk(a.sel.indices, T, a.k, E, c, a.chunk_hist, a.sorted_token,
+                                a.slot_of, base);
+    __syncthreads();
+    if (warp == 1) prep_tiles_warp(a.offsets, E, a.G, a.sh, a.t1, a.t2);
+  }
+  if (!grid_sync(a, &s_flag)) return;
+
+  // 4. the expert-contiguous rows (one warp per row), then made visible to
+  //    the TMA loads of the next phase
+  {
+    const int vec = D * 2 / 16;
+    const uint4 *x4 = reinterpret_cast<const uint4 *>(a.x);
+    const int lane = threadIdx.x % 32;
+    for (int row = gwarp; row < a.rows_total; row += nwarps) {
+      const int src = row < a.rows_routed ? a.sorted_token[row] : row - a.rows_routed;
+      const uint4 *s = x4 + (size_t)src * vec;
+      uint4 *d = a.xperm + (size_t)row * vec;
+      for (int v = lane; v < vec; v += 32) d[v] = __ldg(s + v);
+    }
+    sm100::fence_proxy_async_global();
+  }
+  if (!grid_sync(a, &s_flag)) return;
+  sm100::fence_proxy_async_global();  // (the reading side of the same ordering)
+
+  // 5. first matmul + SwiGLU (h is then made visible to the next TMA loads);
+  //    this CTA allocates tensor memory again in phase 6, so it keeps the
+  //    right to allocate
+  tc::gemm_body<1, 1, 1, BN, 32, STAGES, false>(tmW1, tmW3, tmX, p1, sm, false);
+  sm100::fence_proxy_async_global();
+  if (!grid_sync(a, &s_flag)) return;
+  sm100::fence_proxy_async_global();
+
+  // 6. second matmul, gate times output added into y
+  tc::gemm_body<3, 1, 1, BN, 32, STAGES, false>(tmW2, tmW2, tmH, p2, sm, true);
+}
+
+}  // namespace fused
 
 // ----------------------------------------------------------- CUDA-core path
 
@@ -2091,6 +2271,142 @@ moe_status make_job(Job &j, const moe_cfg *cfg, int64_t T, const void *x, moe_dt
   return MOE_OK;
 }
 
+// ------------------------------------------------ fused decode block (host)
+
+struct DecodePlan {
+  int nsplit, cols_per_split, nchunks;
+  size_t z_off, hist_off, ex_off, total;
+  WsLayout l;
+};
+
+// Workspace of the fused decode launch: the grid barrier's two words, the
+// router's split partial scores (sized for the most splits, dim / 256), the
+// grouping's chunk histograms, then the experts' workspace.
+DecodePlan decode_plan(const moe_cfg *c, int64_t T, int grid) {
+  DecodePlan d;
+  const int mt = (int)((T + route::SC_BM - 1) / route::SC_BM);
+  const int nt = (c->n_routed + route::SC_BN - 1) / route::SC_BN;
+  const int max_split = c->dim / 256 > 1 ? c->dim / 256 : 1;
+  int ns = grid > 0 ? (grid + mt * nt - 1) / (mt * nt) : 1;
+  ns = ns < 1 ? 1 : (ns > max_split ? max_split : ns);
+  int cps = (c->dim + ns - 1) / ns;
+  cps = (cps + route::SC_BK - 1) / route::SC_BK * route::SC_BK;
+  d.nsplit = (c->dim + cps - 1) / cps;
+  d.cols_per_split = cps;
+  d.nchunks = (int)((T + grouping::CHUNK_TOKENS - 1) / grouping::CHUNK_TOKENS);
+  if (d.nchunks < 1) d.nchunks = 1;
+  d.z_off = 256;
+  d.hist_off = align_up(d.z_off + (size_t)max_split * T * c->n_routed * 4, 256);
+  d.ex_off = align_up(d.hist_off + (size_t)d.nchunks * c->n_routed * 4, 1024);
+  d.l = ws_layout(c, T, MOE_BF16, MOE_BF16);
+  d.total = d.ex_off + d.l.total;
+  return d;
+}
+
+// the decode tile shape of the expert GEMMs (one SM per tile)
+template <int BN, int STAGES>
+moe_status launch_decode_block(const Job &j, const DecodePlan &pl, const float *w_r,
+                               const float *bias, float *weights, int32_t *indices,
+                               float *sel_gap, int32_t *counts, int32_t *slot_of) {
+  using L1 = tc::Layout<1, 1, 1, BN, 32, STAGES, false>;
+  using L3 = tc::Layout<3, 1, 1, BN, 32, STAGES, false>;
+  const moe_cfg *c = j.c;
+  const int G = j.G(), D = c->dim, I = c->inter, E = c->n_routed;
+  const int nsm = sm_count();
+  if (nsm < 1) return MOE_ERR_CUDA;
+  int32_t *tab = j.tab();
+  Tiling t1{BN, I / L1::FEAT, tab, tab + (G + 1)};
+  Tiling t2{BN, D / L3::FEAT, tab + (2 * G + 1), tab + (3 * G + 2)};
+  bf16 *xperm = reinterpret_cast<bf16 *>(j.ws + j.l.xperm);
+  bf16 *h = reinterpret_cast<bf16 *>(j.ws + j.l.h);
+  CUtensorMap mw1, mw3, mx, mw2, mh;
+  if (!weight_tmap(&mw1, j.w->w1, false, (uint64_t)G * I, D, L1::PART_ROWS) ||
+      !weight_tmap(&mw3, j.w->w3, false, (uint64_t)G * I, D, L1::PART_ROWS) ||
+      !make_tmap(&mx, xperm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)j.l.rows_pad, D, 32,
+                 64) ||
+      !weight_tmap(&mw2, j.w->w2, false, (uint64_t)G * D, I, tc::BM) ||
+      !make_tmap(&mh, h, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)j.l.rows_pad, I, 32, 64))
+    return cuda_fail("fused decode tensor maps", cudaErrorInvalidValue);
+  tc::Params p1 = tc_params(j);
+  p1.tile_start = t1.tile_start;
+  p1.tile_base = t1.tile_base;
+  p1.KB = D / tc::BK;
+  p1.out = h;
+  tc::Params p2 = tc_params(j);
+  p2.tile_start = t2.tile_start;
+  p2.tile_base = t2.tile_base;
+  p2.KB = I / tc::BK;
+  p2.out = nullptr;
+
+  fused::Args a;
+  uint8_t *ws = static_cast<uint8_t *>(j.ws) - pl.ex_off;  // the whole workspace
+  a.x = static_cast<const __nv_bfloat16 *>(j.x);
+  a.w_r = w_r;
+  a.z_part = reinterpret_cast<float *>(ws + pl.z_off);
+  a.nsplit = pl.nsplit;
+  a.cols_per_split = pl.cols_per_split;
+  a.sel.z_part = a.z_part;
+  a.sel.nsplit = pl.nsplit;
+  a.sel.bias = c->has_bias ? bias : nullptr;
+  a.sel.weights = weights;
+  a.sel.indices = indices;
+  a.sel.sel_gap = sel_gap;
+  a.sel.T = (int)j.T;
+  a.sel.E = E;
+  a.sel.G = c->n_groups;
+  a.sel.Gk = c->topk_groups;
+  a.sel.k = c->topk;
+  a.sel.route_scale = c->route_scale;
+  a.sel.softmax = c->score_func == MOE_SCORE_SOFTMAX;
+  a.chunk_hist = reinterpret_cast<int32_t *>(ws + pl.hist_off);
+  a.nchunks = pl.nchunks;
+  a.counts = counts;
+  a.offsets = const_cast<int32_t *>(j.offsets);
+  a.sorted_token = const_cast<int32_t *>(j.sorted_token);
+  a.slot_of = slot_of;
+  a.t1 = t1;
+  a.t2 = t2;
+  a.sh = j.sh;
+  a.xperm = reinterpret_cast<uint4 *>(xperm);
+  a.y = j.y;
+  a.status = j.status;
+  a.bar = reinterpret_cast<unsigned *>(ws);
+  a.timeout_ns = 1000000000LL;
+  a.T = (int)j.T;
+  a.D = D;
+  a.E = E;
+  a.G = G;
+  a.k = c->topk;
+  a.rows_routed = j.rows_routed();
+  a.rows_total = j.rows_total();
+
+  size_t smem = L1::smem_bytes(G, E);
+  if (L3::smem_bytes(G, E) > smem) smem = L3::smem_bytes(G, E);
+  const size_t sel_smem = 1024 + (size_t)(fused::THREADS / 32) * 2 * E * sizeof(float);
+  if (sel_smem > smem) smem = sel_smem;
+  if (smem > 232448 - 16) return MOE_ERR_UNSUPPORTED;
+  auto kern = fused::decode_block<BN, STAGES>;
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail("before the fused decode launch", e);
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return cuda_fail("fused decode shared memory", e);
+  e = cudaMemsetAsync(a.bar, 0, 2 * sizeof(unsigned), j.s);
+  if (e != cudaSuccess) return cuda_fail("fused decode barrier reset", e);
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;  // every CTA resident: the grid barriers need it
+  attr[0].val.cooperative = 1;
+  cfg.gridDim = dim3(nsm);
+  cfg.blockDim = dim3(fused::THREADS);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = j.s;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, kern, mw1, mw3, mx, mw2, mh, a, p1, p2);
+  if (e != cudaSuccess) return cuda_fail("fused decode launch", e);
+  return checked_launch("fused decode launch");
+}
+
 }  // namespace
 }  // namespace moe
 
@@ -2225,6 +2541,45 @@ MOE_EXPORT moe_status moe_quantize_e4m3_rows(const void *src, int64_t rows, int3
       static_cast<const uint2 *>(src), nullptr, reinterpret_cast<uint32_t *>(q), scales, 0,
       (int)rows, 1, K, nullptr, Shard{0, 0, 0, 0});
   return launch_status();
+}
+
+MOE_EXPORT size_t moe_block_decode_workspace_size(const moe_cfg *cfg, int64_t T) {
+  if (check_cfg(cfg) != MOE_OK || T < 0) return 0;
+  return decode_plan(cfg, T, 0).total;
+}
+
+MOE_EXPORT moe_status moe_block_forward_decode(
+    const moe_cfg *cfg, int64_t T, const void *x, moe_dtype x_dt, const float *w_r,
+    const float *bias, const moe_expert_weights *w, float *weights, int32_t *indices,
+    float *sel_gap, int32_t *counts, int32_t *offsets, int32_t *sorted_token, int32_t *slot_of,
+    float *y, void *ws, size_t ws_bytes, int32_t *dev_status, moe_stream_t stream) {
+  moe_status st = check_cfg(cfg);
+  if (st != MOE_OK) return st;
+  if (T < 0) return MOE_ERR_INVALID;
+  if (!w) return MOE_ERR_INVALID;
+  if (x_dt != MOE_BF16 || w->w_dt != MOE_BF16 || w->act_e4m3) return MOE_ERR_UNSUPPORTED;
+  if (cfg->n_shared != 1 || cfg->n_routed > 256 || cfg->n_groups > 32 || cfg->topk > 32 ||
+      cfg->dim % 128 != 0 || cfg->inter % 128 != 0)
+    return MOE_ERR_UNSUPPORTED;
+  // the decode regime: at most 16 rows per expert on average
+  if (T * cfg->topk > (int64_t)16 * cfg->n_routed) return MOE_ERR_UNSUPPORTED;
+  if (T == 0) return MOE_OK;
+  if (!x || !w_r || !weights || !indices || !counts || !offsets || !sorted_token || !slot_of ||
+      !y || !ws || (cfg->has_bias && !bias))
+    return MOE_ERR_INVALID;
+  const DecodePlan pl = decode_plan(cfg, T, sm_count());
+  if (ws_bytes < decode_plan(cfg, T, 0).total) return MOE_ERR_WORKSPACE;
+  Job j;
+  st = make_job(j, cfg, T, x, x_dt, w, offsets, sorted_token, y, y, static_cast<uint8_t *>(ws) + pl.ex_off,
+                ws_bytes - pl.ex_off, dev_status, stream, true, true);
+  if (st != MOE_OK) return st;
+  j.out_perm = nullptr;
+  j.out_shared = nullptr;
+  j.indices = indices;
+  j.weights = weights;
+  j.y = y;
+  return launch_decode_block<DC_BN, DC_ST>(j, pl, w_r, bias, weights, indices, sel_gap, counts,
+                                           slot_of);
 }
 
 MOE_EXPORT moe_status moe_experts_set_profile_events(void *const *events, int32_t n) {

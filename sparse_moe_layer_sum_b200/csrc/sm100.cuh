@@ -85,6 +85,12 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+// Orders this thread's generic-proxy global-memory writes before later
+// async-proxy (TMA) reads of them.
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
 // Waits for the phase with the given parity to complete, for at most
 // limit_ns.  Returns false (after raising *abort and recording
 // MOE_ERR_TIMEOUT) when the limit expires, or false at once when another

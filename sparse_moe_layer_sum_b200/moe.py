@@ -288,7 +288,7 @@ class MoEBlock:
 
     def __init__(self, shape: BlockShape, params: BlockParams, T: int, x_dtype: torch.dtype,
                  device=None, combine: str = "scatter", fp8_act: bool = False,
-                 ep: tuple = (0, 1), ep_group=None):
+                 ep: tuple = (0, 1), ep_group=None, fused_decode: bool = False):
         if combine not in ("scatter", "ordered"):
             raise ValueError(combine)
         # expert parallelism: (rank, world); params then hold the rank's
@@ -298,6 +298,11 @@ class MoEBlock:
         self.ep_group = ep_group
         if self.ep_world > 1 and combine != "scatter":
             raise ValueError("expert parallelism uses the scatter combine")
+        # the whole block in one launch (moe_block_forward_decode): decode
+        # batches, bf16, scatter combine, one GPU
+        self.fused_decode = fused_decode
+        if fused_decode and (combine != "scatter" or fp8_act or self.ep_world > 1):
+            raise ValueError("the fused decode launch uses the scatter combine on one GPU")
         if fp8_act and params.s1 is None:
             raise ValueError("fp8_act needs e4m3 expert weights")
         self.fp8_act = fp8_act
@@ -338,6 +343,8 @@ class MoEBlock:
                            if shape.n_shared else None)
         self.y = torch.empty(T, D, dtype=f32, device=dev)
         self.status = torch.zeros(1, dtype=i32, device=dev)
+        self.ws_fused = (_ws(fn("moe_experts", "moe_block_decode_workspace_size")(cfgp, T), dev)
+                         if fused_decode else None)
 
     # kernels one forward launches: router 2 (scores, selection; the weight
     # split is prepared once), dispatch 3, experts 5 on the
@@ -346,6 +353,8 @@ class MoEBlock:
     # or nothing (scatter; y is zeroed by a memset node)
     @property
     def launches_per_forward(self) -> int:
+        if self.fused_decode:
+            return 1  # (plus a 8-byte memset of its grid barrier)
         sh = self.shape
         tc_router = (self.x_dtype == torch.bfloat16 and sh.n_routed % 128 == 0
                      and sh.dim % 64 == 0 and self.T >= 32)
@@ -423,17 +432,36 @@ class MoEBlock:
             y = self.y
         assert y.shape == (self.T, self.shape.dim) and y.dtype == torch.float32 and y.is_contiguous()
         cfgp, s = ctypes.byref(self.cfg), _stream()
+        if self.fused_decode:
+            self._fused(x, cfgp, s, y)
+            return y
         self._router(x, cfgp, s)
         self._dispatch(cfgp, s)
         self._experts(x, cfgp, s, y)
         self._combine(cfgp, s, y)
         return y
 
+    def _fused(self, x, cfgp, s, y):
+        p = self.p
+        check(fn("moe_experts", "moe_block_forward_decode")(
+            cfgp, self.T, x.data_ptr(), _dt(x), p.w_r.data_ptr(), _ptr(p.bias),
+            ctypes.byref(self.wstruct), self.weights.data_ptr(), self.indices.data_ptr(),
+            self.sel_gap.data_ptr(), self.counts.data_ptr(), self.offsets.data_ptr(),
+            self.sorted_token.data_ptr(), self.slot_of.data_ptr(), y.data_ptr(),
+            self.ws_fused.data_ptr(), self.ws_fused.numel(), self.status.data_ptr(), s),
+            "moe_block_forward_decode")
+
     def forward_profiled(self, x: torch.Tensor, ev) -> torch.Tensor:
         """forward() with 10 CUDA events recorded on the stream: around the
         router [0,1], dispatch [1,2], the row gather [3,4], the two expert
         GEMMs [4,5] and [6,7], and the combine [8,9]."""
         cfgp, s = ctypes.byref(self.cfg), _stream()
+        if self.fused_decode:  # one launch: the whole step is the router's span
+            ev[0].record()
+            self._fused(x, cfgp, s, self.y)
+            for e in ev[1:]:
+                e.record()
+            return self.y
         ev[0].record()
         self._router(x, cfgp, s)
         ev[1].record()

@@ -195,6 +195,28 @@ def test_expert_parallel_plan_and_validation():
              1 << 40, None, None) == 0                          # empty batch
 
 
+def test_fused_decode_validation():
+    size = fn("moe_experts", "moe_block_decode_workspace_size")
+    f = fn("moe_experts", "moe_block_forward_decode")
+    c = v3_cfg()
+    assert size(ctypes.byref(c), 64) > size(ctypes.byref(c), 8) > 0
+    assert size(ctypes.byref(v3_cfg(topk=200)), 8) == 0
+    w = MoEExpertWeights(0x1000, 0x1000, 0x1000, 1, None, None, None)
+
+    def call(cfg=c, T=64, x_dt=1, wt=w, ws=1 << 40, x=P):
+        return f(ctypes.byref(cfg), T, x, x_dt, P, P, ctypes.byref(wt), P, P, None, P, P, P, P, P,
+                 P, ws, None, None)
+    assert call(T=4096) == UNSUPPORTED                          # not a decode batch
+    assert call(x_dt=0) == UNSUPPORTED                          # bf16 x only
+    fp8 = MoEExpertWeights(0x1000, 0x1000, 0x1000, 2, 0x1000, 0x1000, 0x1000)
+    assert call(wt=fp8) == UNSUPPORTED                          # bf16 weights only
+    assert call(cfg=v3_cfg(n_routed=512, n_groups=8)) == UNSUPPORTED
+    assert call(x=None) == INVALID
+    assert call(ws=1024) == WORKSPACE
+    assert call(T=0) == 0                                       # empty batch
+    assert call(T=-1) == INVALID
+
+
 def test_combine_and_selftest_validation():
     f = fn("moe_combine", "moe_combine")
     c = v3_cfg()
