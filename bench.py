@@ -36,8 +36,10 @@ METRIC = "MoE block tokens/s (V3 shape, bf16, T=4096) and % of roofline on 1 B20
 N_X_BATCHES = 4  # rotating input batches: with the 22.6 GB of weights, > L2 per step
 # the other configurations timed in short loops after the headline one:
 # (workload, FP8 x FP8 activations)
-OTHER_CONFIGS = [("v3_decode_t64", False), ("v3_skew_t16384", False), ("v3_fp8_t8192", False),
-                 ("v3_fp8_t8192", True)]
+# (workload, variant): "" the default kernels, "fp8act" FP8 x FP8 matmuls,
+# "fused" the whole block in one launch (decode)
+OTHER_CONFIGS = [("v3_decode_t64", ""), ("v3_decode_t64", "fused"), ("v3_skew_t16384", ""),
+                 ("v3_fp8_t8192", ""), ("v3_fp8_t8192", "fp8act")]
 
 
 def parse():
@@ -57,6 +59,8 @@ def parse():
     ap.add_argument("--fp8-act", action="store_true",
                     help="e4m3-weight workloads: quantise the activations to e4m3 too "
                          "(FP8 x FP8 matmuls)")
+    ap.add_argument("--fused-decode", action="store_true",
+                    help="decode batches: the whole block in one persistent launch")
     ap.add_argument("--parallel", choices=["replicas", "ep"], default="replicas",
                     help="N>1: independent replicas (weak scaling), or expert parallelism: "
                          "one batch, the experts split over the ranks, y all-reduced "
@@ -297,10 +301,18 @@ def rooflines(w, blk, K, tm, fp8_act=False, share=1.0):
         return sum(f(b) * steps_per_batch[b] for b in range(N_X_BATCHES)) / K
 
     dur = tm["dur"]
-    dominant = max(("gemm1", "gemm2", "router", "combine", "gather", "dispatch"), key=dur.get)
+    if getattr(blk, "fused_decode", False):
+        # one launch: its span is recorded as the router's; its work is the block's
+        dur = {"fused_block": dur["router"], "router": 0.0, "dispatch": 0.0, "gather": 0.0,
+               "gemm1": 0.0, "gemm2": 0.0, "combine": 0.0}
+        for b in range(len(kw)):
+            kw[b]["fused_block"] = bw[b]
+            mb[b]["fused_block"] = bw[b].bytes
+    dominant = max(("gemm1", "gemm2", "router", "combine", "gather", "dispatch", "fused_block"),
+                   key=lambda k: dur.get(k, 0.0))
     bytes_dom = share * avg(lambda b: kw[b][dominant].bytes)
-    bytes_meth = (share * avg(lambda b: mb[b][dominant]) if dominant in ("gemm1", "gemm2")
-                  else bytes_dom)
+    bytes_meth = (share * avg(lambda b: mb[b][dominant])
+                  if dominant in ("gemm1", "gemm2", "fused_block") else bytes_dom)
     flops_dom = share * avg(lambda b: kw[b][dominant].flops)
     # tensor peak: the sustained (power-capped) figure when the timed loop runs
     # long enough for the clocks to settle under the power cap, else the burst one
@@ -310,8 +322,8 @@ def rooflines(w, blk, K, tm, fp8_act=False, share=1.0):
     tflops = tensor_peak(peaks, sustained, mma)
     dsec = dur[dominant] / 1e3
     kname = {"gemm1": "tc_expert_gemm<1>",
-             "gemm2": "tc_expert_gemm<3>" if blk.combine_mode == "scatter" else "tc_expert_gemm<2>"
-             }.get(dominant, dominant)
+             "gemm2": "tc_expert_gemm<3>" if blk.combine_mode == "scatter" else "tc_expert_gemm<2>",
+             "fused_block": "fused::decode_block"}.get(dominant, dominant)
     if bytes_meth / (hbm * 1e9) >= flops_dom / (tflops * 1e12):
         roof = {"bound": "hbm", "achieved": bytes_meth / dsec / 1e9, "peak": hbm, "unit": "GB/s"}
         roof["frac"] = roof["achieved"] / hbm
@@ -351,24 +363,33 @@ def rooflines(w, blk, K, tm, fp8_act=False, share=1.0):
     return roof, step_roof, touched
 
 
+def kernel_times(blk, tm):
+    """Per-kernel milliseconds; the fused decode launch is one span."""
+    if getattr(blk, "fused_decode", False):
+        return {"fused_block": tm["dur"]["router"]}
+    return tm["dur"]
+
+
 def near_tie_report(w, tm):
     n = tm["near_ties"]
     return {"threshold": 1e-6, "tokens_per_batch": n, "fraction": sum(n) / (len(n) * w.T)}
 
 
-def other_config(name, args, dev, local_rank, fp8_act=False):
+def other_config(name, args, dev, local_rank, variant=""):
     """A short timed loop of another configuration, for the same JSON line."""
     w = WORKLOADS[name]
     xs, params = make_inputs(w, dev, 0)
+    fp8_act = variant == "fp8act"
     blk = moe.MoEBlock(w.shape, params, w.T, w.x_dtype, device=dev, combine=args.combine,
-                       fp8_act=fp8_act)
+                       fp8_act=fp8_act, fused_decode=variant == "fused")
     K = args.other_steps
     tm = time_block(w, blk, xs, K, 3, 1, dev, local_rank)
     roof, step_roof, touched = rooflines(w, blk, K, tm, fp8_act)
     out = {"value": job_tokens_per_s(1, w.T, K, tm["ms_total"]), "unit": "tokens/s",
            "ms_per_step": tm["ms_step"], "steps": K, "warmup": 3, "T": w.T,
            "weights": w.w_format, "mma_type": mma_type(w, fp8_act),
-           "step_roofline": step_roof, "roofline": roof, "kernels_ms": tm["dur"],
+           "step_roofline": step_roof, "roofline": roof, "kernels_ms": kernel_times(blk, tm),
+           "gpu_launches_per_step": blk.launches_per_forward,
            "near_ties": near_tie_report(w, tm), "clocks": tm["clocks"],
            "touched_experts": touched}
     if w.hot_experts:
@@ -396,7 +417,8 @@ def run_ours(args, rank, local_rank, world):
     x0 = xs[0]
     blk = moe.MoEBlock(sh, params, w.T, w.x_dtype, device=dev, combine=args.combine,
                        fp8_act=args.fp8_act, ep=(rank, world) if ep else (0, 1),
-                       ep_group=torch.distributed.group.WORLD if ep else None)
+                       ep_group=torch.distributed.group.WORLD if ep else None,
+                       fused_decode=args.fused_decode)
     K = args.steps
     tm = time_block(w, blk, xs, K, args.warmup, world, dev, local_rank)
     ms_total, ms_step = tm["ms_total"], tm["ms_step"]
@@ -493,12 +515,13 @@ def run_ours(args, rank, local_rank, world):
         del blk, xs, params, x_host, y_host, pipe
         torch.cuda.empty_cache()
         others = {}
-        for name, fp8 in OTHER_CONFIGS:
-            if name == w.name and fp8 == args.fp8_act:
+        main_variant = "fp8act" if args.fp8_act else "fused" if args.fused_decode else ""
+        for name, variant in OTHER_CONFIGS:
+            if name == w.name and variant == main_variant:
                 continue
-            key = name + ("_fp8act" if fp8 else "")
+            key = name + ("_" + variant if variant else "")
             try:
-                others[key] = other_config(name, args, dev, local_rank, fp8)
+                others[key] = other_config(name, args, dev, local_rank, variant)
             except Exception as exc:  # reported, never fatal to the headline
                 others[key] = {"error": repr(exc)[:300]}
 
@@ -521,7 +544,7 @@ def run_ours(args, rank, local_rank, world):
                          f"{(sh.n_routed + 1) * 3 * sh.dim * sh.inter * w_bytes / 1e9:.1f} GB "
                          "of expert weights per step"},
         "roofline": roof, "step_roofline": step_roof,
-        "kernels_ms": tm["dur"], "cpu_baseline": cpu, "e2e": e2e, "graph": graph,
+        "kernels_ms": kernel_times(blk, tm), "cpu_baseline": cpu, "e2e": e2e, "graph": graph,
         "gpu_launches": launches,
         "clocks": tm["clocks"], "touched_experts": touched, "hot_share": hot,
         "near_ties": near_tie_report(w, tm),
