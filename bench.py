@@ -508,6 +508,7 @@ def run_ours(args, rank, local_rank, world):
         hot_ids = torch.randperm(sh.n_routed, generator=torch.Generator().manual_seed(2024))[:16]
         hot = float(tm["counts"][0][hot_ids].sum() / tm["counts"][0].sum())
     launches = K * blk.launches_per_forward
+    kernels_ms = kernel_times(blk, tm)
 
     # the other configurations, each in a short loop of its own (one GPU only)
     others = None
@@ -544,7 +545,7 @@ def run_ours(args, rank, local_rank, world):
                          f"{(sh.n_routed + 1) * 3 * sh.dim * sh.inter * w_bytes / 1e9:.1f} GB "
                          "of expert weights per step"},
         "roofline": roof, "step_roofline": step_roof,
-        "kernels_ms": kernel_times(blk, tm), "cpu_baseline": cpu, "e2e": e2e, "graph": graph,
+        "kernels_ms": kernels_ms, "cpu_baseline": cpu, "e2e": e2e, "graph": graph,
         "gpu_launches": launches,
         "clocks": tm["clocks"], "touched_experts": touched, "hot_share": hot,
         "near_ties": near_tie_report(w, tm),
