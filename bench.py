@@ -22,6 +22,7 @@ import tempfile
 import time
 from datetime import timedelta
 
+import numpy as np
 import torch
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
@@ -49,7 +50,7 @@ def parse():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="v3_prefill_t4096", choices=sorted(WORKLOADS))
-    ap.add_argument("--cpu-sample", type=int, default=8,
+    ap.add_argument("--cpu-sample", type=int, default=32,
                     help="tokens the oracle pushes through the block for cpu_baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-graph", action="store_true",
@@ -151,15 +152,20 @@ class ClockSampler:
 # ---------------------------------------------------------------- oracle leg
 
 
-def cpu_oracle_tokens_per_s(w, x, params, n_tokens: int, seed: int = 7, fp8_act=False):
-    """Time the oracle (as it stands) on a seeded sample of the workload's
-    tokens: routing and the block output of each sampled token.  Host copies
-    of the expert weights are fetched outside the timed part."""
+def cpu_oracle_tokens_per_s(w, x, params, n_tokens: int, seed: int = 7, fp8_act=False,
+                            route_all: bool = False):
+    """Time the oracle (as it stands) on the workload: the routing of every
+    token when route_all (else of the sample only) and the block output of a
+    seeded sample of n_tokens tokens.  Returns (tokens/s, cores, seconds):
+    the per-token cost is the routing time per routed token plus the expert
+    time per sampled token.  Host copies of the expert weights are fetched
+    outside the timed part."""
     from oracle import moe_oracle as O
     from threadpoolctl import threadpool_info
 
     toks = sample_tokens(w.T, n_tokens, seed).numpy()
     xs = x[torch.from_numpy(toks).to(x.device)].float().cpu().numpy()
+    x_all = x.float().cpu().numpy() if route_all else xs
     w_r = params.w_r.cpu().numpy()
     bias = None if params.bias is None else params.bias.cpu().numpy()
     b = w.shape
@@ -185,12 +191,21 @@ def cpu_oracle_tokens_per_s(w, x, params, n_tokens: int, seed: int = 7, fp8_act=
     act = ("f32" if w.x_dtype == torch.float32 else
            ("e4m3" if fp8_act else "f16") if w.w_format == "e4m3" else "bf16")
     t0 = time.perf_counter()
-    route = O.router(xs, w_r, bias, shape)
+    route_all_tok = O.router(x_all, w_r, bias, shape)
+    t_route = time.perf_counter() - t0
+    route = O.RouterResult(*[a[toks] if route_all and a is not None and not np.isscalar(a)
+                             and getattr(a, "shape", (0,))[0] == w.T else a
+                             for a in (route_all_tok.weights, route_all_tok.indices,
+                                       route_all_tok.scores, route_all_tok.biased,
+                                       route_all_tok.group_scores, route_all_tok.kept_groups,
+                                       route_all_tok.gap_set, route_all_tok.gap_order)])
+    t1 = time.perf_counter()
     O.moe_forward(xs, route, fetch, lambda: fetch(shape.n_routed_experts),
                   shape.n_routed_experts, act)
-    wall = time.perf_counter() - t0 - fetch_s
+    t_ffn = time.perf_counter() - t1 - fetch_s
     cores = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
-    return len(toks) / wall, cores, wall
+    per_token = t_route / x_all.shape[0] + t_ffn / len(toks)
+    return 1.0 / per_token, cores, t_route + t_ffn
 
 
 # ---------------------------------------------------------------- ours
@@ -321,8 +336,9 @@ def rooflines(w, blk, K, tm, fp8_act=False, share=1.0):
     hbm = peaks["hbm_gbs"]
     tflops = tensor_peak(peaks, sustained, mma)
     dsec = dur[dominant] / 1e3
-    kname = {"gemm1": "tc_expert_gemm<1>",
-             "gemm2": "tc_expert_gemm<3>" if blk.combine_mode == "scatter" else "tc_expert_gemm<2>",
+    gemm = "tc_fp8_gemm" if fp8_act else "tc_expert_gemm"
+    kname = {"gemm1": f"{gemm}<1>",
+             "gemm2": f"{gemm}<3>" if blk.combine_mode == "scatter" else f"{gemm}<2>",
              "fused_block": "fused::decode_block"}.get(dominant, dominant)
     if bytes_meth / (hbm * 1e9) >= flops_dom / (tflops * 1e12):
         roof = {"bound": "hbm", "achieved": bytes_meth / dsec / 1e9, "peak": hbm, "unit": "GB/s"}
@@ -495,11 +511,12 @@ def run_ours(args, rank, local_rank, world):
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         try:
             tps, cores, wall = cpu_oracle_tokens_per_s(w, x0, params, args.cpu_sample,
-                                                       fp8_act=args.fp8_act)
+                                                       fp8_act=args.fp8_act, route_all=True)
             cpu = {"value": tps, "unit": "tokens/s", "cores": cores, "kind": "oracle",
-                   "sample": f"{args.cpu_sample} seeded tokens of the {w.name} batch: fp64 "
-                             f"routing and block output ({wall:.1f} s of oracle time; weight "
-                             "copies to the host excluded)"}
+                   "sample": f"routing of all {w.T} tokens of the {w.name} batch and the block "
+                             f"output of {args.cpu_sample} seeded tokens, fp64 ({wall:.1f} s of "
+                             "oracle time; weight copies to the host excluded); tokens/s = 1 / "
+                             "(routing time per token + expert time per sampled token)"}
         except Exception as exc:  # reported, never fatal
             cpu = {"value": None, "error": repr(exc)[:200]}
 
