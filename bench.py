@@ -31,7 +31,7 @@ sys.path.insert(0, ROOT)
 from sparse_moe_layer_sum_b200 import moe  # noqa: E402
 from sparse_moe_layer_sum_b200.inputs import WORKLOADS, make_block, sample_tokens  # noqa: E402
 from sparse_moe_layer_sum_b200.roofline import (block_work, kernel_work, load_peaks,  # noqa: E402
-                                                 method_bytes, tensor_peak)
+                                                 method_bytes, tensor_peak, use_sustained_peak)
 
 METRIC = "MoE block tokens/s (V3 shape, bf16, T=4096) and % of roofline on 1 B200"
 N_X_BATCHES = 4  # rotating input batches: with the 22.6 GB of weights, > L2 per step
@@ -330,8 +330,9 @@ def rooflines(w, blk, K, tm, fp8_act=False, share=1.0):
                   if dominant in ("gemm1", "gemm2", "fused_block") else bytes_dom)
     flops_dom = share * avg(lambda b: kw[b][dominant].flops)
     # tensor peak: the sustained (power-capped) figure when the timed loop runs
-    # long enough for the clocks to settle under the power cap, else the burst one
-    sustained = tm["ms_total"] > 500.0 and "bf16_tflops_sustained" in peaks
+    # long enough for the clocks to settle under the power cap, or when the
+    # clock samples show the power cap engaged during it; else the burst one
+    sustained, capped = use_sustained_peak(peaks, tm["ms_total"], tm.get("clocks"))
     mma = mma_type(w, fp8_act)
     hbm = peaks["hbm_gbs"]
     tflops = tensor_peak(peaks, sustained, mma)
@@ -354,7 +355,7 @@ def rooflines(w, blk, K, tm, fp8_act=False, share=1.0):
     roof["scope"] = "dominant kernel (the whole step is step_roofline)"
     roof["mma_type"] = mma
     roof["peak_source"] = (f"{peak_src} ({'MEASURED_PEAKS.json' if peak_src == 'measured' else 'recipe fallback'}"
-                           f"{', tensor peak sustained' if sustained else ', tensor peak burst'}"
+                           f"{(', tensor peak sustained' + (' (power cap seen)' if capped else '')) if sustained else ', tensor peak burst'}"
                            f"{', e4m3 = 2 x bf16 (nominal ratio)' if mma == 'e4m3' else ''})")
     roof["method_bytes_per_launch"] = bytes_meth
     roof["impl_bytes_per_launch"] = bytes_dom
@@ -370,6 +371,14 @@ def rooflines(w, blk, K, tm, fp8_act=False, share=1.0):
                  "hbm_frac": b_alg / (ms_step / 1e3) / (hbm * 1e9),
                  "tensor_frac": f_alg / (ms_step / 1e3) / (tflops * 1e12),
                  "hbm_frac_vs_nominal_8TBs": b_alg / (ms_step / 1e3) / 8e12}
+    if "bf16_tflops_sustained" in peaks:
+        # the tensor fraction against both peaks, whichever one heads the line
+        for tag, sus in (("burst", False), ("sustained", True)):
+            tp = tensor_peak(peaks, sus, mma)
+            step_roof[f"tensor_frac_{tag}"] = f_alg / (ms_step / 1e3) / (tp * 1e12)
+            step_roof[f"frac_{tag}"] = max(b_alg / (hbm * 1e9), f_alg / (tp * 1e12)) / (ms_step / 1e3)
+            if roof["bound"] == "tensor":
+                roof[f"frac_{tag}"] = flops_dom / dsec / 1e12 / tp
     if w.w_format == "e4m3" and mma != "e4m3":
         # the same step against the dense FP8 peak (2 x bf16), which an
         # FP8 x FP8 matmul could reach

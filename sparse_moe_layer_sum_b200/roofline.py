@@ -51,6 +51,16 @@ def tensor_peak(peaks: dict, sustained: bool, mma: str) -> float:
     return {"bf16": 1.0, "f16": 1.0, "e4m3": 2.0, "f32": 1.0}[mma] * bf16
 
 
+def use_sustained_peak(peaks: dict, ms_timed: float, clocks: dict | None) -> tuple[bool, bool]:
+    """Which bf16 tensor peak heads a line: the sustained (power-capped) one
+    when the timed loop lasts over half a second, long enough for the clocks
+    to settle under the power cap, or when the clock samples taken during it
+    show the power cap engaged; else the burst one.  Returns (sustained,
+    power cap seen)."""
+    capped = "sw_power_cap" in ((clocks or {}).get("reasons") or [])
+    return (ms_timed > 500.0 or capped) and "bf16_tflops_sustained" in peaks, capped
+
+
 def method_bytes(D, I, k, S, T, n_touched, w_bytes, x_bytes, scale_bytes_per_expert=0.0):
     """Bytes of each matmul that the method itself fixes, with no
     implementation buffers: the weights of the touched experts and the

@@ -9,7 +9,7 @@ bias), so a dropped term or a wrong factor shows up against these sums.
 import pytest
 
 from sparse_moe_layer_sum_b200.roofline import (block_work, kernel_work, load_peaks,
-                                                 method_bytes, tensor_peak)
+                                                 method_bytes, tensor_peak, use_sustained_peak)
 
 D, E, I, K, S = 7168, 256, 2048, 8, 1
 PER_EXPERT = 44_040_192  # parameters of one expert, as the page counts them
@@ -89,3 +89,17 @@ def test_tensor_peak_by_operand_type():
     assert tensor_peak(p, False, "bf16") == 1600.0
     assert tensor_peak(p, True, "f16") == 1400.0
     assert tensor_peak(p, False, "e4m3") == 3200.0
+
+
+def test_peak_choice_follows_loop_length_and_power_cap():
+    p = {"bf16_tflops": 1600.0, "bf16_tflops_sustained": 1400.0}
+    # a short loop at full clocks: burst
+    assert use_sustained_peak(p, 100.0, {"reasons": []}) == (False, False)
+    assert use_sustained_peak(p, 100.0, None) == (False, False)
+    # a long loop: sustained, with or without a clock record
+    assert use_sustained_peak(p, 1000.0, None) == (True, False)
+    # a short loop that the clock samples show under the power cap: sustained
+    assert use_sustained_peak(p, 100.0, {"reasons": ["sw_power_cap"]}) == (True, True)
+    # no sustained figure on record: burst, whatever the loop
+    assert use_sustained_peak({"bf16_tflops": 1600.0}, 1000.0,
+                              {"reasons": ["sw_power_cap"]}) == (False, True)
