@@ -296,9 +296,13 @@ struct Layout {
   static constexpr int MISC_OFF = BAR_OFF + NBARS * 8;
   static constexpr int MISC_BYTES = 16 + 8 * STAGES;
   static constexpr int XBUF_OFF = (MISC_OFF + MISC_BYTES + 127) / 128 * 128;
-  // GEMM1 with AT = 1: SwiGLU exchange buffers; MODE 3: the tile's (token, gate) list
+  // an epilogue warp's token columns are chunks of 32, CSTEP apart: NCH chunks
+  static constexpr int CSTEP = 32 * (EPI / 4);
+  static constexpr int NCH = (BN_MAX + CSTEP - 1) / CSTEP;
+  // GEMM1 with AT = 1: SwiGLU exchange buffers; MODE 3: each epilogue warp's
+  // (token, gate) list of its columns
   static constexpr int XBUF_BYTES =
-      MODE == 1 ? (AT == 1 ? 2 * 2 * 32 * XB_STRIDE * 4 : 0) : MODE == 3 ? BN_MAX * 8 : 0;
+      MODE == 1 ? (AT == 1 ? 2 * 2 * 32 * XB_STRIDE * 4 : 0) : MODE == 3 ? EPI * NCH * 32 * 8 : 0;
   static constexpr int TAB_OFF = XBUF_OFF + XBUF_BYTES;
   // TMEM: AT accumulators of BN_MAX columns per tile, double-buffered when
   // two tiles' worth fits in the 512 columns
@@ -687,12 +691,38 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap &tmA0, const CUtenso
     // with eight epilogue warps, the two warps of a lane quarter take
     // alternate 32-column chunks
     const int half = (warp - 2) >> 2;
-    constexpr int CSTEP = 32 * (L::EPI / 4);
+    constexpr int CSTEP = L::CSTEP;
     const float acc_scale = F8 ? F8_SCALE_DOWN : 1.0f;
     int acc = 0;
     uint32_t acc_phase = 0;
+    // MODE 3: this warp's token and gate for each of its columns (chunk i,
+    // lane j: column half * 32 + i * CSTEP + j), private to the warp
+    int32_t *s_tok = reinterpret_cast<int32_t *>(xbuf) + (warp - 2) * L::NCH * 64;
+    float *s_gate = reinterpret_cast<float *>(s_tok + L::NCH * 32);
     for (int tile = unit; tile < total; tile += nunits) {
       const Tile t = decode_tile(tile, s_tstart, s_tbase, s_off, p.G, p.E, p.T, p.rows_routed, p.sh);
+      if (MODE == 3) {
+        // the list for the scatter into y (gate 1 for the shared expert),
+        // built while the tile's MMAs still run
+        __syncwarp();  // this warp is done with the previous tile's list
+        for (int i = 0; i < L::NCH; ++i) {
+          const int c = half * 32 + i * CSTEP + lane;
+          if (c < t.nvalid) {
+            int tok;
+            float gate = 1.0f;
+            if (t.g < p.E) {
+              tok = p.sorted_token[t.rowbase + t.n0 + c];
+              for (int jj = 0; jj < p.k; ++jj)
+                if (p.indices[(size_t)tok * p.k + jj] == t.g) gate = p.weights[(size_t)tok * p.k + jj];
+            } else {
+              tok = t.tok0 + c;
+            }
+            s_tok[i * 32 + lane] = tok;
+            s_gate[i * 32 + lane] = gate;
+          }
+        }
+        __syncwarp();
+      }
       if (!wait_bounded(accf + acc, acc_phase, abort_flag, p.timeout_ns, p.status)) break;
       tc_fence_after();
       const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * L::ACC_COLS);
@@ -709,64 +739,64 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap &tmA0, const CUtenso
         }
         released = true;
       };
-      if (MODE == 3) {
-        // weighted scatter into y: y[t, d] += gate(t) * o[t, d] (gate 1 for the
-        // shared expert), with fp32 reductions; first the tile's token list
-        int32_t *s_tok = reinterpret_cast<int32_t *>(xbuf);
-        float *s_gate = reinterpret_cast<float *>(s_tok + BN_MAX);
-        const int et = threadIdx.x - 64;  // over all epilogue warps
-        named_bar_sync(3, 32 * L::EPI);    // the previous tile's readers are done
-        for (int c = et; c < t.nvalid; c += 32 * L::EPI) {
-          int tok;
-          float gate = 1.0f;
-          if (t.g < p.E) {
-            tok = p.sorted_token[t.rowbase + t.n0 + c];
-            for (int jj = 0; jj < p.k; ++jj)
-              if (p.indices[(size_t)tok * p.k + jj] == t.g) gate = p.weights[(size_t)tok * p.k + jj];
-          } else {
-            tok = t.tok0 + c;
-          }
-          s_tok[c] = tok;
-          s_gate[c] = gate;
-        }
-        named_bar_sync(3, 32 * L::EPI);
-#pragma unroll
-        for (int a = 0; a < AT; ++a) {
-          const int d = t.ft * L::FEAT + a * BM * CG + (int)rank * BM + q * 32 + lane;
-          for (int c0 = half * 32; c0 < t.nvalid; c0 += CSTEP) {
-            uint32_t v[32];
-            tmem_ld_32x32b_x32(tb + (uint32_t)(a * BN_MAX + c0), v);
-            tmem_wait_ld();
-#pragma unroll
-            for (int j = 0; j < 32; ++j)
-              if (c0 + j < t.nvalid)
-                atomicAdd(p.y + (size_t)s_tok[c0 + j] * p.D + d,
-                          s_gate[c0 + j] * (__uint_as_float(v[j]) * acc_scale));
-          }
-        }
-      } else if (MODE == 2) {
-        // lanes are output features d, columns are tokens
-        float *out;
-        size_t row0;
-        if (t.g < p.E) {
+      if (MODE == 2 || MODE == 3) {
+        // lanes are output features d, columns are tokens; MODE 3 adds
+        // gate * o into y with fp32 reductions, MODE 2 writes per-slot rows
+        float *out = nullptr;
+        size_t row0 = 0;
+        if (MODE == 2 && t.g < p.E) {
           out = static_cast<float *>(p.out);
           row0 = (size_t)t.rowbase + t.n0;
-        } else {
+        } else if (MODE == 2) {
           out = p.out_shared;
           row0 = (size_t)(t.g - p.E) * p.T + t.tok0;
         }
-#pragma unroll
-        for (int a = 0; a < AT; ++a) {
+        // the 32 columns from c0 of accumulator a, read into v
+        auto store = [&](int a, int c0, const uint32_t *v) {
           const int d = t.ft * L::FEAT + a * BM * CG + (int)rank * BM + q * 32 + lane;
-          for (int c0 = half * 32; c0 < t.nvalid; c0 += CSTEP) {
-            uint32_t v[32];
-            tmem_ld_32x32b_x32(tb + (uint32_t)(a * BN_MAX + c0), v);
-            tmem_wait_ld();
+          const int li = (c0 - half * 32) / CSTEP * 32;  // the chunk's place in the list
 #pragma unroll
-            for (int j = 0; j < 32; ++j)
-              if (c0 + j < t.nvalid)
-                out[(row0 + c0 + j) * p.D + d] = __uint_as_float(v[j]) * acc_scale;
+          for (int j = 0; j < 32; ++j) {
+            if (c0 + j < t.nvalid) {
+              const float o = __uint_as_float(v[j]) * acc_scale;
+              if (MODE == 3)
+                atomicAdd(p.y + (size_t)s_tok[li + j] * p.D + d, s_gate[li + j] * o);
+              else
+                out[(row0 + c0 + j) * p.D + d] = o;
+            }
           }
+        };
+        if (L::NBUF == 1) {
+          // single-buffered accumulator: this warp's chunks are read in
+          // batches of up to NB (32 registers each) and the accumulator goes
+          // back to the MMA right after the last batch's reads, so that the
+          // stores of that batch overlap the next tile's MMAs
+          constexpr int NB = F8 ? 2 : 4;  // the converter warps leave fewer registers
+          const int nch = t.nvalid > half * 32 ? (t.nvalid - half * 32 + CSTEP - 1) / CSTEP : 0;
+          const int nall = AT * nch;
+          for (int b0 = 0; b0 < nall; b0 += NB) {
+            uint32_t v[NB][32];
+#pragma unroll
+            for (int u = 0; u < NB; ++u)
+              if (b0 + u < nall) {
+                const int a = (b0 + u) / nch, c0 = half * 32 + ((b0 + u) % nch) * CSTEP;
+                tmem_ld_32x32b_x32(tb + (uint32_t)(a * BN_MAX + c0), v[u]);
+              }
+            tmem_wait_ld();
+            if (b0 + NB >= nall) release();
+#pragma unroll
+            for (int u = 0; u < NB; ++u)
+              if (b0 + u < nall) store((b0 + u) / nch, half * 32 + ((b0 + u) % nch) * CSTEP, v[u]);
+          }
+        } else {
+#pragma unroll
+          for (int a = 0; a < AT; ++a)
+            for (int c0 = half * 32; c0 < t.nvalid; c0 += CSTEP) {
+              uint32_t v[32];
+              tmem_ld_32x32b_x32(tb + (uint32_t)(a * BN_MAX + c0), v);
+              tmem_wait_ld();
+              store(a, c0, v);
+            }
         }
       } else if (AT == 2) {
         // lanes are features; the w1.x accumulator (a) and the w3.x one (u)
@@ -2157,13 +2187,18 @@ moe_status simt_down_w(const Job &j) {
 #define MOE_TC_PREFILL_BN 256
 #endif
 // weight tiles per SM in the first matmul (two: w1 and w3 in accumulators of
-// their own, half the token bytes per weight byte) and in the second (one:
-// its K loop is short, and double-buffered accumulators hide the epilogue)
+// their own, half the token bytes per weight byte) and in the second (two
+// blocks of w2 rows with bf16 weights, for the same reason, their single
+// accumulator handed back before the last stores of each tile; one with e4m3
+// weights, where two measured no faster)
 #ifndef MOE_TC_PREFILL_AT_UP
 #define MOE_TC_PREFILL_AT_UP 2
 #endif
 #ifndef MOE_TC_PREFILL_AT_DOWN
-#define MOE_TC_PREFILL_AT_DOWN 1
+#define MOE_TC_PREFILL_AT_DOWN 2
+#endif
+#ifndef MOE_TC_PREFILL_AT_DOWN_F8
+#define MOE_TC_PREFILL_AT_DOWN_F8 1
 #endif
 #ifndef MOE_TC_PREFILL_CG
 #define MOE_TC_PREFILL_CG 2
@@ -2175,7 +2210,8 @@ moe_status simt_down_w(const Job &j) {
 #define MOE_TC_DECODE_STAGES 10
 #endif
 constexpr int PF_BN = MOE_TC_PREFILL_BN;
-constexpr int PF_AT_UP = MOE_TC_PREFILL_AT_UP, PF_AT_DOWN = MOE_TC_PREFILL_AT_DOWN;
+constexpr int PF_AT_UP = MOE_TC_PREFILL_AT_UP;
+constexpr int pf_at_down(bool f8) { return f8 ? MOE_TC_PREFILL_AT_DOWN_F8 : MOE_TC_PREFILL_AT_DOWN; }
 // ring depth filling about 200 KB of shared memory: a stage holds AT 16 KB
 // weight tiles, PF_BN / 2 token rows of 128 bytes and, with e4m3 weights, AT
 // 8 KB code tiles
@@ -2188,11 +2224,11 @@ constexpr int DC_BN = MOE_TC_DECODE_BN, DC_ST = MOE_TC_DECODE_STAGES;
 bool decode_variant(const Job &j) { return j.T * j.c->topk <= (int64_t)16 * j.c->n_routed; }
 
 // an SM pair per tile (cta_group::2) covers 64 * 2 * PF_AT_UP features of
-// w1/w3 and 256 * PF_AT_DOWN rows of w2
-bool pair_ok(const Job &j) {
-  return MOE_TC_PREFILL_CG == 2 && j.c->inter % (128 * PF_AT_UP) == 0 &&
-         j.c->dim % (256 * PF_AT_DOWN) == 0;
+// w1/w3, and 256 rows of w2 per weight tile
+bool pair_up_ok(const Job &j) {
+  return MOE_TC_PREFILL_CG == 2 && j.c->inter % (128 * PF_AT_UP) == 0;
 }
+bool pair_down_ok(const Job &j, int at) { return MOE_TC_PREFILL_CG == 2 && j.c->dim % (256 * at) == 0; }
 
 // e4m3 weights add 8 KB of codes per weight tile and stage; the ring depths
 // shrink to fit shared memory, and half as many weight bytes need to be in
@@ -2200,14 +2236,16 @@ bool pair_ok(const Job &j) {
 template <bool F8>
 moe_status run_up_t(const Job &j) {
   if (decode_variant(j)) return tc_up<1, 1, DC_BN, 32, F8 ? 7 : DC_ST, F8>(j);
-  if (pair_ok(j)) return tc_up<2, PF_AT_UP, PF_BN, 32, pf_stages(PF_AT_UP, F8), F8>(j);
+  if (pair_up_ok(j)) return tc_up<2, PF_AT_UP, PF_BN, 32, pf_stages(PF_AT_UP, F8), F8>(j);
   return tc_up<1, 1, 256, 32, F8 ? 3 : 4, F8>(j);
 }
 
 template <bool F8>
 moe_status run_down_t(const Job &j) {
   if (decode_variant(j)) return tc_down<1, 1, DC_BN, 32, F8 ? 7 : DC_ST, F8>(j);
-  if (pair_ok(j)) return tc_down<2, PF_AT_DOWN, PF_BN, 32, pf_stages(PF_AT_DOWN, F8), F8>(j);
+  constexpr int AT = pf_at_down(F8);
+  if (pair_down_ok(j, AT)) return tc_down<2, AT, PF_BN, 32, pf_stages(AT, F8), F8>(j);
+  if (AT != 1 && pair_down_ok(j, 1)) return tc_down<2, 1, PF_BN, 32, pf_stages(1, F8), F8>(j);
   return tc_down<1, 1, 256, 32, F8 ? 3 : 4, F8>(j);
 }
 
