@@ -291,18 +291,18 @@ struct Layout {
   static constexpr int NPARTS = MODE == 1 ? 2 : AT;
   static constexpr int PART_ROWS = MODE == 1 && AT == 1 ? 64 : BM;
   static constexpr int BAR_OFF = STAGES * STAGE_BYTES;
-  // full, empty, [a8_full, converted], acc_full x2, acc_empty x2, drain
-  static constexpr int NBARS = (F8 ? 4 : 2) * STAGES + 5;
+  // full, empty, [a8_full, converted], acc_full x2, acc_empty x2, drain,
+  // list_full x2, list_empty x2
+  static constexpr int NBARS = (F8 ? 4 : 2) * STAGES + 9;
   static constexpr int MISC_OFF = BAR_OFF + NBARS * 8;
   static constexpr int MISC_BYTES = 16 + 8 * STAGES;
   static constexpr int XBUF_OFF = (MISC_OFF + MISC_BYTES + 127) / 128 * 128;
-  // an epilogue warp's token columns are chunks of 32, CSTEP apart: NCH chunks
+  // an epilogue warp's token columns are chunks of 32, CSTEP apart
   static constexpr int CSTEP = 32 * (EPI / 4);
-  static constexpr int NCH = (BN_MAX + CSTEP - 1) / CSTEP;
-  // GEMM1 with AT = 1: SwiGLU exchange buffers; MODE 3: each epilogue warp's
-  // (token, gate) list of its columns
+  // GEMM1 with AT = 1: SwiGLU exchange buffers; MODE 3: two (token, gate)
+  // lists of a tile's columns, used by alternate tiles
   static constexpr int XBUF_BYTES =
-      MODE == 1 ? (AT == 1 ? 2 * 2 * 32 * XB_STRIDE * 4 : 0) : MODE == 3 ? EPI * NCH * 32 * 8 : 0;
+      MODE == 1 ? (AT == 1 ? 2 * 2 * 32 * XB_STRIDE * 4 : 0) : MODE == 3 ? 2 * BN_MAX * 8 : 0;
   static constexpr int TAB_OFF = XBUF_OFF + XBUF_BYTES;
   // TMEM: AT accumulators of BN_MAX columns per tile, double-buffered when
   // two tiles' worth fits in the 512 columns
@@ -381,6 +381,8 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap &tmA0, const CUtenso
   uint64_t *accf = conv + (F8 ? STAGES : 0);
   uint64_t *acce = accf + 2;
   uint64_t *drain = acce + 2;
+  uint64_t *lfull = drain + 1;   // MODE 3: a tile's token list written
+  uint64_t *lempty = lfull + 2;  // MODE 3: a tile's token list read
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + L::MISC_OFF);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + L::MISC_OFF + 4);
   volatile int *pending = reinterpret_cast<volatile int *>(sm + L::MISC_OFF + 16);
@@ -413,6 +415,10 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap &tmA0, const CUtenso
     mbar_init(acce + 0, L::EPI * CG);
     mbar_init(acce + 1, L::EPI * CG);
     mbar_init(drain, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(lfull + b, L::EPI);
+      mbar_init(lempty + b, L::EPI);
+    }
     *abort_flag = 0;
     fence_mbar_init();
     tma_prefetch_desc(&tmA0);
@@ -695,33 +701,48 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap &tmA0, const CUtenso
     const float acc_scale = F8 ? F8_SCALE_DOWN : 1.0f;
     int acc = 0;
     uint32_t acc_phase = 0;
-    // MODE 3: this warp's token and gate for each of its columns (chunk i,
-    // lane j: column half * 32 + i * CSTEP + j), private to the warp
-    int32_t *s_tok = reinterpret_cast<int32_t *>(xbuf) + (warp - 2) * L::NCH * 64;
-    float *s_gate = reinterpret_cast<float *>(s_tok + L::NCH * 32);
-    for (int tile = unit; tile < total; tile += nunits) {
+    // MODE 3: the tile's token and gate of each column (gate 1 for the shared
+    // expert), in one of two lists that alternate between tiles; every
+    // epilogue warp writes a share of it before waiting for the accumulator
+    // and reads all of it in the stores
+    int32_t *s_tok = nullptr;
+    float *s_gate = nullptr;
+    int ntile = 0;
+    for (int tile = unit; tile < total; tile += nunits, ++ntile) {
       const Tile t = decode_tile(tile, s_tstart, s_tbase, s_off, p.G, p.E, p.T, p.rows_routed, p.sh);
       if (MODE == 3) {
-        // the list for the scatter into y (gate 1 for the shared expert),
-        // built while the tile's MMAs still run
-        __syncwarp();  // this warp is done with the previous tile's list
-        for (int i = 0; i < L::NCH; ++i) {
-          const int c = half * 32 + i * CSTEP + lane;
-          if (c < t.nvalid) {
-            int tok;
-            float gate = 1.0f;
-            if (t.g < p.E) {
-              tok = p.sorted_token[t.rowbase + t.n0 + c];
-              for (int jj = 0; jj < p.k; ++jj)
-                if (p.indices[(size_t)tok * p.k + jj] == t.g) gate = p.weights[(size_t)tok * p.k + jj];
-            } else {
-              tok = t.tok0 + c;
-            }
-            s_tok[i * 32 + lane] = tok;
-            s_gate[i * 32 + lane] = gate;
+        const int lb = ntile & 1;
+        const uint32_t lph = (uint32_t)(ntile >> 1) & 1u;
+        s_tok = reinterpret_cast<int32_t *>(xbuf) + lb * 2 * BN_MAX;
+        s_gate = reinterpret_cast<float *>(s_tok + BN_MAX);
+        // the list's previous tile has been read by every epilogue warp
+        if (!wait_bounded(lempty + lb, lph ^ 1u, abort_flag, p.timeout_ns, p.status)) break;
+        // this warp's columns, all loads issued together
+        constexpr int PER = (BN_MAX + 32 * L::EPI - 1) / (32 * L::EPI);
+        int tok[PER], pos[PER];
+#pragma unroll
+        for (int i = 0; i < PER; ++i) {
+          const int c = ((warp - 2) + i * L::EPI) * 32 + lane;
+          tok[i] = c >= t.nvalid ? -1 : t.g < p.E ? p.sorted_token[t.rowbase + t.n0 + c] : t.tok0 + c;
+          pos[i] = -1;
+        }
+        if (t.g < p.E) {
+          for (int jj = 0; jj < p.k; ++jj)
+#pragma unroll
+            for (int i = 0; i < PER; ++i)
+              if (tok[i] >= 0 && p.indices[(size_t)tok[i] * p.k + jj] == t.g) pos[i] = jj;
+        }
+#pragma unroll
+        for (int i = 0; i < PER; ++i) {
+          const int c = ((warp - 2) + i * L::EPI) * 32 + lane;
+          if (tok[i] >= 0) {
+            s_tok[c] = tok[i];
+            s_gate[c] = pos[i] >= 0 ? p.weights[(size_t)tok[i] * p.k + pos[i]] : 1.0f;
           }
         }
         __syncwarp();
+        if (lane == 0) mbar_arrive(lfull + lb);
+        if (!wait_bounded(lfull + lb, lph, abort_flag, p.timeout_ns, p.status)) break;
       }
       if (!wait_bounded(accf + acc, acc_phase, abort_flag, p.timeout_ns, p.status)) break;
       tc_fence_after();
@@ -754,13 +775,12 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap &tmA0, const CUtenso
         // the 32 columns from c0 of accumulator a, read into v
         auto store = [&](int a, int c0, const uint32_t *v) {
           const int d = t.ft * L::FEAT + a * BM * CG + (int)rank * BM + q * 32 + lane;
-          const int li = (c0 - half * 32) / CSTEP * 32;  // the chunk's place in the list
 #pragma unroll
           for (int j = 0; j < 32; ++j) {
             if (c0 + j < t.nvalid) {
               const float o = __uint_as_float(v[j]) * acc_scale;
               if (MODE == 3)
-                atomicAdd(p.y + (size_t)s_tok[li + j] * p.D + d, s_gate[li + j] * o);
+                atomicAdd(p.y + (size_t)s_tok[c0 + j] * p.D + d, s_gate[c0 + j] * o);
               else
                 out[(row0 + c0 + j) * p.D + d] = o;
             }
@@ -861,6 +881,10 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap &tmA0, const CUtenso
         }
       }
       if (!released) release();
+      if (MODE == 3) {
+        __syncwarp();  // this warp's reads of the list are done
+        if (lane == 0) mbar_arrive(lempty + (ntile & 1));
+      }
       if (++acc == L::NBUF) {
         acc = 0;
         acc_phase ^= 1u;

@@ -329,10 +329,27 @@ TcPlan plan_tc(const moe_cfg *c, int64_t T) {
   p.mt = c->n_routed / tcr::BM;
   p.nt = (int)((T + TC_BN - 1) / TC_BN);
   const int tiles = p.mt * p.nt;
-  int ns = (148 + tiles - 1) / tiles;  // fill the SMs of a B200 at small T
-  ns = ns < 1 ? 1 : (ns > p.KB ? p.KB : ns);
-  p.kb_per_split = (p.KB + ns - 1) / ns;
-  p.nsplit = (p.KB + p.kb_per_split - 1) / p.kb_per_split;
+  // splits of dim: the count with the least estimated time on the B200's
+  // 148 SMs -- waves of tiles times k-blocks per tile at about 1 us each
+  // (64 KB of operands per k-block and SM), plus writing and reading back
+  // each split's fp32 partial sums at about 6.5 TB/s; ties go to fewer
+  // splits
+  constexpr int SMS = 148;
+  int best = 1;
+  int64_t best_cost = INT64_MAX;
+  for (int ns = 1; ns <= p.KB; ++ns) {
+    const int kbps = (p.KB + ns - 1) / ns;
+    const int n = (p.KB + kbps - 1) / kbps;
+    if (n != ns) continue;  // the same split as a smaller count
+    const int64_t waves = ((int64_t)tiles * n + SMS - 1) / SMS;
+    const int64_t cost = waves * kbps * 1000 + (int64_t)n * T * c->n_routed * 8 / 6500;
+    if (cost < best_cost) {
+      best_cost = cost;
+      best = n;
+    }
+  }
+  p.kb_per_split = (p.KB + best - 1) / best;
+  p.nsplit = best;
   return p;
 }
 
