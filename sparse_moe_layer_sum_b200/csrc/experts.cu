@@ -1040,21 +1040,22 @@ constexpr int XB_STRIDE = 17;
 template <int MODE, int STAGES>
 struct Layout {
   static constexpr int BAR_OFF = STAGES * STAGE_BYTES;
-  // full, empty per stage; partial full, partial empty per buffer; drain
-  static constexpr int NBARS = 2 * STAGES + 2 * NPBUF + 1;
+  // full, empty per stage; partial full, partial empty per buffer; drain;
+  // list full, list empty per token list
+  static constexpr int NBARS = 2 * STAGES + 2 * NPBUF + 1 + 4;
   static constexpr int MISC_OFF = BAR_OFF + NBARS * 8;
   static constexpr int MISC_BYTES = 16 + 4 * STAGES;  // TMEM slot, abort flag, pending loads
   static constexpr int SC_OFF = (MISC_OFF + MISC_BYTES + 127) / 128 * 128;
   static constexpr int SC_BYTES = EPI * CHUNKS * 32 * 4;  // the tile's token scales, per warp
   static constexpr int XBUF_OFF = SC_OFF + SC_BYTES;
-  // SwiGLU exchange of the four warp pairs (first matmul), or the tile's
-  // (token, gate) list (second matmul with the scatter)
+  // SwiGLU exchange of the four warp pairs (first matmul), or two (token,
+  // gate) lists used by alternate tiles (second matmul with the scatter)
   static constexpr int XBUF_BYTES = 4 * 2 * 32 * XB_STRIDE * 4;
   static constexpr int TAB_OFF = XBUF_OFF + XBUF_BYTES;
   static size_t smem_bytes(int G, int E) {
     return 1024 + TAB_OFF + sizeof(int32_t) * (size_t)((G + 1) + G + (E + 1));
   }
-  static_assert(BN_MAX * 8 <= XBUF_BYTES, "token list");
+  static_assert(2 * BN_MAX * 8 <= XBUF_BYTES, "token lists");
   static_assert(NPBUF * BN_MAX <= 512, "TMEM columns");
 };
 
@@ -1077,6 +1078,8 @@ __global__ void __launch_bounds__(NT, 1)
   uint64_t *pfull = empty + STAGES;
   uint64_t *pempty = pfull + NPBUF;
   uint64_t *drain = pempty + NPBUF;
+  uint64_t *lfull = drain + 1;   // MODE 3: a tile's token list written
+  uint64_t *lempty = lfull + 2;  // MODE 3: a tile's token list read
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + L::MISC_OFF);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + L::MISC_OFF + 4);
   volatile int *pending = reinterpret_cast<volatile int *>(sm + L::MISC_OFF + 16);
@@ -1104,6 +1107,10 @@ __global__ void __launch_bounds__(NT, 1)
       mbar_init(pempty + b, EPI * 2);
     }
     mbar_init(drain, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(lfull + b, 2);      // the two list-builder warps
+      mbar_init(lempty + b, EPI);   // the epilogue warps
+    }
     *abort_flag = 0;
     fence_mbar_init();
     tma_prefetch_desc(&tmA0);
@@ -1216,6 +1223,46 @@ __global__ void __launch_bounds__(NT, 1)
         mma_commit_pair(drain);
         drain_wait(drain, 0, p.timeout_ns);
       }
+    } else if (MODE == 3 && warp >= 2) {
+      // ------------------------------------------------ token-list builders
+      // the (token, gate) list of each tile for the scatter into y (gate 1
+      // for the shared expert), written ahead of the tile's end into one of
+      // two lists that alternate between tiles
+      const int bt = threadIdx.x - 64;  // 0 .. 63
+      int ntile = 0;
+      for (int tile = unit; tile < total; tile += nunits, ++ntile) {
+        const Tile t = decode_tile(tile, s_tstart, s_tbase, s_off, p.G, p.E, p.T, p.rows_routed, p.sh);
+        const int lb = ntile & 1;
+        const uint32_t lph = (uint32_t)(ntile >> 1) & 1u;
+        int32_t *s_tok = reinterpret_cast<int32_t *>(xbuf) + lb * 2 * BN_MAX;
+        float *s_gate = reinterpret_cast<float *>(s_tok + BN_MAX);
+        // every epilogue warp is done with this list's previous tile
+        if (!wait_bounded(lempty + lb, lph ^ 1u, abort_flag, p.timeout_ns, p.status)) break;
+        constexpr int PER = BN_MAX / 64;
+        int tok[PER], pos[PER];
+#pragma unroll
+        for (int i = 0; i < PER; ++i) {
+          const int c = bt + 64 * i;
+          tok[i] = c >= t.nvalid ? -1 : t.g < p.E ? p.sorted_token[t.rowbase + t.n0 + c] : t.tok0 + c;
+          pos[i] = -1;
+        }
+        if (t.g < p.E) {
+          for (int jj = 0; jj < p.k; ++jj)
+#pragma unroll
+            for (int i = 0; i < PER; ++i)
+              if (tok[i] >= 0 && p.indices[(size_t)tok[i] * p.k + jj] == t.g) pos[i] = jj;
+        }
+#pragma unroll
+        for (int i = 0; i < PER; ++i) {
+          const int c = bt + 64 * i;
+          if (tok[i] >= 0) {
+            s_tok[c] = tok[i];
+            s_gate[c] = pos[i] >= 0 ? p.weights[(size_t)tok[i] * p.k + pos[i]] : 1.0f;
+          }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(lfull + lb);
+      }
     }
   } else {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(REG_HIGH));
@@ -1227,7 +1274,8 @@ __global__ void __launch_bounds__(NT, 1)
     int pb = 0;
     uint32_t pphase = 0;
     bool ok = true;
-    for (int tile = unit; ok && tile < total; tile += nunits) {
+    int ntile = 0;
+    for (int tile = unit; ok && tile < total; tile += nunits, ++ntile) {
       const Tile t = decode_tile(tile, s_tstart, s_tbase, s_off, p.G, p.E, p.T, p.rows_routed, p.sh);
       const int row0 = t.rowbase + t.n0;
       // weight scales of this CTA's rows, one per k-block
@@ -1236,34 +1284,19 @@ __global__ void __launch_bounds__(NT, 1)
         sw = (q < 2 ? p.sA0 : p.sA1) + ((size_t)t.wg * (p.I / 128) + t.ft) * KB;
       else
         sw = p.sA0 + ((size_t)t.wg * (p.D / 128) + t.ft * 2 + (int)rank) * KB;
-      // what the tile's end needs from memory is fetched now, so that its
-      // latency passes during the k-loop: each lane's token scales and (second
-      // matmul with the scatter) the tile's token and gate list
+      // each lane's token scales, which the tile's end needs, are fetched now
+      // so that their latency passes during the k-loop
       float sxr[CHUNKS];
 #pragma unroll
       for (int j = 0; j < CHUNKS; ++j) {
         const int c = (2 * j + half) * 32 + lane;
         sxr[j] = c < t.nvalid ? __ldg(p.sX + row0 + c) : 0.0f;
       }
-      int32_t *s_tok = reinterpret_cast<int32_t *>(xbuf);
-      float *s_gate = reinterpret_cast<float *>(s_tok + BN_MAX);
-      if (MODE == 3) {
-        const int et = threadIdx.x - 32 * EPI0;
-        named_bar_sync(5, 32 * EPI);  // the previous tile's readers are done
-        for (int c = et; c < t.nvalid; c += 32 * EPI) {
-          int tok;
-          float gate = 1.0f;
-          if (t.g < p.E) {
-            tok = p.sorted_token[row0 + c];
-            for (int jj = 0; jj < p.k; ++jj)
-              if (p.indices[(size_t)tok * p.k + jj] == t.g) gate = p.weights[(size_t)tok * p.k + jj];
-          } else {
-            tok = t.tok0 + c;
-          }
-          s_tok[c] = tok;
-          s_gate[c] = gate;
-        }
-      }
+      // MODE 3: this tile's (token, gate) list, written by the list builders
+      const int lb = ntile & 1;
+      const uint32_t lph = (uint32_t)(ntile >> 1) & 1u;
+      const int32_t *s_tok = reinterpret_cast<const int32_t *>(xbuf) + lb * 2 * BN_MAX;
+      const float *s_gate = reinterpret_cast<const float *>(s_tok + BN_MAX);
       // running sums: this lane's row, the warp's columns
       float acc[CHUNKS][32];
 #pragma unroll
@@ -1365,8 +1398,8 @@ __global__ void __launch_bounds__(NT, 1)
         }
       } else {
         // weighted scatter into y (gate 1 for the shared expert) with fp32
-        // atomic adds; the tile's token and gate list was written at its start
-        named_bar_sync(5, 32 * EPI);
+        // atomic adds
+        if (!wait_bounded(lfull + lb, lph, abort_flag, p.timeout_ns, p.status)) break;
         const int d = t.ft * 256 + (int)rank * BM + q * 32 + lane;
 #pragma unroll
         for (int j = 0; j < CHUNKS; ++j) {
@@ -1376,6 +1409,8 @@ __global__ void __launch_bounds__(NT, 1)
             if (c0 + e < t.nvalid)
               atomicAdd(p.y + (size_t)s_tok[c0 + e] * p.D + d, s_gate[c0 + e] * ACC(j, e));
         }
+        __syncwarp();  // this warp's reads of the list are done
+        if (lane == 0) mbar_arrive(lempty + lb);
       }
     }
   }
