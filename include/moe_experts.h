@@ -91,6 +91,8 @@ moe_status moe_experts_forward(const moe_cfg *cfg, int64_t T, const void *x, moe
  * into y is not fixed, so results may differ in the last bits from run to
  * run (use moe_experts_forward + moe_combine for bit-reproducible sums).
  * indices, weights [T, topk] from moe_router_forward; y [T, dim] fp32 out.
+ * With act_e4m3 = 1 y must be 16-byte aligned (the FP8 x FP8 epilogue adds
+ * 16-byte vectors into it); otherwise MOE_ERR_INVALID.
  */
 moe_status moe_experts_forward_combine(const moe_cfg *cfg, int64_t T, const void *x,
                                        moe_dtype x_dt, const moe_expert_weights *w,

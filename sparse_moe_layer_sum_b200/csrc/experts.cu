@@ -1037,12 +1037,16 @@ constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr int NPBUF = 2;               // TMEM partial-sum buffers of BN_MAX columns
 constexpr int CHUNKS = BN_MAX / 32 / 2;  // 32-column chunks per promotion warp
 constexpr int XB_STRIDE = 17;
+// second matmul with the scatter: chunks 0 .. SCH-1 of each promotion warp's
+// sums are handed to the two helper warps through shared memory, which add
+// them into y while the next tile's k-loop runs
+constexpr int SCH = 2;
 template <int MODE, int STAGES>
 struct Layout {
   static constexpr int BAR_OFF = STAGES * STAGE_BYTES;
   // full, empty per stage; partial full, partial empty per buffer; drain;
-  // list full, list empty per token list
-  static constexpr int NBARS = 2 * STAGES + 2 * NPBUF + 1 + 4;
+  // list full, list empty per token list; staged sums full, empty
+  static constexpr int NBARS = 2 * STAGES + 2 * NPBUF + 1 + 4 + 2;
   static constexpr int MISC_OFF = BAR_OFF + NBARS * 8;
   static constexpr int MISC_BYTES = 16 + 4 * STAGES;  // TMEM slot, abort flag, pending loads
   static constexpr int SC_OFF = (MISC_OFF + MISC_BYTES + 127) / 128 * 128;
@@ -1050,13 +1054,17 @@ struct Layout {
   static constexpr int XBUF_OFF = SC_OFF + SC_BYTES;
   // SwiGLU exchange of the four warp pairs (first matmul), or two (token,
   // gate) lists used by alternate tiles (second matmul with the scatter)
-  static constexpr int XBUF_BYTES = 4 * 2 * 32 * XB_STRIDE * 4;
-  static constexpr int TAB_OFF = XBUF_OFF + XBUF_BYTES;
+  static constexpr int XBUF_BYTES = MODE == 1 ? 4 * 2 * 32 * XB_STRIDE * 4 : 2 * BN_MAX * 8;
+  // staged sums (scatter): [promotion warp][chunk < SCH][token column][d]
+  static constexpr int STG_OFF = XBUF_OFF + XBUF_BYTES;
+  static constexpr int STG_BYTES = MODE == 3 ? EPI * SCH * 32 * 32 * 4 : 0;
+  static constexpr int TAB_OFF = STG_OFF + STG_BYTES;
   static size_t smem_bytes(int G, int E) {
     return 1024 + TAB_OFF + sizeof(int32_t) * (size_t)((G + 1) + G + (E + 1));
   }
   static_assert(2 * BN_MAX * 8 <= XBUF_BYTES, "token lists");
   static_assert(NPBUF * BN_MAX <= 512, "TMEM columns");
+  static_assert(SCH <= CHUNKS, "staged chunks");
 };
 
 // MODE 1: h = silu(x w1^T) * (x w3^T), bf16 out (the pair's 256 weight rows
@@ -1080,6 +1088,8 @@ __global__ void __launch_bounds__(NT, 1)
   uint64_t *drain = pempty + NPBUF;
   uint64_t *lfull = drain + 1;   // MODE 3: a tile's token list written
   uint64_t *lempty = lfull + 2;  // MODE 3: a tile's token list read
+  uint64_t *sfull = lempty + 2;  // MODE 3: a tile's staged sums written
+  uint64_t *sempty = sfull + 1;  // MODE 3: the staged sums added into y
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + L::MISC_OFF);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + L::MISC_OFF + 4);
   volatile int *pending = reinterpret_cast<volatile int *>(sm + L::MISC_OFF + 16);
@@ -1108,9 +1118,11 @@ __global__ void __launch_bounds__(NT, 1)
     }
     mbar_init(drain, 1);
     for (int b = 0; b < 2; ++b) {
-      mbar_init(lfull + b, 2);      // the two list-builder warps
-      mbar_init(lempty + b, EPI);   // the epilogue warps
+      mbar_init(lfull + b, 2);          // the two helper warps
+      mbar_init(lempty + b, EPI + 2);   // the epilogue and helper warps
     }
+    mbar_init(sfull, EPI);
+    mbar_init(sempty, 2);
     *abort_flag = 0;
     fence_mbar_init();
     tma_prefetch_desc(&tmA0);
@@ -1224,11 +1236,16 @@ __global__ void __launch_bounds__(NT, 1)
         drain_wait(drain, 0, p.timeout_ns);
       }
     } else if (MODE == 3 && warp >= 2) {
-      // ------------------------------------------------ token-list builders
-      // the (token, gate) list of each tile for the scatter into y (gate 1
-      // for the shared expert), written ahead of the tile's end into one of
-      // two lists that alternate between tiles
+      // ----------------------------------------------------- helper warps
+      // per tile: the (token, gate) list for the scatter into y (gate 1 for
+      // the shared expert), written into one of two lists that alternate
+      // between tiles well before the tile's end; then, once the promotion
+      // warps have staged their first SCH chunks of the tile's sums (gate
+      // applied), those sums are added into y with 16-byte reductions while
+      // the next tile's k-loop runs
+      const int hw = warp - 2;          // 0, 1
       const int bt = threadIdx.x - 64;  // 0 .. 63
+      const float *stg = reinterpret_cast<const float *>(sm + L::STG_OFF);
       int ntile = 0;
       for (int tile = unit; tile < total; tile += nunits, ++ntile) {
         const Tile t = decode_tile(tile, s_tstart, s_tbase, s_off, p.G, p.E, p.T, p.rows_routed, p.sh);
@@ -1236,7 +1253,7 @@ __global__ void __launch_bounds__(NT, 1)
         const uint32_t lph = (uint32_t)(ntile >> 1) & 1u;
         int32_t *s_tok = reinterpret_cast<int32_t *>(xbuf) + lb * 2 * BN_MAX;
         float *s_gate = reinterpret_cast<float *>(s_tok + BN_MAX);
-        // every epilogue warp is done with this list's previous tile
+        // every reader is done with this list's previous tile
         if (!wait_bounded(lempty + lb, lph ^ 1u, abort_flag, p.timeout_ns, p.status)) break;
         constexpr int PER = BN_MAX / 64;
         int tok[PER], pos[PER];
@@ -1262,6 +1279,31 @@ __global__ void __launch_bounds__(NT, 1)
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(lfull + lb);
+        // the tile's staged sums: unit u = promotion warp u / SCH, its chunk
+        // u % SCH; this warp takes every other unit.  Lane l adds 4
+        // consecutive d (l % 8) of token column l / 8 + 4 eb.
+        if (!wait_bounded(sfull, (uint32_t)ntile & 1u, abort_flag, p.timeout_ns, p.status)) break;
+        const int i4 = lane & 7, es = lane >> 3;
+        for (int u = hw; u < EPI * SCH; u += 2) {
+          const int w = u / SCH, jc = u % SCH;
+          const int c0 = (2 * jc + (w >> 2)) * 32;
+          if (c0 >= t.nvalid) continue;
+          float *yq = p.y + t.ft * 256 + (int)rank * BM + (w & 3) * 32 + 4 * i4;
+          const float *src = stg + (size_t)u * 32 * 32;
+#pragma unroll 4
+          for (int eb = 0; eb < 8; ++eb) {
+            const int e = 4 * eb + es;
+            if (c0 + e < t.nvalid) {
+              const float4 v = *reinterpret_cast<const float4 *>(src + e * 32 + 4 * i4);
+              red_add_v4_f32(yq + (size_t)s_tok[c0 + e] * p.D, v.x, v.y, v.z, v.w);
+            }
+          }
+        }
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(sempty);
+          mbar_arrive(lempty + lb);
+        }
       }
     }
   } else {
@@ -1397,17 +1439,59 @@ __global__ void __launch_bounds__(NT, 1)
             if (c0 + e < t.nvalid) out[(r0 + c0 + e) * p.D + d] = ACC(j, e);
         }
       } else {
-        // weighted scatter into y (gate 1 for the shared expert) with fp32
-        // atomic adds
+        // weighted scatter into y (gate 1 for the shared expert).  The first
+        // SCH chunks go to the helper warps through shared memory (gate
+        // applied), which add them into y during the next tile's k-loop;
+        // the rest are added here, while the MMA waits, with 16-byte fp32
+        // reductions: a lane holds one d for 32 tokens, so each quad of
+        // lanes transposes its 4 x 4 blocks (4 d by 4 tokens) with two
+        // shuffle rounds and lane t of a quad adds 4 consecutive d of token
+        // 4u + t -- a quarter of the reductions of one per element.
         if (!wait_bounded(lfull + lb, lph, abort_flag, p.timeout_ns, p.status)) break;
-        const int d = t.ft * 256 + (int)rank * BM + q * 32 + lane;
+        // the helpers are done with the previous tile's staged sums
+        if (!wait_bounded(sempty, ((uint32_t)ntile & 1u) ^ 1u, abort_flag, p.timeout_ns, p.status))
+          break;
+        {
+          float *stg = reinterpret_cast<float *>(sm + L::STG_OFF) +
+                       (size_t)(warp - EPI0) * SCH * 32 * 32;
 #pragma unroll
-        for (int j = 0; j < CHUNKS; ++j) {
+          for (int j = 0; j < SCH; ++j) {
+            const int c0 = (2 * j + half) * 32;
+            if (c0 >= t.nvalid) continue;
+#pragma unroll
+            for (int e = 0; e < 32; ++e) stg[(j * 32 + e) * 32 + lane] = s_gate[c0 + e] * ACC(j, e);
+          }
+          __syncwarp();
+          if (lane == 0) mbar_arrive(sfull);
+        }
+        const int t4 = lane & 3, hi = t4 >> 1, lo = t4 & 1;
+        float *yrow = p.y + t.ft * 256 + (int)rank * BM + q * 32 + (lane & ~3);
+#pragma unroll
+        for (int j = SCH; j < CHUNKS; ++j) {
           const int c0 = (2 * j + half) * 32;
+          if (c0 >= t.nvalid) continue;
 #pragma unroll
-          for (int e = 0; e < 32; ++e)
-            if (c0 + e < t.nvalid)
-              atomicAdd(p.y + (size_t)s_tok[c0 + e] * p.D + d, s_gate[c0 + e] * ACC(j, e));
+          for (int u = 0; u < 8; ++u) {
+            // M[r][s]: d = (lane & ~3) + r of the quarter, token c0 + 4u + s;
+            // this lane holds row r = t4
+            const float a0 = s_gate[c0 + 4 * u + 0] * ACC(j, 4 * u + 0);
+            const float a1 = s_gate[c0 + 4 * u + 1] * ACC(j, 4 * u + 1);
+            const float a2 = s_gate[c0 + 4 * u + 2] * ACC(j, 4 * u + 2);
+            const float a3 = s_gate[c0 + 4 * u + 3] * ACC(j, 4 * u + 3);
+            // round 1 (lanes t, t ^ 2): b[2 rr + cc] = M[lo + 2 rr][2 hi + cc]
+            const float y0 = __shfl_xor_sync(0xffffffffu, hi ? a0 : a2, 2);
+            const float y1 = __shfl_xor_sync(0xffffffffu, hi ? a1 : a3, 2);
+            const float b0 = hi ? y0 : a0, b1 = hi ? y1 : a1;
+            const float b2 = hi ? a2 : y0, b3 = hi ? a3 : y1;
+            // round 2 (lanes t, t ^ 1): column t4 of all four rows
+            const float z0 = __shfl_xor_sync(0xffffffffu, lo ? b0 : b1, 1);
+            const float z1 = __shfl_xor_sync(0xffffffffu, lo ? b2 : b3, 1);
+            const float o0 = lo ? b1 : b0, o1 = lo ? b3 : b2;
+            const int c = c0 + 4 * u + t4;
+            if (c < t.nvalid)
+              red_add_v4_f32(yrow + (size_t)s_tok[c] * p.D, lo ? z0 : o0, lo ? o0 : z0,
+                             lo ? z1 : o1, lo ? o1 : z1);
+          }
         }
         __syncwarp();  // this warp's reads of the list are done
         if (lane == 0) mbar_arrive(lempty + lb);
@@ -2074,6 +2158,10 @@ moe_status tc_down(const Job &j) {
 #ifndef MOE_F8_STAGES
 #define MOE_F8_STAGES 6
 #endif
+// the scatter variant gives 64 KB to its staged sums: four stages
+#ifndef MOE_F8_STAGES_SCATTER
+#define MOE_F8_STAGES_SCATTER 4
+#endif
 
 bool e4m3_tmap(CUtensorMap *m, const void *base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
   return make_tmap(m, base, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, rows, cols, box_rows, 128);
@@ -2149,7 +2237,7 @@ moe_status fp8_down(const Job &j) {
   p.sX = reinterpret_cast<const float *>(j.ws + j.l.hs);
   prof(3, j.s);
   if (j.y)
-    st = launch_fp8<3, MOE_F8_STAGES>(mw2, mw2, mh, p, j.s);
+    st = launch_fp8<3, MOE_F8_STAGES_SCATTER>(mw2, mw2, mh, p, j.s);
   else
     st = launch_fp8<2, MOE_F8_STAGES>(mw2, mw2, mh, p, j.s);
   prof(4, j.s);
@@ -2565,6 +2653,8 @@ MOE_EXPORT moe_status moe_experts_forward_combine(const moe_cfg *cfg, int64_t T,
                            dev_status, stream, true, true);
   if (st != MOE_OK || T == 0) return st;
   if (!indices || !weights || !y) return MOE_ERR_INVALID;
+  // the FP8 x FP8 scatter adds 16-byte vectors into y
+  if (w->act_e4m3 && (reinterpret_cast<uintptr_t>(y) & 15u) != 0) return MOE_ERR_INVALID;
   j.out_perm = nullptr;
   j.out_shared = nullptr;
   j.indices = indices;
@@ -2616,6 +2706,8 @@ MOE_EXPORT moe_status moe_experts_forward_combine_ep(
   if ((st = ep_plan(cfg, T, shard, &sh)) != MOE_OK) return st;
   if (T == 0) return MOE_OK;
   if (!indices || !weights || !y) return MOE_ERR_INVALID;
+  // the FP8 x FP8 scatter adds 16-byte vectors into y
+  if (w->act_e4m3 && (reinterpret_cast<uintptr_t>(y) & 15u) != 0) return MOE_ERR_INVALID;
   j.out_perm = nullptr;
   j.out_shared = nullptr;
   j.indices = indices;

@@ -91,6 +91,14 @@ __device__ __forceinline__ void fence_proxy_async_global() {
   asm volatile("fence.proxy.async.global;" ::: "memory");
 }
 
+// *addr .. addr[3] += (a, b, c, d): one 16-byte fp32 reduction in global
+// memory (relaxed, device scope); addr must be 16-byte aligned.
+__device__ __forceinline__ void red_add_v4_f32(float *addr, float a, float b, float c, float d) {
+  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b), "f"(c),
+               "f"(d)
+               : "memory");
+}
+
 // Waits for the phase with the given parity to complete, for at most
 // limit_ns.  Returns false (after raising *abort and recording
 // MOE_ERR_TIMEOUT) when the limit expires, or false at once when another

@@ -162,6 +162,11 @@ def test_fp8_activation_path_validation():
     assert call(c, bf) == UNSUPPORTED                          # e4m3 weights only
     assert call(c, fp8(1), x_dt=0) == UNSUPPORTED              # bf16 activations in
     assert call(v3_cfg(dim=7296), fp8(1)) == UNSUPPORTED       # dim % 256 != 0
+    # the FP8 x FP8 scatter adds 16-byte vectors into y: a y off that
+    # alignment is refused before any launch
+    fc = fn("moe_experts", "moe_experts_forward_combine")
+    assert fc(ctypes.byref(c), 8, P, 1, ctypes.byref(fp8(1)), P, P, P, P, ctypes.c_void_p(0x1004), P, 1 << 40,
+              None, None) == INVALID
     q = fn("moe_experts", "moe_quantize_e4m3_rows")
     assert q(P, 4, 102, P, P, None) == INVALID                 # K % 4 != 0
     assert q(None, 4, 128, P, P, None) == INVALID
