@@ -1379,10 +1379,12 @@ __global__ void __launch_bounds__(NT, 1)
       }
       if (!ok) break;
       // times each token's activation scale (one per row, the same for every
-      // k-block), handed from the lane that holds it to all lanes through
-      // this warp's shared-memory slots
+      // k-block) -- and, for the scatter, its gate -- handed from the lane
+      // that holds it to all lanes through this warp's shared-memory slots
+      if (MODE == 3 && !wait_bounded(lfull + lb, lph, abort_flag, p.timeout_ns, p.status)) break;
 #pragma unroll
-      for (int j = 0; j < CHUNKS; ++j) comb[j * 32 + lane] = sxr[j];
+      for (int j = 0; j < CHUNKS; ++j)
+        comb[j * 32 + lane] = MODE == 3 ? sxr[j] * s_gate[(2 * j + half) * 32 + lane] : sxr[j];
       __syncwarp();
 #pragma unroll
       for (int j = 0; j < CHUNKS; ++j)
@@ -1439,15 +1441,15 @@ __global__ void __launch_bounds__(NT, 1)
             if (c0 + e < t.nvalid) out[(r0 + c0 + e) * p.D + d] = ACC(j, e);
         }
       } else {
-        // weighted scatter into y (gate 1 for the shared expert).  The first
-        // SCH chunks go to the helper warps through shared memory (gate
-        // applied), which add them into y during the next tile's k-loop;
+        // weighted scatter into y (the sums already carry the gate, 1 for
+        // the shared expert).  The first SCH chunks go to the helper warps
+        // through shared memory, which add them into y during the next
+        // tile's k-loop;
         // the rest are added here, while the MMA waits, with 16-byte fp32
         // reductions: a lane holds one d for 32 tokens, so each quad of
         // lanes transposes its 4 x 4 blocks (4 d by 4 tokens) with two
         // shuffle rounds and lane t of a quad adds 4 consecutive d of token
         // 4u + t -- a quarter of the reductions of one per element.
-        if (!wait_bounded(lfull + lb, lph, abort_flag, p.timeout_ns, p.status)) break;
         // the helpers are done with the previous tile's staged sums
         if (!wait_bounded(sempty, ((uint32_t)ntile & 1u) ^ 1u, abort_flag, p.timeout_ns, p.status))
           break;
@@ -1459,7 +1461,7 @@ __global__ void __launch_bounds__(NT, 1)
             const int c0 = (2 * j + half) * 32;
             if (c0 >= t.nvalid) continue;
 #pragma unroll
-            for (int e = 0; e < 32; ++e) stg[(j * 32 + e) * 32 + lane] = s_gate[c0 + e] * ACC(j, e);
+            for (int e = 0; e < 32; ++e) stg[(j * 32 + e) * 32 + lane] = ACC(j, e);
           }
           __syncwarp();
           if (lane == 0) mbar_arrive(sfull);
@@ -1474,10 +1476,8 @@ __global__ void __launch_bounds__(NT, 1)
           for (int u = 0; u < 8; ++u) {
             // M[r][s]: d = (lane & ~3) + r of the quarter, token c0 + 4u + s;
             // this lane holds row r = t4
-            const float a0 = s_gate[c0 + 4 * u + 0] * ACC(j, 4 * u + 0);
-            const float a1 = s_gate[c0 + 4 * u + 1] * ACC(j, 4 * u + 1);
-            const float a2 = s_gate[c0 + 4 * u + 2] * ACC(j, 4 * u + 2);
-            const float a3 = s_gate[c0 + 4 * u + 3] * ACC(j, 4 * u + 3);
+            const float a0 = ACC(j, 4 * u + 0), a1 = ACC(j, 4 * u + 1);
+            const float a2 = ACC(j, 4 * u + 2), a3 = ACC(j, 4 * u + 3);
             // round 1 (lanes t, t ^ 2): b[2 rr + cc] = M[lo + 2 rr][2 hi + cc]
             const float y0 = __shfl_xor_sync(0xffffffffu, hi ? a0 : a2, 2);
             const float y1 = __shfl_xor_sync(0xffffffffu, hi ? a1 : a3, 2);
