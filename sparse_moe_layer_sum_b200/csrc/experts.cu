@@ -1037,10 +1037,12 @@ constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr int NPBUF = 2;               // TMEM partial-sum buffers of BN_MAX columns
 constexpr int CHUNKS = BN_MAX / 32 / 2;  // 32-column chunks per promotion warp
 constexpr int XB_STRIDE = 17;
-// second matmul with the scatter: chunks 0 .. SCH-1 of each promotion warp's
-// sums are handed to the two helper warps through shared memory, which add
-// them into y while the next tile's k-loop runs
+// chunks 0 .. SCH-1 of each promotion warp's sums (token columns 0-127 of a
+// tile) are handed to the two helper warps through shared memory, which
+// finish them while the next tile's k-loop runs: the SwiGLU and h in the
+// first matmul, the reductions into y in the second with the scatter
 constexpr int SCH = 2;
+__host__ __device__ constexpr bool staged(int mode) { return mode == 1 || mode == 3; }
 template <int MODE, int STAGES>
 struct Layout {
   static constexpr int BAR_OFF = STAGES * STAGE_BYTES;
@@ -1057,7 +1059,7 @@ struct Layout {
   static constexpr int XBUF_BYTES = MODE == 1 ? 4 * 2 * 32 * XB_STRIDE * 4 : 2 * BN_MAX * 8;
   // staged sums (scatter): [promotion warp][chunk < SCH][token column][d]
   static constexpr int STG_OFF = XBUF_OFF + XBUF_BYTES;
-  static constexpr int STG_BYTES = MODE == 3 ? EPI * SCH * 32 * 32 * 4 : 0;
+  static constexpr int STG_BYTES = staged(MODE) ? EPI * SCH * 32 * 32 * 4 : 0;
   static constexpr int TAB_OFF = STG_OFF + STG_BYTES;
   static size_t smem_bytes(int G, int E) {
     return 1024 + TAB_OFF + sizeof(int32_t) * (size_t)((G + 1) + G + (E + 1));
@@ -1088,8 +1090,8 @@ __global__ void __launch_bounds__(NT, 1)
   uint64_t *drain = pempty + NPBUF;
   uint64_t *lfull = drain + 1;   // MODE 3: a tile's token list written
   uint64_t *lempty = lfull + 2;  // MODE 3: a tile's token list read
-  uint64_t *sfull = lempty + 2;  // MODE 3: a tile's staged sums written
-  uint64_t *sempty = sfull + 1;  // MODE 3: the staged sums added into y
+  uint64_t *sfull = lempty + 2;  // MODES 1, 3: a tile's staged sums written
+  uint64_t *sempty = sfull + 1;  // MODES 1, 3: the staged sums finished
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + L::MISC_OFF);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + L::MISC_OFF + 4);
   volatile int *pending = reinterpret_cast<volatile int *>(sm + L::MISC_OFF + 16);
@@ -1234,6 +1236,39 @@ __global__ void __launch_bounds__(NT, 1)
         // make sure no MMA is still writing TMEM before it is freed
         mma_commit_pair(drain);
         drain_wait(drain, 0, p.timeout_ns);
+      }
+    } else if (MODE == 1 && warp >= 2) {
+      // ----------------------------------------------------- helper warps
+      // the staged sums of each tile (columns 0-127): a = w1.x in TMEM rows
+      // 0-63 and u = w3.x in rows 64-127 of the same 64 features meet here;
+      // h = silu(a) * u in bf16.  Lane l takes features 2l, 2l + 1 (4-byte
+      // stores, 128 bytes per token row and warp), the two warps alternate
+      // token columns.
+      const int hw = warp - 2;
+      const float *stg = reinterpret_cast<const float *>(sm + L::STG_OFF);
+      const int qa = lane >> 4;             // TMEM lane quarter of the two a rows
+      const int fl = (2 * lane) & 31;        // their lane within the quarter
+      bf16 *out = static_cast<bf16 *>(p.out);
+      int ntile = 0;
+      for (int tile = unit; tile < total; tile += nunits, ++ntile) {
+        const Tile t = decode_tile(tile, s_tstart, s_tbase, s_off, p.G, p.E, p.T, p.rows_routed, p.sh);
+        const int row0 = t.rowbase + t.n0;
+        __nv_bfloat162 *orow =
+            reinterpret_cast<__nv_bfloat162 *>(out + t.ft * 128 + (int)rank * 64 + 2 * lane);
+        if (!wait_bounded(sfull, (uint32_t)ntile & 1u, abort_flag, p.timeout_ns, p.status)) break;
+        const int ncol = t.nvalid < 128 ? t.nvalid : 128;
+        for (int c = hw; c < ncol; c += 2) {
+          // column c: warp half (c / 32) % 2, chunk c / 64, element c % 32
+          const int h2 = (c >> 5) & 1, jc = c >> 6, e = c & 31;
+          const float2 a = *reinterpret_cast<const float2 *>(
+              stg + ((size_t)((qa + 4 * h2) * SCH + jc) * 32 + e) * 32 + fl);
+          const float2 u = *reinterpret_cast<const float2 *>(
+              stg + ((size_t)((qa + 2 + 4 * h2) * SCH + jc) * 32 + e) * 32 + fl);
+          orow[(size_t)(row0 + c) * (p.I / 2)] =
+              __floats2bfloat162_rn(swiglu_h(a.x, u.x), swiglu_h(a.y, u.y));
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(sempty);
       }
     } else if (MODE == 3 && warp >= 2) {
       // ----------------------------------------------------- helper warps
@@ -1392,10 +1427,28 @@ __global__ void __launch_bounds__(NT, 1)
         for (int e = 0; e < 32; ++e) acc[j][e] *= comb[j * 32 + e];
       __syncwarp();
 
+      if (staged(MODE)) {
+        // the first SCH chunks go to the helper warps through shared memory,
+        // once they are done with the previous tile's
+        if (!wait_bounded(sempty, ((uint32_t)ntile & 1u) ^ 1u, abort_flag, p.timeout_ns, p.status))
+          break;
+        float *stg = reinterpret_cast<float *>(sm + L::STG_OFF) + (size_t)(warp - EPI0) * SCH * 32 * 32;
+#pragma unroll
+        for (int j = 0; j < SCH; ++j) {
+          const int c0 = (2 * j + half) * 32;
+          if (c0 >= t.nvalid) continue;
+#pragma unroll
+          for (int e = 0; e < 32; ++e) stg[(j * 32 + e) * 32 + lane] = ACC(j, e);
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(sfull);
+      }
+
       if (MODE == 1) {
         // lanes 0-63 of the CTA hold w1.x (a), lanes 64-127 w3.x (u) of the
-        // same 64 features; warps q and q+2 of one half pair up through
-        // shared memory, each finishing 16 of the 32 columns of a chunk
+        // same 64 features; for the chunks not staged, warps q and q+2 of
+        // one half pair up through shared memory, each finishing 16 of the
+        // 32 columns of a chunk
         const int pr = q & 1;
         const bool is_a = q < 2;
         float *buf_a = xbuf + (pr + 2 * half) * 2 * 32 * XB_STRIDE;
@@ -1404,7 +1457,7 @@ __global__ void __launch_bounds__(NT, 1)
         const int f = t.ft * 128 + (int)rank * 64 + pr * 32 + lane;
         bf16 *out = static_cast<bf16 *>(p.out);
 #pragma unroll
-        for (int j = 0; j < CHUNKS; ++j) {
+        for (int j = SCH; j < CHUNKS; ++j) {
           const int c0 = (2 * j + half) * 32;
           if (c0 >= t.nvalid) continue;
           float *mine = is_a ? buf_a : buf_u;
@@ -1450,22 +1503,6 @@ __global__ void __launch_bounds__(NT, 1)
         // lanes transposes its 4 x 4 blocks (4 d by 4 tokens) with two
         // shuffle rounds and lane t of a quad adds 4 consecutive d of token
         // 4u + t -- a quarter of the reductions of one per element.
-        // the helpers are done with the previous tile's staged sums
-        if (!wait_bounded(sempty, ((uint32_t)ntile & 1u) ^ 1u, abort_flag, p.timeout_ns, p.status))
-          break;
-        {
-          float *stg = reinterpret_cast<float *>(sm + L::STG_OFF) +
-                       (size_t)(warp - EPI0) * SCH * 32 * 32;
-#pragma unroll
-          for (int j = 0; j < SCH; ++j) {
-            const int c0 = (2 * j + half) * 32;
-            if (c0 >= t.nvalid) continue;
-#pragma unroll
-            for (int e = 0; e < 32; ++e) stg[(j * 32 + e) * 32 + lane] = ACC(j, e);
-          }
-          __syncwarp();
-          if (lane == 0) mbar_arrive(sfull);
-        }
         const int t4 = lane & 3, hi = t4 >> 1, lo = t4 & 1;
         float *yrow = p.y + t.ft * 256 + (int)rank * BM + q * 32 + (lane & ~3);
 #pragma unroll
@@ -2158,9 +2195,10 @@ moe_status tc_down(const Job &j) {
 #ifndef MOE_F8_STAGES
 #define MOE_F8_STAGES 6
 #endif
-// the scatter variant gives 64 KB to its staged sums: four stages
-#ifndef MOE_F8_STAGES_SCATTER
-#define MOE_F8_STAGES_SCATTER 4
+// the first matmul and the scatter variant give 64 KB to their staged sums:
+// four stages
+#ifndef MOE_F8_STAGES_STAGED
+#define MOE_F8_STAGES_STAGED 4
 #endif
 
 bool e4m3_tmap(CUtensorMap *m, const void *base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
@@ -2208,7 +2246,7 @@ moe_status fp8_up(const Job &j) {
   p.sA1 = j.w->s3;
   p.sX = reinterpret_cast<const float *>(j.ws + j.l.xs);
   prof(1, j.s);
-  st = launch_fp8<1, MOE_F8_STAGES>(mw1, mw3, mx, p, j.s);
+  st = launch_fp8<1, MOE_F8_STAGES_STAGED>(mw1, mw3, mx, p, j.s);
   prof(2, j.s);
   if (st != MOE_OK) return st;
   // h (bf16) to e4m3 codes and scales for the second matmul
@@ -2237,7 +2275,7 @@ moe_status fp8_down(const Job &j) {
   p.sX = reinterpret_cast<const float *>(j.ws + j.l.hs);
   prof(3, j.s);
   if (j.y)
-    st = launch_fp8<3, MOE_F8_STAGES_SCATTER>(mw2, mw2, mh, p, j.s);
+    st = launch_fp8<3, MOE_F8_STAGES_STAGED>(mw2, mw2, mh, p, j.s);
   else
     st = launch_fp8<2, MOE_F8_STAGES>(mw2, mw2, mh, p, j.s);
   prof(4, j.s);
