@@ -90,9 +90,9 @@ moe_status moe_experts_forward(const moe_cfg *cfg, int64_t T, const void *x, moe
  * round trip through memory; in exchange the order of the fp32 additions
  * into y is not fixed, so results may differ in the last bits from run to
  * run (use moe_experts_forward + moe_combine for bit-reproducible sums).
- * indices, weights [T, topk] from moe_router_forward; y [T, dim] fp32 out.
- * With act_e4m3 = 1 y must be 16-byte aligned (the FP8 x FP8 epilogue adds
- * 16-byte vectors into it); otherwise MOE_ERR_INVALID.
+ * indices, weights [T, topk] from moe_router_forward; y [T, dim] fp32 out,
+ * 16-byte aligned (the epilogue adds 16-byte vectors into it; otherwise
+ * MOE_ERR_INVALID).
  */
 moe_status moe_experts_forward_combine(const moe_cfg *cfg, int64_t T, const void *x,
                                        moe_dtype x_dt, const moe_expert_weights *w,
@@ -158,7 +158,7 @@ moe_status moe_experts_forward_combine_ep(const moe_cfg *cfg, int64_t T, const v
  *   weights, indices [T, topk], sel_gap [T] (may be NULL): as moe_router_forward
  *   counts [n_routed], offsets [n_routed + 1], sorted_token, slot_of
  *             [T * topk]: as moe_dispatch_build
- *   y         [T, dim] fp32 out (zeroed by the call first)
+ *   y         [T, dim] fp32 out (zeroed by the call first), 16-byte aligned
  *   ws        moe_block_decode_workspace_size(cfg, T) bytes
  * Limits: the decode regime, T * topk <= 16 * n_routed; n_routed <= 256,
  * n_groups <= 32, topk <= 32, n_shared == 1, dim and inter multiples of 128;

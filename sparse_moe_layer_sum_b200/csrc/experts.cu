@@ -775,15 +775,36 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap &tmA0, const CUtenso
         // the 32 columns from c0 of accumulator a, read into v
         auto store = [&](int a, int c0, const uint32_t *v) {
           const int d = t.ft * L::FEAT + a * BM * CG + (int)rank * BM + q * 32 + lane;
+          if (MODE == 3) {
+            // 16-byte fp32 reductions: a lane holds one d for 32 tokens, so
+            // each quad of lanes transposes its 4 x 4 blocks (4 d by 4
+            // tokens) in two shuffle rounds and lane t of a quad adds 4
+            // consecutive d of token 4u + t -- a quarter of the reductions
+            const int t4 = lane & 3, hi = t4 >> 1, lo = t4 & 1;
+            float *yq = p.y + (d - (lane & 3));
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            if (c0 + j < t.nvalid) {
-              const float o = __uint_as_float(v[j]) * acc_scale;
-              if (MODE == 3)
-                atomicAdd(p.y + (size_t)s_tok[c0 + j] * p.D + d, s_gate[c0 + j] * o);
-              else
-                out[(row0 + c0 + j) * p.D + d] = o;
+            for (int u = 0; u < 8; ++u) {
+              // M[r][s]: d of lane (lane & ~3) + r, token c0 + 4u + s
+              const float m0 = s_gate[c0 + 4 * u + 0] * (__uint_as_float(v[4 * u + 0]) * acc_scale);
+              const float m1 = s_gate[c0 + 4 * u + 1] * (__uint_as_float(v[4 * u + 1]) * acc_scale);
+              const float m2 = s_gate[c0 + 4 * u + 2] * (__uint_as_float(v[4 * u + 2]) * acc_scale);
+              const float m3 = s_gate[c0 + 4 * u + 3] * (__uint_as_float(v[4 * u + 3]) * acc_scale);
+              const float y0 = __shfl_xor_sync(0xffffffffu, hi ? m0 : m2, 2);
+              const float y1 = __shfl_xor_sync(0xffffffffu, hi ? m1 : m3, 2);
+              const float b0 = hi ? y0 : m0, b1 = hi ? y1 : m1;
+              const float b2 = hi ? m2 : y0, b3 = hi ? m3 : y1;
+              const float z0 = __shfl_xor_sync(0xffffffffu, lo ? b0 : b1, 1);
+              const float z1 = __shfl_xor_sync(0xffffffffu, lo ? b2 : b3, 1);
+              const float o0 = lo ? b1 : b0, o1 = lo ? b3 : b2;
+              const int c = c0 + 4 * u + t4;
+              if (c < t.nvalid)
+                red_add_v4_f32(yq + (size_t)s_tok[c] * p.D, lo ? z0 : o0, lo ? o0 : z0,
+                               lo ? z1 : o1, lo ? o1 : z1);
             }
+          } else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              if (c0 + j < t.nvalid) out[(row0 + c0 + j) * p.D + d] = __uint_as_float(v[j]) * acc_scale;
           }
         };
         if (L::NBUF == 1) {
@@ -2691,8 +2712,8 @@ MOE_EXPORT moe_status moe_experts_forward_combine(const moe_cfg *cfg, int64_t T,
                            dev_status, stream, true, true);
   if (st != MOE_OK || T == 0) return st;
   if (!indices || !weights || !y) return MOE_ERR_INVALID;
-  // the FP8 x FP8 scatter adds 16-byte vectors into y
-  if (w->act_e4m3 && (reinterpret_cast<uintptr_t>(y) & 15u) != 0) return MOE_ERR_INVALID;
+  // the scatter adds 16-byte vectors into y
+  if ((reinterpret_cast<uintptr_t>(y) & 15u) != 0) return MOE_ERR_INVALID;
   j.out_perm = nullptr;
   j.out_shared = nullptr;
   j.indices = indices;
@@ -2744,8 +2765,8 @@ MOE_EXPORT moe_status moe_experts_forward_combine_ep(
   if ((st = ep_plan(cfg, T, shard, &sh)) != MOE_OK) return st;
   if (T == 0) return MOE_OK;
   if (!indices || !weights || !y) return MOE_ERR_INVALID;
-  // the FP8 x FP8 scatter adds 16-byte vectors into y
-  if (w->act_e4m3 && (reinterpret_cast<uintptr_t>(y) & 15u) != 0) return MOE_ERR_INVALID;
+  // the scatter adds 16-byte vectors into y
+  if ((reinterpret_cast<uintptr_t>(y) & 15u) != 0) return MOE_ERR_INVALID;
   j.out_perm = nullptr;
   j.out_shared = nullptr;
   j.indices = indices;
@@ -2794,6 +2815,7 @@ MOE_EXPORT moe_status moe_block_forward_decode(
   if (!x || !w_r || !weights || !indices || !counts || !offsets || !sorted_token || !slot_of ||
       !y || !ws || (cfg->has_bias && !bias))
     return MOE_ERR_INVALID;
+  if ((reinterpret_cast<uintptr_t>(y) & 15u) != 0) return MOE_ERR_INVALID;  // 16-byte reductions
   const DecodePlan pl = decode_plan(cfg, T, sm_count());
   if (ws_bytes < decode_plan(cfg, T, 0).total) return MOE_ERR_WORKSPACE;
   Job j;

@@ -145,6 +145,9 @@ def test_experts_validation():
               None) == INVALID
     assert fc(ctypes.byref(c), 8, P, 1, ctypes.byref(w), P, P, P, P, P, P, 8, None,
               None) == WORKSPACE
+    # y must be 16-byte aligned (the scatter adds 16-byte vectors)
+    assert fc(ctypes.byref(c), 8, P, 1, ctypes.byref(w), P, P, P, P, ctypes.c_void_p(0x1008), P,
+              1 << 40, None, None) == INVALID
     # empty batch: validated, then nothing to launch
     assert f(ctypes.byref(c), 0, P, 1, ctypes.byref(w), P, P, P, P, P, 1 << 40, None, None) == 0
     assert fc(ctypes.byref(c), 0, P, 1, ctypes.byref(w), P, P, P, P, P, P, 1 << 40, None,
@@ -162,8 +165,8 @@ def test_fp8_activation_path_validation():
     assert call(c, bf) == UNSUPPORTED                          # e4m3 weights only
     assert call(c, fp8(1), x_dt=0) == UNSUPPORTED              # bf16 activations in
     assert call(v3_cfg(dim=7296), fp8(1)) == UNSUPPORTED       # dim % 256 != 0
-    # the FP8 x FP8 scatter adds 16-byte vectors into y: a y off that
-    # alignment is refused before any launch
+    # the scatter adds 16-byte vectors into y: a y off that alignment is
+    # refused before any launch
     fc = fn("moe_experts", "moe_experts_forward_combine")
     assert fc(ctypes.byref(c), 8, P, 1, ctypes.byref(fp8(1)), P, P, P, P, ctypes.c_void_p(0x1004), P, 1 << 40,
               None, None) == INVALID
@@ -208,8 +211,8 @@ def test_fused_decode_validation():
     assert size(ctypes.byref(v3_cfg(topk=200)), 8) == 0
     w = MoEExpertWeights(0x1000, 0x1000, 0x1000, 1, None, None, None)
 
-    def call(cfg=c, T=64, x_dt=1, wt=w, ws=1 << 40, x=P):
-        return f(ctypes.byref(cfg), T, x, x_dt, P, P, ctypes.byref(wt), P, P, None, P, P, P, P, P,
+    def call(cfg=c, T=64, x_dt=1, wt=w, ws=1 << 40, x=P, y=P):
+        return f(ctypes.byref(cfg), T, x, x_dt, P, P, ctypes.byref(wt), P, P, None, P, P, P, P, y,
                  P, ws, None, None)
     assert call(T=4096) == UNSUPPORTED                          # not a decode batch
     assert call(x_dt=0) == UNSUPPORTED                          # bf16 x only
@@ -217,6 +220,7 @@ def test_fused_decode_validation():
     assert call(wt=fp8) == UNSUPPORTED                          # bf16 weights only
     assert call(cfg=v3_cfg(n_routed=512, n_groups=8)) == UNSUPPORTED
     assert call(x=None) == INVALID
+    assert call(y=ctypes.c_void_p(0x1004)) == INVALID           # y not 16-byte aligned
     assert call(ws=1024) == WORKSPACE
     assert call(T=0) == 0                                       # empty batch
     assert call(T=-1) == INVALID
