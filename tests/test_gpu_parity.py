@@ -41,6 +41,9 @@ ROUTER_TC_SPLIT = custom("router_tc_split", 40, dim=2048, n_routed=256, n_groups
 # dim % 256 != 0: the prefill path falls back to one SM per tile
 CG1_PREFILL = custom("cg1_prefill", 230, dim=384, n_routed=16, n_groups=4, topk_groups=2, topk=4,
                      inter=128, seed=22)
+# dim % 512 == 256: the second matmul's SM pairs keep one weight tile per SM
+PAIR_AT1 = custom("pair_at1", 300, dim=768, n_routed=32, n_groups=4, topk_groups=2, topk=8,
+                  inter=256, seed=27)
 FP8_SMALL = custom("fp8_small", 260, w_format="e4m3", dim=512, n_routed=16, n_groups=4,
                    topk_groups=2, topk=4, inter=256, seed=17)
 FP8_DECODE = custom("fp8_decode", 40, w_format="e4m3", dim=1024, n_routed=64, n_groups=8,
@@ -155,7 +158,7 @@ def test_dispatch_reports_out_of_range():
 
 
 @pytest.mark.parametrize("w", [WORKLOADS["tiny_f32"], TINY_BF16, MID, MID_F32, DECODE_SMALL,
-                               ONE_TOKEN, CG1_PREFILL, FP8_SMALL, FP8_DECODE, FP8_CG1],
+                               ONE_TOKEN, CG1_PREFILL, PAIR_AT1, FP8_SMALL, FP8_DECODE, FP8_CG1],
                          ids=lambda w: w.name)
 def test_experts_rows_match_oracle(w):
     """Expert outputs row by row, on a seeded index set (routing held fixed)."""
@@ -197,8 +200,8 @@ def test_experts_rows_match_oracle(w):
 
 @pytest.mark.parametrize("combine", ["scatter", "ordered"])
 @pytest.mark.parametrize("w", [WORKLOADS["tiny_f32"], TINY_BF16, MID, MID_F32, SOFTMAX_NOBIAS,
-                               ONE_GROUP, DECODE_SMALL, ONE_TOKEN, CG1_PREFILL, FP8_SMALL,
-                               FP8_DECODE, FP8_CG1, MID_SKEW, FP8_SKEW],
+                               ONE_GROUP, DECODE_SMALL, ONE_TOKEN, CG1_PREFILL, PAIR_AT1,
+                               FP8_SMALL, FP8_DECODE, FP8_CG1, MID_SKEW, FP8_SKEW],
                          ids=lambda w: w.name)
 def test_block_matches_oracle(w, combine):
     x, p = make_block(w)
