@@ -197,23 +197,50 @@ __global__ void __launch_bounds__(256) gather_rows(const uint4 *__restrict__ x,
   const int src = row < rows_routed ? sorted_token[row] : (row - rows_routed) % T;
   const uint4 *s = x + (size_t)src * vec_per_row;
   uint4 *d = xp + (size_t)row * vec_per_row;
-  for (int v = lane; v < vec_per_row; v += 32) d[v] = __ldg(s + v);
+  // four 16-byte loads in flight per lane before their stores
+  int v = lane;
+  for (; v + 96 < vec_per_row; v += 128) {
+    const uint4 a = __ldg(s + v), b = __ldg(s + v + 32), c = __ldg(s + v + 64), e = __ldg(s + v + 96);
+    d[v] = a;
+    d[v + 32] = b;
+    d[v + 64] = c;
+    d[v + 96] = e;
+  }
+  for (; v < vec_per_row; v += 32) d[v] = __ldg(s + v);
 }
 
 // The same rows converted to fp16 (the e4m3 path computes in fp16; bf16 values
 // in the fp16 normal range convert exactly).
-__global__ void __launch_bounds__(256) gather_rows_f16(const __nv_bfloat162 *__restrict__ x,
+__device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t v) {
+  const __half2 h = __float22half2_rn(__bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&v)));
+  return *reinterpret_cast<const uint32_t *>(&h);
+}
+
+__global__ void __launch_bounds__(256) gather_rows_f16(const uint4 *__restrict__ x,
                                                        const int32_t *__restrict__ sorted_token,
-                                                       __half2 *__restrict__ xp, int rows_routed,
-                                                       int rows_total, int T, int pairs_per_row,
+                                                       uint4 *__restrict__ xp, int rows_routed,
+                                                       int rows_total, int T, int vec_per_row,
                                                        const int32_t *off, Shard sh) {
   const int row = (int)((blockIdx.x * (size_t)blockDim.x + threadIdx.x) / 32);
   const int lane = threadIdx.x % 32;
   if (row >= rows_total || !row_in_shard(row, rows_routed, T, off, sh)) return;
   const int src = row < rows_routed ? sorted_token[row] : (row - rows_routed) % T;
-  const __nv_bfloat162 *s = x + (size_t)src * pairs_per_row;
-  __half2 *d = xp + (size_t)row * pairs_per_row;
-  for (int v = lane; v < pairs_per_row; v += 32) d[v] = __float22half2_rn(__bfloat1622float2(s[v]));
+  const uint4 *s = x + (size_t)src * vec_per_row;
+  uint4 *d = xp + (size_t)row * vec_per_row;
+  // 8 values per 16-byte vector, two vectors in flight per lane
+  int v = lane;
+  for (; v + 32 < vec_per_row; v += 64) {
+    const uint4 a = __ldg(s + v), b = __ldg(s + v + 32);
+    d[v] = make_uint4(bf16x2_to_f16x2(a.x), bf16x2_to_f16x2(a.y), bf16x2_to_f16x2(a.z),
+                      bf16x2_to_f16x2(a.w));
+    d[v + 32] = make_uint4(bf16x2_to_f16x2(b.x), bf16x2_to_f16x2(b.y), bf16x2_to_f16x2(b.z),
+                           bf16x2_to_f16x2(b.w));
+  }
+  for (; v < vec_per_row; v += 32) {
+    const uint4 a = __ldg(s + v);
+    d[v] = make_uint4(bf16x2_to_f16x2(a.x), bf16x2_to_f16x2(a.y), bf16x2_to_f16x2(a.z),
+                      bf16x2_to_f16x2(a.w));
+  }
 }
 
 // ------------------------------------------------------- tensor-core GEMMs
@@ -2152,9 +2179,8 @@ moe_status tc_up(const Job &j) {
   const int64_t threads = (int64_t)j.rows_total() * 32;
   if (F8)
     gather_rows_f16<<<(unsigned)((threads + 255) / 256), 256, 0, j.s>>>(
-        static_cast<const __nv_bfloat162 *>(j.x), j.sorted_token,
-        reinterpret_cast<__half2 *>(xperm), j.rows_routed(), j.rows_total(), (int)j.T, D / 2,
-        j.shard_off(), j.sh);
+        static_cast<const uint4 *>(j.x), j.sorted_token, reinterpret_cast<uint4 *>(xperm),
+        j.rows_routed(), j.rows_total(), (int)j.T, D * 2 / 16, j.shard_off(), j.sh);
   else
     gather_rows<<<(unsigned)((threads + 255) / 256), 256, 0, j.s>>>(
         static_cast<const uint4 *>(j.x), j.sorted_token, reinterpret_cast<uint4 *>(xperm),
@@ -2394,9 +2420,8 @@ moe_status simt_down_w(const Job &j) {
 #endif
 // weight tiles per SM in the first matmul (two: w1 and w3 in accumulators of
 // their own, half the token bytes per weight byte) and in the second (two
-// blocks of w2 rows with bf16 weights, for the same reason, their single
-// accumulator handed back before the last stores of each tile; one with e4m3
-// weights, where two measured no faster)
+// blocks of w2 rows, for the same reason, their single accumulator handed
+// back before the last stores of each tile)
 #ifndef MOE_TC_PREFILL_AT_UP
 #define MOE_TC_PREFILL_AT_UP 2
 #endif
@@ -2404,7 +2429,7 @@ moe_status simt_down_w(const Job &j) {
 #define MOE_TC_PREFILL_AT_DOWN 2
 #endif
 #ifndef MOE_TC_PREFILL_AT_DOWN_F8
-#define MOE_TC_PREFILL_AT_DOWN_F8 1
+#define MOE_TC_PREFILL_AT_DOWN_F8 2
 #endif
 #ifndef MOE_TC_PREFILL_CG
 #define MOE_TC_PREFILL_CG 2
