@@ -124,13 +124,37 @@ __device__ __forceinline__ void select_token(const SelectArgs &a, int t, float *
   const int E = a.E;
   const float NEG_INF = -INFINITY;
 
-  // z (split partials summed in split order), then s and c = s + b
+  // z (split partials summed in split order), then s and c = s + b.  With
+  // at most 8 experts per lane the lane's partial sums advance together, so
+  // that the loads of a split are in flight at once rather than one chain
+  // of dependent loads per expert; the order of the additions is the same.
   float zmax = NEG_INF;
-  for (int e = lane; e < E; e += 32) {
-    float z = 0.f;
-    for (int p = 0; p < a.nsplit; ++p) z += a.z_part[((size_t)p * a.T + t) * E + e];
-    s[e] = z;
-    zmax = fmaxf(zmax, z);
+  if (E <= 256) {
+    float z[8];
+#pragma unroll
+    for (int m = 0; m < 8; ++m) z[m] = 0.f;
+    const float *zt = a.z_part + (size_t)t * E;
+    const size_t pstride = (size_t)a.T * E;
+#pragma unroll 4
+    for (int p = 0; p < a.nsplit; ++p) {
+      const float *zp = zt + p * pstride;
+#pragma unroll
+      for (int m = 0; m < 8; ++m)
+        if (lane + 32 * m < E) z[m] += zp[lane + 32 * m];
+    }
+#pragma unroll
+    for (int m = 0; m < 8; ++m)
+      if (lane + 32 * m < E) {
+        s[lane + 32 * m] = z[m];
+        zmax = fmaxf(zmax, z[m]);
+      }
+  } else {
+    for (int e = lane; e < E; e += 32) {
+      float z = 0.f;
+      for (int p = 0; p < a.nsplit; ++p) z += a.z_part[((size_t)p * a.T + t) * E + e];
+      s[e] = z;
+      zmax = fmaxf(zmax, z);
+    }
   }
   if (a.softmax) {
     zmax = warp_max(zmax);
