@@ -117,44 +117,220 @@ struct SelectArgs {
   int softmax;
 };
 
-// Token t's selection by one warp; s and c are that warp's shared-memory
+// An unsigned key with the order of the float v (larger v, larger key; -0
+// taken as +0, as the float comparison does; no NaN), and back.
+__device__ __forceinline__ uint32_t order_key(float v) {
+  const uint32_t u = __float_as_uint(v + 0.0f);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+__device__ __forceinline__ float key_value(uint32_t k) {
+  return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
+}
+
+// warp_argmax on keys: the largest key, ties to the lowest index, in every
+// lane; two warp reductions instead of five shuffle rounds of two values.
+__device__ __forceinline__ void warp_argmax_key(uint32_t &key, int &i) {
+  const uint32_t mk = __reduce_max_sync(0xffffffffu, key);
+  i = (int)__reduce_min_sync(0xffffffffu, key == mk ? (uint32_t)i : 0xffffffffu);
+  key = mk;
+}
+
+// Token t's selection by one warp with at most 8 experts per lane (E <= 256),
+// each lane's scores in registers.  The same arithmetic, in the same order,
+// and the same decisions (ties to the lower index) as the general form
+// below; s is the warp's shared-memory row of E scores (for the gates).
+__device__ __forceinline__ void select_token_e256(const SelectArgs &a, int t, float *s) {
+  const int lane = threadIdx.x % 32;
+  const int E = a.E;
+  const float NEG_INF = -INFINITY;
+  const uint32_t KEY_NEG_INF = order_key(NEG_INF);
+
+  // z: split partials summed in split order, four splits' loads in flight
+  float z[8];
+#pragma unroll
+  for (int m = 0; m < 8; ++m) z[m] = 0.f;
+  {
+    const float *zt = a.z_part + (size_t)t * E;
+    const size_t ps = (size_t)a.T * E;
+    int p = 0;
+    for (; p + 4 <= a.nsplit; p += 4) {
+      float v[4][8];
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+#pragma unroll
+        for (int m = 0; m < 8; ++m)
+          v[q][m] = lane + 32 * m < E ? zt[(p + q) * ps + lane + 32 * m] : 0.f;
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+#pragma unroll
+        for (int m = 0; m < 8; ++m) z[m] += v[q][m];
+    }
+    for (; p < a.nsplit; ++p)
+#pragma unroll
+      for (int m = 0; m < 8; ++m)
+        if (lane + 32 * m < E) z[m] += zt[p * ps + lane + 32 * m];
+  }
+  // s = sigmoid(z) (or softmax), c = s + b
+  float sr[8], cr[8];
+  if (a.softmax) {
+    float zmax = NEG_INF;
+#pragma unroll
+    for (int m = 0; m < 8; ++m)
+      if (lane + 32 * m < E) zmax = fmaxf(zmax, z[m]);
+    zmax = warp_max(zmax);
+    float part = 0.f;
+#pragma unroll
+    for (int m = 0; m < 8; ++m)
+      if (lane + 32 * m < E) {
+        sr[m] = expf(z[m] - zmax);
+        part += sr[m];
+      }
+    const float tot = warp_sum(part);
+#pragma unroll
+    for (int m = 0; m < 8; ++m)
+      if (lane + 32 * m < E) sr[m] = sr[m] / tot;
+  } else {
+#pragma unroll
+    for (int m = 0; m < 8; ++m)
+      if (lane + 32 * m < E) sr[m] = 1.0f / (1.0f + expf(-z[m]));
+  }
+#pragma unroll
+  for (int m = 0; m < 8; ++m)
+    if (lane + 32 * m < E) {
+      const int e = lane + 32 * m;
+      cr[m] = a.bias ? sr[m] + a.bias[e] : sr[m];
+      s[e] = sr[m];
+    } else {
+      cr[m] = NEG_INF;
+    }
+
+  // group selection
+  const int P = E / a.G;
+  float gap = INFINITY;
+  uint32_t kept = 0xffffffffu;
+  if (a.G > 1) {
+    float gs = NEG_INF;  // lane q < G: the score of group q
+    if (P == 32) {
+      // group q is experts 32 q .. 32 q + 31: element q of every lane.  The
+      // largest and (with a bias) the second largest, one instance of the
+      // largest left out; their sum in that order
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        if (q >= a.G) break;
+        const uint32_t kq = order_key(cr[q]);
+        const uint32_t k1 = __reduce_max_sync(0xffffffffu, kq);
+        float g = key_value(k1);
+        if (a.bias) {
+          const uint32_t l1 = __reduce_min_sync(0xffffffffu, kq == k1 ? (uint32_t)lane : 32u);
+          const uint32_t k2 = __reduce_max_sync(0xffffffffu, lane == (int)l1 ? 0u : kq);
+          g = g + key_value(k2);
+        }
+        if (lane == q) gs = g;
+      }
+    } else {
+      // a lane per group scans its P experts (as the general form)
+      float *c = s + E;
+#pragma unroll
+      for (int m = 0; m < 8; ++m)
+        if (lane + 32 * m < E) c[lane + 32 * m] = cr[m];
+      __syncwarp();
+      if (lane < a.G) {
+        float m1 = NEG_INF, m2 = NEG_INF;
+        for (int i = 0; i < P; ++i) {
+          const float v = c[lane * P + i];
+          if (v > m1) {
+            m2 = m1;
+            m1 = v;
+          } else if (v > m2) {
+            m2 = v;
+          }
+        }
+        gs = a.bias ? m1 + m2 : m1;
+      }
+    }
+    kept = 0;
+    float prev = 0.f;
+    const int rounds = a.Gk < a.G ? a.Gk + 1 : a.Gk;
+    for (int r = 0; r < rounds; ++r) {
+      const bool open = lane < a.G && !((kept >> lane) & 1u);
+      uint32_t k = open ? order_key(gs) : KEY_NEG_INF;
+      int i = open ? lane : 0x7fffffff;
+      warp_argmax_key(k, i);
+      const float v = key_value(k);
+      if (r < a.Gk) {
+        kept |= 1u << i;
+        prev = v;
+      } else {
+        gap = fminf(gap, prev - v);  // last kept group minus best dropped group
+      }
+    }
+  }
+
+  // expert selection over the kept groups: k arg-max rounds plus one for
+  // the first expert left out
+  uint32_t ck[8];  // keys of the candidates (-inf outside the kept groups)
+#pragma unroll
+  for (int m = 0; m < 8; ++m) {
+    const int e = lane + 32 * m;
+    ck[m] = e < E && ((kept >> (e / P)) & 1u) ? order_key(cr[m]) : KEY_NEG_INF;
+  }
+  uint32_t taken = 0;  // bit m: expert lane + 32 m already chosen
+  float prev_v = 0.f;
+  int chosen_i = 0;
+  const int rounds = a.k < E ? a.k + 1 : a.k;
+  for (int r = 0; r < rounds; ++r) {
+    uint32_t k = KEY_NEG_INF;
+    int i = 0x7fffffff;
+#pragma unroll
+    for (int m = 0; m < 8; ++m) {
+      const int e = lane + 32 * m;
+      if (e >= E || ((taken >> m) & 1u)) continue;
+      if (ck[m] > k || (ck[m] == k && e < i)) {
+        k = ck[m];
+        i = e;
+      }
+    }
+    warp_argmax_key(k, i);
+    const float v = key_value(k);
+    if (r < a.k) {
+      if (i % 32 == lane) taken |= 1u << (i / 32);
+      if (r > 0) gap = fminf(gap, prev_v - v);  // consecutive chosen experts
+      prev_v = v;
+      if (lane == r) chosen_i = i;
+    } else {
+      gap = fminf(gap, prev_v - v);  // k-th chosen minus first left out
+    }
+  }
+  __syncwarp();
+
+  // gates: unbiased scores of the chosen experts, summed in choice order
+  float w = (lane < a.k) ? s[chosen_i] : 0.f;
+  float tot = 0.f;
+  for (int j = 0; j < a.k; ++j) tot += __shfl_sync(0xffffffffu, w, j);
+  if (lane < a.k) {
+    if (!a.softmax) w = w / tot;
+    w = w * a.route_scale;
+    a.weights[(size_t)t * a.k + lane] = w;
+    a.indices[(size_t)t * a.k + lane] = chosen_i;
+  }
+  if (a.sel_gap && lane == 0) a.sel_gap[t] = gap;
+}
+
+// The general form (any E up to 1024): s and c are the warp's shared-memory
 // rows of E floats (the scores and the biased scores).
-__device__ __forceinline__ void select_token(const SelectArgs &a, int t, float *s, float *c) {
+__device__ __forceinline__ void select_token_general(const SelectArgs &a, int t, float *s,
+                                                     float *c) {
   const int lane = threadIdx.x % 32;
   const int E = a.E;
   const float NEG_INF = -INFINITY;
 
-  // z (split partials summed in split order), then s and c = s + b.  With
-  // at most 8 experts per lane the lane's partial sums advance together, so
-  // that the loads of a split are in flight at once rather than one chain
-  // of dependent loads per expert; the order of the additions is the same.
+  // z (split partials summed in split order), then s and c = s + b
   float zmax = NEG_INF;
-  if (E <= 256) {
-    float z[8];
-#pragma unroll
-    for (int m = 0; m < 8; ++m) z[m] = 0.f;
-    const float *zt = a.z_part + (size_t)t * E;
-    const size_t pstride = (size_t)a.T * E;
-#pragma unroll 4
-    for (int p = 0; p < a.nsplit; ++p) {
-      const float *zp = zt + p * pstride;
-#pragma unroll
-      for (int m = 0; m < 8; ++m)
-        if (lane + 32 * m < E) z[m] += zp[lane + 32 * m];
-    }
-#pragma unroll
-    for (int m = 0; m < 8; ++m)
-      if (lane + 32 * m < E) {
-        s[lane + 32 * m] = z[m];
-        zmax = fmaxf(zmax, z[m]);
-      }
-  } else {
-    for (int e = lane; e < E; e += 32) {
-      float z = 0.f;
-      for (int p = 0; p < a.nsplit; ++p) z += a.z_part[((size_t)p * a.T + t) * E + e];
-      s[e] = z;
-      zmax = fmaxf(zmax, z);
-    }
+  for (int e = lane; e < E; e += 32) {
+    float z = 0.f;
+    for (int p = 0; p < a.nsplit; ++p) z += a.z_part[((size_t)p * a.T + t) * E + e];
+    s[e] = z;
+    zmax = fmaxf(zmax, z);
   }
   if (a.softmax) {
     zmax = warp_max(zmax);
@@ -247,6 +423,15 @@ __device__ __forceinline__ void select_token(const SelectArgs &a, int t, float *
     a.indices[(size_t)t * a.k + lane] = chosen_i;
   }
   if (a.sel_gap && lane == 0) a.sel_gap[t] = gap;
+}
+
+// Token t's selection by one warp; s and c are that warp's shared-memory
+// rows of E floats.
+__device__ __forceinline__ void select_token(const SelectArgs &a, int t, float *s, float *c) {
+  if (a.E <= 256)
+    select_token_e256(a, t, s);
+  else
+    select_token_general(a, t, s, c);
 }
 
 }  // namespace route
