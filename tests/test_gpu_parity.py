@@ -41,6 +41,13 @@ ROUTER_TC_SPLIT = custom("router_tc_split", 40, dim=2048, n_routed=256, n_groups
 # dim % 256 != 0: the prefill path falls back to one SM per tile
 CG1_PREFILL = custom("cg1_prefill", 230, dim=384, n_routed=16, n_groups=4, topk_groups=2, topk=4,
                      inter=128, seed=22)
+# more than 256 experts: the selection's general form (scores in shared
+# memory), and 384 experts in groups of 48
+ROUTER_E512 = custom("router_e512", 120, dim=512, n_routed=512, n_groups=8, topk_groups=4,
+                     topk=8, inter=128, seed=29)
+ROUTER_E384 = custom("router_e384", 90, dim=256, n_routed=384, n_groups=8, topk_groups=3,
+                     topk=6, inter=128, seed=30, score_func="softmax", has_bias=False,
+                     route_scale=1.0)
 # dim % 512 == 256: the second matmul's SM pairs keep one weight tile per SM
 PAIR_AT1 = custom("pair_at1", 300, dim=768, n_routed=32, n_groups=4, topk_groups=2, topk=8,
                   inter=256, seed=27)
@@ -88,7 +95,8 @@ def run_block(w, x, params, combine="scatter"):
 
 
 @pytest.mark.parametrize("w", [WORKLOADS["tiny_f32"], TINY_BF16, MID, MID_F32, SOFTMAX_NOBIAS,
-                               NOBIAS_SIGMOID, ONE_GROUP, ROUTER_TC, ROUTER_TC_SPLIT],
+                               NOBIAS_SIGMOID, ONE_GROUP, ROUTER_TC, ROUTER_TC_SPLIT,
+                               ROUTER_E512, ROUTER_E384],
                          ids=lambda w: w.name)
 def test_router_matches_oracle(w):
     x, p = make_block(w)
