@@ -48,10 +48,12 @@ __global__ void __launch_bounds__(1024) dispatch_scan(int32_t *__restrict__ chun
 __global__ void __launch_bounds__(32) dispatch_scatter(const int32_t *__restrict__ idx, int T,
                                                        int k, int E,
                                                        const int32_t *__restrict__ chunk_base,
+                                                       const int32_t *__restrict__ offsets,
                                                        int32_t *__restrict__ sorted_token,
                                                        int32_t *__restrict__ slot_of) {
   extern __shared__ int32_t base[];
-  grouping::scatter_chunk(idx, T, k, E, blockIdx.x, chunk_base, sorted_token, slot_of, base);
+  grouping::scatter_chunk(idx, T, k, E, blockIdx.x, chunk_base, offsets, sorted_token, slot_of,
+                          base);
 }
 
 // ------------------------------------------------- no-allocation variant
@@ -150,8 +152,8 @@ MOE_EXPORT moe_status moe_dispatch_build(const moe_cfg *cfg, int64_t T, const in
   dispatch_scan<<<1, scan_threads, 0, s>>>(chunk_hist, nchunks, E, counts, offsets);
   if ((st = launch_status()) != MOE_OK) return st;
   if (nchunks > 0) {
-    dispatch_scatter<<<nchunks, 32, hsmem, s>>>(indices, (int)T, k, E, chunk_hist, sorted_token,
-                                                slot_of);
+    dispatch_scatter<<<nchunks, 32, hsmem, s>>>(indices, (int)T, k, E, chunk_hist, offsets,
+                                                sorted_token, slot_of);
     if ((st = launch_status()) != MOE_OK) return st;
   }
   return MOE_OK;

@@ -36,16 +36,29 @@ __device__ __forceinline__ void hist_chunk(const int32_t *__restrict__ idx, int 
   for (int e = threadIdx.x; e < E; e += blockDim.x) chunk_hist[(size_t)chunk * E + e] = h[e];
 }
 
-// Per expert, an exclusive scan over the chunks, then over the experts: counts,
-// offsets, and each chunk's first row for each expert in chunk_hist.  One
-// block of >= E threads (E <= 1024); warp_tot is shared memory of 32 ints.
+// Per expert, an exclusive scan over the chunks (each chunk's first row
+// within the expert's rows, left in chunk_hist), then over the experts:
+// counts and offsets.  One block of >= E threads (E <= 1024); warp_tot is
+// shared memory of 32 ints.
 __device__ __forceinline__ void scan_chunks(int32_t *__restrict__ chunk_hist, int nchunks, int E,
                                             int32_t *__restrict__ counts,
                                             int32_t *__restrict__ offsets, int32_t *warp_tot) {
   const int e = threadIdx.x;
   int run = 0;
   if (e < E) {
-    for (int c = 0; c < nchunks; ++c) {
+    // eight chunks' loads in flight before their stores
+    int c = 0;
+    for (; c + 8 <= nchunks; c += 8) {
+      int v[8];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) v[q] = chunk_hist[(size_t)(c + q) * E + e];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        chunk_hist[(size_t)(c + q) * E + e] = run;
+        run += v[q];
+      }
+    }
+    for (; c < nchunks; ++c) {
       const int v = chunk_hist[(size_t)c * E + e];
       chunk_hist[(size_t)c * E + e] = run;
       run += v;
@@ -79,40 +92,52 @@ __device__ __forceinline__ void scan_chunks(int32_t *__restrict__ chunk_hist, in
   if (e < E) {
     offsets[e] = excl;
     if (e == E - 1) offsets[E] = excl + v;
-    for (int c = 0; c < nchunks; ++c) chunk_hist[(size_t)c * E + e] += excl;
   }
 }
 
-// The stable scatter of chunk `chunk` by one warp; base is that warp's shared
-// memory of E ints.
+// The stable scatter of chunk `chunk` by one warp: chunk_base holds each
+// chunk's first row within each expert, offsets each expert's first row;
+// base is that warp's shared memory of E ints.
 __device__ __forceinline__ void scatter_chunk(const int32_t *__restrict__ idx, int T, int k, int E,
                                               int chunk, const int32_t *__restrict__ chunk_base,
+                                              const int32_t *__restrict__ offsets,
                                               int32_t *__restrict__ sorted_token,
                                               int32_t *__restrict__ slot_of, int32_t *base) {
   const int lane = threadIdx.x % 32;
-  for (int e = lane; e < E; e += 32) base[e] = chunk_base[(size_t)chunk * E + e];
+  for (int e = lane; e < E; e += 32) base[e] = chunk_base[(size_t)chunk * E + e] + offsets[e];
   __syncwarp();
   const int t0 = chunk * CHUNK_TOKENS;
   const int n = min(CHUNK_TOKENS, T - t0) * k;
   const size_t flat0 = (size_t)t0 * k;
   const unsigned lt = (1u << lane) - 1u;
-  for (int i0 = 0; i0 < n; i0 += 32) {
-    const int i = i0 + lane;
-    int e = -1;
-    if (i < n) e = idx[flat0 + i];
-    const bool ok = i < n && e >= 0 && e < E;
-    const int key = ok ? e : -1 - lane;  // invalid lanes get a key of their own
-    const unsigned same = __match_any_sync(0xffffffffu, key);
-    if (ok) {
-      const int rank = __popc(same & lt);
-      const int pos = base[e] + rank;
-      sorted_token[pos] = t0 + i / k;
-      slot_of[flat0 + i] = pos;
+  // the indices of eight rounds of 32 slots are loaded before the rounds run
+  for (int i00 = 0; i00 < n; i00 += 256) {
+    int ev[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int i = i00 + 32 * j + lane;
+      ev[j] = i < n ? idx[flat0 + i] : -1;
     }
-    __syncwarp();
-    // the highest lane of each group advances that expert's next free row
-    if (ok && (same >> lane) == 1u) base[e] += __popc(same);
-    __syncwarp();
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int i0 = i00 + 32 * j;
+      if (i0 >= n) break;
+      const int i = i0 + lane;
+      const int e = ev[j];
+      const bool ok = i < n && e >= 0 && e < E;
+      const int key = ok ? e : -1 - lane;  // invalid lanes get a key of their own
+      const unsigned same = __match_any_sync(0xffffffffu, key);
+      if (ok) {
+        const int rank = __popc(same & lt);
+        const int pos = base[e] + rank;
+        sorted_token[pos] = t0 + i / k;
+        slot_of[flat0 + i] = pos;
+      }
+      __syncwarp();
+      // the highest lane of each group advances that expert's next free row
+      if (ok && (same >> lane) == 1u) base[e] += __popc(same);
+      __syncwarp();
+    }
   }
 }
 

@@ -1728,8 +1728,8 @@ __global__ void __launch_bounds__(THREADS, 1)
     __syncthreads();
     if (warp == 0)
       for (int c = 0; c < a.nchunks; ++c)
-        grouping::scatter_chunk(a.sel.indices, T, a.k, E, c, a.chunk_hist, a.sorted_token,
-                                a.slot_of, base);
+        grouping::scatter_chunk(a.sel.indices, T, a.k, E, c, a.chunk_hist, a.offsets,
+                                a.sorted_token, a.slot_of, base);
     __syncthreads();
     if (warp == 1) prep_tiles_warp(a.offsets, E, a.G, a.sh, a.t1, a.t2);
   }
