@@ -52,7 +52,8 @@ def built():
     build.build_all()
 
 
-@pytest.mark.parametrize("rows,K", [(1, 128), (33, 512), (300, 2048), (97, 7168), (5, 36)])
+@pytest.mark.parametrize("rows,K", [(1, 128), (33, 512), (300, 2048), (97, 7168), (5, 36),
+                                   (3, 2056), (4, 8)])
 def test_quantiser_is_bit_exact(rows, K):
     g = torch.Generator(device="cuda").manual_seed(rows + K)
     # magnitudes spread over many binades, an all-zero row, a row with a
