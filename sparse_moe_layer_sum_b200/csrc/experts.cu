@@ -27,7 +27,18 @@
 // holds 128 rows of W1 and the same 128 rows of W3 in two accumulators (AT =
 // 2), so a thread holds both SwiGLU halves of its feature; at decode a
 // 128-row tile holds 64 rows of each and the epilogue pairs the warps that
-// hold them (AT = 1).
+// hold them (AT = 1).  In the second matmul each SM of a pair holds two
+// 128-row blocks of W2 (AT = 2), whose single accumulator the epilogue reads
+// in register batches and hands back before its last stores; the weighted
+// scatter adds 16-byte vectors into y after a 4 x 4 transpose in each quad
+// of lanes.
+//
+// FP8 x FP8 path (e4m3 weights and activations, act_e4m3): quant_rows_e4m3
+// quantises the expert rows of x and later h (one scale per row), and
+// tc_fp8_gemm runs both matmuls as e4m3 x e4m3 MMAs whose per-k-block partial
+// sums eight promotion warps scale by the weight block's scale and add in
+// fp32 registers; two helper warps build the scatter's gate lists and finish
+// half of each tile's sums from shared memory.
 //
 // CUDA-core path: any other dtype combination (the fp32 configuration) runs
 // on simt_gemm1 / simt_gemm2 in fp32.
